@@ -1,0 +1,126 @@
+"""The fine-grained block-scaled FP8 NT GEMM and its MoE grouped forms.
+
+Lesson 13, Fig. 13-1: for A [M, K] with 1x128 scales alpha and B with 128x128
+scales beta,
+
+    C[i, j] = sum_g alpha[i, g] * beta[g, floor(j / 128)]
+                    * sum_{k < 128} A[i, 128 g + k] * B[128 g + k, j].
+
+The page writes B as K x N; the exercise (Lesson 13 practice task) and the NT
+convention (Deep dive, section 3: ``fp8_gemm_nt`` computes A @ B.T) store it as
+[N, K], which is what is used here: B[128 g + k, j] above is ``qb[j, 128 g + k]``.
+
+The oracle follows the exercise's order: for each 128-wide K block, the block's
+partial product of the decoded codes (a float64 matmul), times the outer
+product of the block's scales, added into a float64 accumulator.  Then the
+result is rounded once to BF16 (Lesson 13, Fig. 13-1: the epilogue only
+converts and writes back).
+
+Grouped forms (Lesson 13, Fig. 13-3 and the answer to Q3; Deep dive,
+section 3, the grouped GEMM table):
+
+* m-grouped contiguous: the tokens of all experts are concatenated along M;
+  each expert segment is aligned to the M tile; a per-row expert index names
+  the expert, -1 on padding rows; N and K are shared by all experts.
+* m-grouped masked: A is [G, M_max, K]; masked_m[g] rows of expert g are
+  valid; only those rows are computed.
+
+Rows that are not computed (padding, rows >= masked_m[g]) are left exactly as
+they were in the output (reading stated in the design doc); the oracle copies the
+caller's initial output for them.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from . import bf16, e4m3
+
+GROUP = 128
+
+
+def fp8_gemm_nt_f64(qa: np.ndarray, alpha: np.ndarray,
+                    qb: np.ndarray, beta: np.ndarray) -> np.ndarray:
+    """float64 D [M, N] of the Fig. 13-1 formula.
+
+    qa uint8 [M, K] E4M3 codes, alpha float32 [M, K/128];
+    qb uint8 [N, K] E4M3 codes, beta float32 [ceil(N/128), K/128].
+    """
+    M, K = qa.shape
+    N, Kb = qb.shape
+    if K != Kb or K % GROUP:
+        raise ValueError("K mismatch or K not a multiple of 128")
+    kg = K // GROUP
+    if alpha.shape != (M, kg) or beta.shape != (-(-N // GROUP), kg):
+        raise ValueError("scale shapes do not match the 1x128 / 128x128 grids")
+    n_block_of_col = np.arange(N) // GROUP
+    a_vals = e4m3.decode(qa)
+    b_vals = e4m3.decode(qb)
+    alpha64 = np.asarray(alpha, np.float64)
+    beta64 = np.asarray(beta, np.float64)
+    d = np.zeros((M, N), dtype=np.float64)
+    for g in range(kg):
+        ks = slice(g * GROUP, (g + 1) * GROUP)
+        partial = a_vals[:, ks] @ b_vals[:, ks].T  # exact: small integers x 2^k
+        scale = alpha64[:, g][:, None] * beta64[n_block_of_col, g][None, :]
+        d += partial * scale
+    return d
+
+
+def fp8_gemm_nt(qa, alpha, qb, beta) -> np.ndarray:
+    """BF16 bit patterns (uint16 [M, N]) of the dense NT GEMM."""
+    return bf16.to_bits(fp8_gemm_nt_f64(qa, alpha, qb, beta))
+
+
+def m_grouped_contiguous_f64(qa, alpha, qb, beta, m_indices, d_init):
+    """Contiguous m-grouped GEMM in float64.
+
+    qa [M_total, K], alpha [M_total, K/128]; qb [G, N, K], beta
+    [G, ceil(N/128), K/128]; m_indices int [M_total] (expert of each row, -1 =
+    padding); d_init float64 [M_total, N]: returned unchanged on padding rows.
+    """
+    m_indices = np.asarray(m_indices)
+    d = np.array(d_init, dtype=np.float64, copy=True)
+    for e in np.unique(m_indices[m_indices >= 0]):
+        rows = np.nonzero(m_indices == e)[0]
+        d[rows] = fp8_gemm_nt_f64(qa[rows], alpha[rows], qb[e], beta[e])
+    return d
+
+
+def m_grouped_contiguous(qa, alpha, qb, beta, m_indices, d_init_bits):
+    """BF16 bits of the contiguous form; padding rows keep ``d_init_bits``."""
+    m_indices = np.asarray(m_indices)
+    out = np.array(d_init_bits, dtype=np.uint16, copy=True)
+    d = m_grouped_contiguous_f64(qa, alpha, qb, beta, m_indices,
+                                 np.zeros(out.shape))
+    valid = m_indices >= 0
+    out[valid] = bf16.to_bits(d[valid])
+    return out
+
+
+def m_grouped_masked_f64(qa, alpha, qb, beta, masked_m, d_init):
+    """Masked m-grouped GEMM in float64.
+
+    qa [G, M_max, K], alpha [G, M_max, K/128]; qb [G, N, K], beta
+    [G, ceil(N/128), K/128]; masked_m int [G]; d_init [G, M_max, N]: rows
+    >= masked_m[g] are returned unchanged.  A masked_m outside [0, M_max] is
+    clamped into that range.
+    """
+    d = np.array(d_init, dtype=np.float64, copy=True)
+    G, m_max, _ = qa.shape
+    for e in range(G):
+        m = int(min(max(int(masked_m[e]), 0), m_max))
+        if m:
+            d[e, :m] = fp8_gemm_nt_f64(qa[e, :m], alpha[e, :m], qb[e], beta[e])
+    return d
+
+
+def m_grouped_masked(qa, alpha, qb, beta, masked_m, d_init_bits):
+    """BF16 bits of the masked form; rows >= masked_m keep ``d_init_bits``."""
+    out = np.array(d_init_bits, dtype=np.uint16, copy=True)
+    G, m_max, _ = qa.shape
+    for e in range(G):
+        m = int(min(max(int(masked_m[e]), 0), m_max))
+        if m:
+            out[e, :m] = fp8_gemm_nt(qa[e, :m], alpha[e, :m], qb[e], beta[e])
+    return out
