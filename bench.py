@@ -1,0 +1,458 @@
+"""Benchmark of the fine-grained block-scaled FP8 GEMM hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload W]
+                    [--impl reference]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+for every (N, K) pair of the workload, quantize the FP32 activations A with the
+1x128 quantizer kernel, then run the FP8 GEMM against the pre-quantized
+(128x128) weights B.  Weights are quantized once before timing (they are
+offline-quantized model parameters).  The default workload is the dense
+prefill set: M = 4096 and (N, K) in {(7168, 16384), (4096, 7168),
+(24576, 1536), (2112, 7168)}.
+
+Reported (one JSON line on rank 0):
+* value       whole-job TFLOP/s (2 M N K per GEMM, summed over shapes and
+              ranks) with inputs resident in HBM, CUDA events on the launch
+              stream, max over ranks;
+* e2e         the same metric through the public API with pinned host buffers:
+              host->device copy of A, B and scales, quantize, GEMM, and the
+              device->host copy of D, all inside the timed region;
+* roofline    the GEMM kernel's achieved TFLOP/s (or GB/s for the memory-bound
+              workloads) over the measured peak;
+* cpu_baseline the CPU oracle timed on a bounded row sample of the same work.
+
+With --gpus N > 1 (launched by torch.distributed.run) every rank runs an
+independent replica of the workload on its own GPU (the method has no
+cross-GPU exchange): scaling is weak and the only collectives are the timing
+barrier and the max-over-ranks reduction.
+
+``--impl reference`` times the CPU oracle (the reference of this library) on
+the host cores instead, one bounded row sample per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from moe_grouped_gemm_act_b200 import inputs  # noqa: E402
+
+METRIC = "FP8 block-scaled GEMM TFLOPS & % of B200 FP8 peak / HBM roofline, per shape"
+FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
+
+
+# ---------------------------------------------------------------- workloads
+def workload_spec(name: str) -> dict:
+    if name == "prefill":
+        return dict(name=name, kind="dense", m=inputs.PREFILL_M, nk=inputs.PREFILL_NK,
+                    seeds=inputs.PREFILL_SEEDS, bound="tensor",
+                    desc="dense NT prefill, M=4096, (N,K) in "
+                         "{(7168,16384),(4096,7168),(24576,1536),(2112,7168)}; "
+                         "A~N(0,1) with 0.1% x50 outliers, B~N(0,0.02); "
+                         "1x128 / 128x128 FP32 scales, BF16 out")
+    if name in ("decode64", "decode128"):
+        m = 64 if name == "decode64" else 128
+        return dict(name=name, kind="dense", m=m, nk=inputs.PREFILL_NK,
+                    seeds=inputs.DECODE_SEEDS, bound="hbm",
+                    desc=f"dense NT decode, M={m}, same four (N,K) pairs")
+    if name == "contiguous":
+        return dict(name=name, kind="contiguous", bound="tensor", **inputs.CONTIGUOUS,
+                    desc="m-grouped contiguous, G=8, N=4096 K=7168, 32768 tokens "
+                         "multinomial over experts, segments padded to 128")
+    if name == "masked":
+        return dict(name=name, kind="masked", bound="hbm", **inputs.MASKED,
+                    desc="m-grouped masked, G=32, M_max=256, N=7168 K=2048, "
+                         "masked_m ~ U{0..256}")
+    raise SystemExit(f"unknown workload {name}")
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- device data
+class DenseData:
+    def __init__(self, spec, device):
+        import torch
+        import moe_grouped_gemm_act_b200 as dg
+        self.dg = dg
+        m = spec["m"]
+        self.m = m
+        self.shapes = []
+        for n, k in spec["nk"]:
+            x = inputs.activations(m, k, seed=spec["seeds"]["seed_a"] + k, outliers=True)
+            w = inputs.weights((n, k), seed=spec["seeds"]["seed_b"] + n + k)
+            a32 = torch.from_numpy(x).to(device)
+            qb, sfb = dg.dg_quantize_128x128(torch.from_numpy(w).to(device))
+            ld = dg.dg_get_tma_aligned_size(m, 4)
+            qa = torch.empty((m, k), dtype=torch.uint8, device=device)
+            sfa = torch.empty((k // 128, ld), dtype=torch.float32, device=device)
+            d = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+            wsb = dg.dg_fp8_gemm_nt_workspace_size(m, n, k)
+            ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=device) if wsb else None
+            self.shapes.append(dict(n=n, k=k, a32=a32, qb=qb, sfb=sfb, qa=qa, sfa=sfa, d=d,
+                                    ws=ws, x_host=x, w_host=w))
+        torch.cuda.synchronize()
+
+    def flops(self) -> float:
+        return sum(2.0 * self.m * s["n"] * s["k"] for s in self.shapes)
+
+    def gemm_bytes(self) -> float:
+        """Algorithmic bytes of the GEMM launches (A, alpha, B, beta, D)."""
+        tot = 0.0
+        for s in self.shapes:
+            n, k = s["n"], s["k"]
+            tot += self.m * k + 4 * self.m * (k // 128) + n * k + \
+                4 * (-(-n // 128)) * (k // 128) + 2 * self.m * n
+        return tot
+
+    def step(self, gemm_events=None):
+        dg = self.dg
+        for i, s in enumerate(self.shapes):
+            dg.dg_quantize_1x128(s["a32"], q=s["qa"], sf=s["sfa"])
+            if gemm_events is not None:
+                gemm_events[i][0].record()
+            dg.dg_fp8_gemm_nt(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"], workspace=s["ws"])
+            if gemm_events is not None:
+                gemm_events[i][1].record()
+
+    def launches_per_step(self) -> int:
+        return 2 * len(self.shapes)
+
+    # end-to-end through the public API from pinned host buffers
+    def make_host(self):
+        import torch
+        self.host = []
+        for s in self.shapes:
+            self.host.append(dict(
+                a=torch.from_numpy(s["x_host"]).pin_memory(),
+                qb=s["qb"].cpu().pin_memory(), sfb=s["sfb"].cpu().pin_memory(),
+                d=torch.empty(s["d"].shape, dtype=torch.bfloat16).pin_memory()))
+        self.h2d = sum(h["a"].numel() * 4 + h["qb"].numel() + h["sfb"].numel() * 4
+                       for h in self.host)
+        self.d2h = sum(h["d"].numel() * 2 for h in self.host)
+
+    def e2e_step(self, device):
+        dg = self.dg
+        for s, h in zip(self.shapes, self.host):
+            a = h["a"].to(device, non_blocking=True)
+            qb = h["qb"].to(device, non_blocking=True)
+            sfb = h["sfb"].to(device, non_blocking=True)
+            qa, sfa = dg.dg_quantize_1x128(a)
+            dg.dg_fp8_gemm_nt(qa, sfa, qb, sfb, s["d"], workspace=s["ws"])
+            h["d"].copy_(s["d"], non_blocking=True)
+
+
+class OracleSample:
+    """The CPU oracle on a bounded sample of the workload: for every (N, K)
+    pair, the first ``rows`` rows of A and the first ``cols`` columns of D over
+    the full K.  One run = quantize the sampled A rows (1x128) and compute the
+    sampled block of every GEMM.  Weights are quantized once beforehand, as on
+    the GPU (the first 128-aligned rows of B quantize exactly as in full)."""
+
+    def __init__(self, spec, rows: int, cols: int):
+        from oracle import quant as oq
+        self.prepared = []
+        for n, k in spec["nk"]:
+            x = inputs.activations(spec["m"], k, seed=spec["seeds"]["seed_a"] + k,
+                                   outliers=True)
+            w = inputs.weights((n, k), seed=spec["seeds"]["seed_b"] + n + k)
+            c = min(n, cols)
+            qb, beta = oq.quantize_128x128(w[:c])
+            self.prepared.append((x[:rows].copy(), qb, beta, c, k))
+        self.desc = (f"{rows} rows of A x first {cols} columns of D per (N,K) pair, "
+                     f"full K")
+
+    def run(self) -> tuple[float, float]:
+        """Returns (seconds, FLOPs) of one pass."""
+        from oracle import gemm as og, quant as oq
+        t0 = time.perf_counter()
+        flops = 0.0
+        for xs, qb, beta, c, k in self.prepared:
+            qa, alpha = oq.quantize_1x128(xs)
+            og.fp8_gemm_nt(qa, alpha, qb, beta)
+            flops += 2.0 * xs.shape[0] * c * k
+        return time.perf_counter() - t0, flops
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(int(i.get("num_threads", 1)) for i in info)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args, rank: int) -> None:
+    """The oracle arm: rank 0 times the CPU oracle on bounded samples."""
+    if rank != 0:
+        return
+    spec = workload_spec(args.workload)
+    if spec["kind"] != "dense":
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "reference arm implemented for the dense workloads only"}))
+        return
+    sampler = OracleSample(spec, args.ref_rows, args.ref_cols)
+    for _ in range(args.warmup):
+        sampler.run()
+    secs, flops = 0.0, 0.0
+    for _ in range(args.steps):
+        s, f = sampler.run()
+        secs += s
+        flops += f
+    value = flops / secs / 1e12
+    cores = blas_threads()
+    sample = sampler.desc
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec["desc"], "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import moe_grouped_gemm_act_b200 as dg
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dg.load_library()
+    spec = workload_spec(args.workload)
+    if spec["kind"] != "dense":
+        raise SystemExit("the GPU arm of bench.py times the dense workloads; "
+                         "grouped layouts are covered by bench_grouped in the tests")
+    data = DenseData(spec, device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ------------------------------------------------ device-resident timing
+    for _ in range(args.warmup):
+        data.step()
+    nshape = len(data.shapes)
+    gemm_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(nshape)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local_rank) as clocks:
+        start.record()
+        for i in range(args.steps):
+            data.step(gemm_ev[i])
+        stop.record()
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = start.elapsed_time(stop)
+    gemm_ms = [sum(e0.elapsed_time(e1) for e0, e1 in gemm_ev[i]) for i in range(args.steps)]
+    per_shape_ms = [statistics.mean(gemm_ev[i][j][0].elapsed_time(gemm_ev[i][j][1])
+                                    for i in range(args.steps)) for j in range(nshape)]
+
+    # ------------------------------------------------ end-to-end timing
+    data.make_host()
+    for _ in range(max(1, args.warmup // 2)):
+        data.e2e_step(device)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        data.e2e_step(device)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    # ------------------------------------------------ max over ranks
+    t = torch.tensor([total_ms, e2e_ms, sum(gemm_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms, gemm_total_ms = t.tolist()
+    if rank != 0:
+        return
+
+    flops_step = data.flops()
+    value = flops_step * args.steps * world / (total_ms * 1e-3) / 1e12
+    e2e = flops_step * args.steps * world / (e2e_ms * 1e-3) / 1e12
+    pk = peaks()
+    # dominant kernel: the GEMM
+    if spec["bound"] == "tensor":
+        achieved = flops_step * args.steps / (gemm_total_ms * 1e-3) / 1e12
+        peak = pk["bf16"] * FP8_OVER_BF16
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                "peak_source": f"{pk['source']} bf16 burst x {FP8_OVER_BF16} (nominal FP8/BF16)"}
+    else:
+        achieved = data.gemm_bytes() * args.steps / (gemm_total_ms * 1e-3) / 1e9
+        peak = pk["hbm"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"{pk['source']} copy bandwidth"}
+    roof["traffic"] = args.traffic
+    per_shape = [{"n": s["n"], "k": s["k"], "gemm_us": 1e3 * ms,
+                  "tflops": 2.0 * data.m * s["n"] * s["k"] / (ms * 1e-3) / 1e12}
+                 for s, ms in zip(data.shapes, per_shape_ms)]
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        sampler = OracleSample(spec, args.ref_rows, args.ref_cols)
+        sampler.run()
+        secs, fl = 0.0, 0.0
+        while secs < 10.0:          # about 10 s of CPU work
+            s_, f_ = sampler.run()
+            secs += s_
+            fl += f_
+        cpu = {"value": fl / secs / 1e12, "unit": "TFLOPS", "cores": blas_threads(),
+               "kind": "oracle", "sample": f"{sampler.desc} ({secs:.1f} s on the host)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": spec["desc"], "m": data.m,
+                   "nk": [[s["n"], s["k"]] for s in data.shapes],
+                   "l2": "not flushed: each step streams %.0f MB of inputs (> 126 MB L2)"
+                         % ((sum(s["a32"].numel() * 4 + s["qb"].numel() for s in data.shapes))
+                            / 1e6),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "per_shape": per_shape},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e, "unit": "TFLOPS", "h2d_bytes_per_step": data.h2d,
+                "d2h_bytes_per_step": data.d2h},
+        "gpu_launches": data.launches_per_step() * args.steps,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill",
+                    choices=["prefill", "decode64", "decode128"])
+    ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=16,
+                    help="rows of A per shape in the oracle's timed sample")
+    ap.add_argument("--ref-cols", type=int, default=1024,
+                    help="columns of D per shape in the oracle's timed sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu DRAM bytes per GEMM launch, when measured for this build")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

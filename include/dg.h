@@ -1,0 +1,228 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) fine-grained block-scaled FP8 GEMM
+ * library (libdg.so).
+ *
+ * What is computed (sources named by page title and figure/section):
+ *
+ *   "Lesson 13: DeepSeek DeepGEMM core architecture and Hopper FP8 kernel
+ *   breakdown" (hpc.payai.win), Fig. 13-1:
+ *       D[i, j] = sum_g alpha[i, g] * beta[g, j / 128]
+ *                       * sum_{k < 128} A[i, 128 g + k] * B[j, 128 g + k]
+ *   with A, B in E4M3, alpha one FP32 scale per row per 128-wide K group
+ *   (alpha = max|group| / 448), beta one FP32 scale per 128 x 128 block of B,
+ *   each 128-K block's partial product scaled and promoted into an FP32
+ *   accumulator inside the main loop, and D written as BF16.
+ *
+ *   "DeepGEMM architecture deep dive" (blog.123qwe.co.kr), section 3: NT
+ *   layout (A row-major [M, K], B row-major [N, K], D = A * B^T), LHS scales
+ *   stored transposed (MN-major) and TMA-aligned, contiguous grouped layout
+ *   with expert segments aligned to the M block, masked grouped layout with a
+ *   per-expert valid row count.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument marked "device" must point to device memory of
+ *     the current CUDA device; the caller owns all buffers and the stream.
+ *   - All calls are asynchronous on `stream` (NULL = the legacy default
+ *     stream) unless stated otherwise; none allocates device memory.
+ *   - The return value is a dg_status code.  Argument errors are detected on
+ *     the host before anything is launched and leave outputs untouched.
+ *     Errors found by a kernel on the device (bad expert index, masked_m out
+ *     of range, a pipeline wait that timed out) are recorded in a device
+ *     status word read by dg_get_device_status().
+ *   - The library keeps a small amount of per-device state (device
+ *     properties, the device status word), created by the first call on that
+ *     device.  Make one call before capturing any call into a CUDA graph.
+ *   - E4M3 here is the FN variant: max 448, no infinities, 0x7F/0xFF NaN.
+ *   - BF16 outputs are round-to-nearest-even.
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (CUstream); NULL selects the legacy default stream. */
+typedef struct CUstream_st *dg_stream_t;
+
+/* Status codes. */
+#define DG_OK 0
+#define DG_ERR_INVALID_ARG -1      /* bad shape, null pointer, bad flag       */
+#define DG_ERR_ALIGNMENT -2        /* pointer or leading dim not 16-B aligned */
+#define DG_ERR_UNSUPPORTED_ARCH -3 /* current device is not sm_100            */
+#define DG_ERR_CUDA -4             /* a CUDA runtime/driver call failed        */
+#define DG_ERR_WORKSPACE -5        /* workspace missing or too small           */
+#define DG_ERR_TIMEOUT -6          /* device: a pipeline wait gave up          */
+#define DG_ERR_DEVICE_DATA -7      /* device: bad m_indices / masked_m data    */
+
+/* Input element types for the quantizers. */
+#define DG_DTYPE_F32 0
+#define DG_DTYPE_BF16 1
+
+/* Quantizer flags. */
+#define DG_SCALE_FP32 0 /* scale = fl32(amax / 448)                          */
+#define DG_SCALE_POW2 1 /* scale rounded up to a power of two (UE8M0-exact)  */
+
+/* Text for a status code (static string, never NULL). */
+const char *dg_status_string(int status);
+
+/* Row alignment each expert segment must have in the contiguous grouped
+ * layout (Deep dive, section 3: get_mk_alignment_for_contiguous_layout).
+ * Always 128, the M block of every kernel here. */
+int dg_get_mk_alignment_for_contiguous_layout(void);
+
+/* Smallest n' >= n such that n' * elem_bytes is a multiple of 16 bytes, the
+ * TMA alignment of a leading dimension (DeepGEMM launch article: "get TMA
+ * aligned size" utility).  Returns -1 for n < 0 or elem_bytes not in
+ * {1, 2, 4, 8}.  Use it for ld_sf / ld_sfa. */
+int64_t dg_get_tma_aligned_size(int64_t n, int elem_bytes);
+
+/* Cap the number of SMs the GEMM kernels use (DeepGEMM launch article:
+ * "set max SM count").  n <= 0 restores "all SMs".  Returns DG_OK.  The
+ * setting is process-wide and read at each launch. */
+int dg_set_num_sms(int n);
+
+/* The SM cap in effect for the current device (all SMs when unset). */
+int dg_get_num_sms(void);
+
+/*
+ * dg_quantize_1x128 -- 1 x 128 activation quantization (Lesson 13,
+ * Fig. 13-1; answer to Q1).
+ *
+ * For every batch b, row i < M and group g < K/128 of x:
+ *     amax  = max_k |x[b, i, 128 g + k]|
+ *     alpha = fl32(amax / 448)            (DG_SCALE_POW2: rounded up to 2^e)
+ *     q[b, i, 128 g + k] = E4M3_RNE_satfinite(fl32(x / alpha))
+ * A group with amax == 0 gets alpha = 0 and all codes 0x00.  A negative value
+ * that rounds to zero keeps its sign (0x80).  NaN/Inf inputs are unsupported.
+ *
+ *   x      device, dtype x_dtype (DG_DTYPE_F32 or DG_DTYPE_BF16),
+ *          [batch][M][ld_x] row-major; batch stride M * ld_x elements.
+ *   batch  >= 1; M >= 0 (M == 0 is a no-op); K > 0, K % 128 == 0.
+ *   ld_x   >= K, elements; the row stride must be 16-byte aligned.
+ *   q      device uint8 [batch][M][ld_q] (E4M3 codes); ld_q >= K, ld_q % 16 == 0.
+ *   sf     device float [batch][K/128][ld_sf], MN-major (scale of row i, group
+ *          g of batch b at sf[(b * K/128 + g) * ld_sf + i]);
+ *          ld_sf >= M, ld_sf % 4 == 0 (see dg_get_tma_aligned_size).
+ *   flags  DG_SCALE_FP32 or DG_SCALE_POW2.
+ * All pointers 16-byte aligned.  Output is bit-exact (deterministic).
+ */
+int dg_quantize_1x128(const void *x, int x_dtype, int64_t batch, int64_t M,
+                      int64_t K, int64_t ld_x, uint8_t *q, int64_t ld_q,
+                      float *sf, int64_t ld_sf, int flags, dg_stream_t stream);
+
+/*
+ * dg_quantize_128x128 -- 128 x 128 weight block quantization (Lesson 13,
+ * Fig. 13-1: "one scale beta per 128 x 128 block, quantized offline").
+ *
+ * For every group b < G, block (nb, g) of w[b] (rows 128 nb .. min(N, 128 nb
+ * + 128), columns 128 g .. 128 g + 128): beta = fl32(amax / 448) (or its
+ * power-of-two round-up), q = E4M3_RNE_satfinite(fl32(w / beta)); amax == 0
+ * gives beta = 0 and codes 0x00.
+ *
+ *   w      device float [G][N][K] row-major, 16-byte aligned.
+ *   q      device uint8 [G][N][K].
+ *   sf     device float [G][ceil(N/128)][K/128] row-major.
+ *   G >= 1, N >= 0, K % 128 == 0, K > 0.
+ */
+int dg_quantize_128x128(const float *w, int64_t G, int64_t N, int64_t K,
+                        uint8_t *q, float *sf, int flags, dg_stream_t stream);
+
+/*
+ * dg_fp8_gemm_nt -- dense NT GEMM, D = A * B^T with 1x128 / 128x128 scales
+ * (Lesson 13, Fig. 13-1; DeepGEMM launch article: gemm_fp8_fp8_bf16_nt).
+ *
+ *   A      device uint8 [M][K] E4M3, row-major (K-major), 16-byte aligned.
+ *   sfa    device float [K/128][ld_sfa] MN-major alpha (as written by
+ *          dg_quantize_1x128 with batch 1); ld_sfa >= M, ld_sfa % 4 == 0.
+ *   B      device uint8 [N][K] E4M3, row-major (K-major).
+ *   sfb    device float [ceil(N/128)][K/128] row-major beta.
+ *   D      device BF16 [M][N] row-major, written for all i < M, j < N.
+ *   workspace, workspace_bytes
+ *          optional device scratch (may be NULL / 0).  When at least
+ *          dg_fp8_gemm_nt_workspace_size(M, N, K) bytes are given, small-M
+ *          (decode) shapes may split K across CTAs: FP32 partial results go
+ *          to the workspace and the last CTA of each tile sums them in a fixed
+ *          order.  The workspace must not be used by another call that runs
+ *          at the same time; its contents between calls do not matter.
+ *   M >= 0 (0 is a no-op), N > 0 with N % 8 == 0, K > 0 with K % 128 == 0.
+ * Deterministic: repeated calls give identical bits (also with split K).
+ */
+int dg_fp8_gemm_nt(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                   const uint8_t *B, const float *sfb, void *D, int64_t M,
+                   int64_t N, int64_t K, void *workspace,
+                   size_t workspace_bytes, dg_stream_t stream);
+
+/* Workspace size in bytes that lets dg_fp8_gemm_nt use its split-K path for
+ * this shape (0 when the shape never splits).  16-byte aligned. */
+size_t dg_fp8_gemm_nt_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * dg_m_grouped_fp8_gemm_nt_contiguous -- MoE m-grouped GEMM, contiguous
+ * layout (Lesson 13, Fig. 13-3 "contiguous"; Deep dive, section 3).
+ *
+ * The tokens of all experts are concatenated along M.  Row i belongs to
+ * expert m_indices[i] (-1 = padding row).  Every aligned block of 128 rows
+ * belongs to at most one expert; blocks holding only padding are skipped.
+ *   D[i, :] = A[i, :] * B[m_indices[i]]^T  (with the scales of that expert)
+ * for m_indices[i] >= 0; padding rows of D are not written.
+ *
+ *   A          device uint8 [M_total][K]; sfa device float [K/128][ld_sfa]
+ *              (ld_sfa >= M_total, % 4 == 0).
+ *   B          device uint8 [G][N][K]; sfb device float [G][ceil(N/128)][K/128].
+ *   D          device BF16 [M_total][N].
+ *   m_indices  device int32 [M_total].
+ *   M_total % 128 == 0 (dg_get_mk_alignment_for_contiguous_layout), G >= 1,
+ *   N % 8 == 0, K % 128 == 0.
+ * Device-side errors (recorded, the offending rows are skipped):
+ *   an index >= G, or two different experts inside one 128-row block.
+ */
+int dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sfa,
+                                        int64_t ld_sfa, const uint8_t *B,
+                                        const float *sfb, void *D,
+                                        const int32_t *m_indices,
+                                        int64_t M_total, int64_t N, int64_t K,
+                                        int G, dg_stream_t stream);
+
+/*
+ * dg_m_grouped_fp8_gemm_nt_masked -- MoE m-grouped GEMM, masked layout
+ * (Lesson 13, Fig. 13-3 "masked" and the answer to Q3; Deep dive, section 3).
+ *
+ * Expert g owns the fixed slab A[g] of M_max rows; only its first
+ * masked_m[g] rows are valid.  masked_m is read on the device, so launch
+ * parameters do not depend on it and the call can be replayed from a CUDA
+ * graph with new counts.
+ *   D[g, i, :] = A[g, i, :] * B[g]^T  for i < masked_m[g];
+ * rows i >= masked_m[g] of D are not written.
+ *
+ *   A         device uint8 [G][M_max][K]; sfa device float [G][K/128][ld_sfa]
+ *             (ld_sfa >= M_max, % 4 == 0).
+ *   B         device uint8 [G][N][K]; sfb device float [G][ceil(N/128)][K/128].
+ *   D         device BF16 [G][M_max][N].
+ *   masked_m  device int32 [G]; values outside [0, M_max] are clamped and
+ *             recorded as DG_ERR_DEVICE_DATA.
+ *   1 <= G <= 1024, M_max >= 1, N % 8 == 0, K % 128 == 0.
+ */
+int dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *A, const float *sfa,
+                                    int64_t ld_sfa, const uint8_t *B,
+                                    const float *sfb, void *D,
+                                    const int32_t *masked_m, int G,
+                                    int64_t M_max, int64_t N, int64_t K,
+                                    dg_stream_t stream);
+
+/*
+ * dg_get_device_status -- synchronizes `stream`, then reads and clears the
+ * current device's status word.  *status receives DG_OK or the first device
+ * error recorded since the last read (DG_ERR_TIMEOUT, DG_ERR_DEVICE_DATA).
+ * Returns DG_OK, or DG_ERR_CUDA if the synchronization itself failed.
+ */
+int dg_get_device_status(dg_stream_t stream, int *status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

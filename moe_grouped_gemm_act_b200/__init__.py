@@ -1,0 +1,239 @@
+"""B200 (sm_100a) fine-grained block-scaled FP8 GEMM -- Python binding.
+
+A thin ctypes layer over ``libdg.so`` (declared in ``include/dg.h``).  The
+functions here only marshal torch tensors into pointers, sizes and the current
+CUDA stream; every step of the computation runs in the library's CUDA kernels.
+There is no CPU fallback: if the library is missing or the device is not
+sm_100, the calls raise.
+
+Entry points (same names as the C ABI):
+
+* ``dg_quantize_1x128(x, pow2=False)`` -> (q, sf)    1 x 128 E4M3 activations
+* ``dg_quantize_128x128(w, pow2=False)`` -> (q, sf)  128 x 128 E4M3 weights
+* ``dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace=None)``
+* ``dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices)``
+* ``dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m)``
+* ``dg_get_device_status()``, helpers ``dg_get_tma_aligned_size``,
+  ``dg_get_mk_alignment_for_contiguous_layout``, ``dg_set_num_sms``,
+  ``dg_get_num_sms``, ``dg_fp8_gemm_nt_workspace_size``.
+
+Layouts follow the header: A [M, K] uint8 (E4M3 codes), its scales MN-major
+[K/128, ld] (``sf.t()`` of the logical [M, K/128]), B [N, K] uint8 with scales
+[ceil(N/128), K/128], D [M, N] bfloat16.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdg.so")
+
+DG_OK = 0
+DG_DTYPE_F32, DG_DTYPE_BF16 = 0, 1
+DG_SCALE_FP32, DG_SCALE_POW2 = 0, 1
+DG_ERR_TIMEOUT, DG_ERR_DEVICE_DATA = -6, -7
+
+EXPORTS = [
+    "dg_status_string", "dg_get_mk_alignment_for_contiguous_layout",
+    "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms",
+    "dg_quantize_1x128", "dg_quantize_128x128", "dg_fp8_gemm_nt",
+    "dg_fp8_gemm_nt_workspace_size", "dg_m_grouped_fp8_gemm_nt_contiguous",
+    "dg_m_grouped_fp8_gemm_nt_masked", "dg_get_device_status",
+]
+
+_lib = None
+
+
+class DGError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libdg.so (once) and declares the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing; build it with `python -m moe_grouped_gemm_act_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "dg_status_string": (ctypes.c_char_p, [I]),
+        "dg_get_mk_alignment_for_contiguous_layout": (I, []),
+        "dg_get_tma_aligned_size": (I64, [I64, I]),
+        "dg_set_num_sms": (I, [I]),
+        "dg_get_num_sms": (I, []),
+        "dg_quantize_1x128": (I, [P, I, I64, I64, I64, I64, P, I64, P, I64, I, P]),
+        "dg_quantize_128x128": (I, [P, I64, I64, I64, P, P, I, P]),
+        "dg_fp8_gemm_nt": (I, [P, P, I64, P, P, P, I64, I64, I64, P, SZ, P]),
+        "dg_fp8_gemm_nt_workspace_size": (SZ, [I64, I64, I64]),
+        "dg_m_grouped_fp8_gemm_nt_contiguous":
+            (I, [P, P, I64, P, P, P, P, I64, I64, I64, I, P]),
+        "dg_m_grouped_fp8_gemm_nt_masked":
+            (I, [P, P, I64, P, P, P, P, I, I64, I64, I64, P]),
+        "dg_get_device_status": (I, [P, ctypes.POINTER(ctypes.c_int)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().dg_status_string(int(status)).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != DG_OK:
+        raise DGError(rc, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+# ------------------------------------------------------------------ helpers
+def dg_get_mk_alignment_for_contiguous_layout() -> int:
+    return load_library().dg_get_mk_alignment_for_contiguous_layout()
+
+
+def dg_get_tma_aligned_size(n: int, elem_bytes: int) -> int:
+    return load_library().dg_get_tma_aligned_size(n, elem_bytes)
+
+
+def dg_set_num_sms(n: int) -> None:
+    _check(load_library().dg_set_num_sms(n), "dg_set_num_sms")
+
+
+def dg_get_num_sms() -> int:
+    return load_library().dg_get_num_sms()
+
+
+def dg_fp8_gemm_nt_workspace_size(m: int, n: int, k: int) -> int:
+    return load_library().dg_fp8_gemm_nt_workspace_size(m, n, k)
+
+
+def dg_get_device_status(stream=None) -> int:
+    st = ctypes.c_int(0)
+    _check(load_library().dg_get_device_status(_stream(stream), ctypes.byref(st)),
+           "dg_get_device_status")
+    return st.value
+
+
+# ------------------------------------------------------------------ quantizers
+def dg_quantize_1x128(x: torch.Tensor, pow2: bool = False, q=None, sf=None,
+                      stream=None):
+    """1 x 128 quantization of x [M, K] or [B, M, K] (float32 or bfloat16).
+
+    Returns (q uint8 like x, sf float32 [K/128, ld] or [B, K/128, ld]) with
+    ld = dg_get_tma_aligned_size(M, 4); sf[..., g, i] is the scale of row i,
+    group g.
+    """
+    _need_cuda(x)
+    batched = x.dim() == 3
+    xb = x if batched else x.unsqueeze(0)
+    b, m, k = xb.shape
+    dtype = {torch.float32: DG_DTYPE_F32, torch.bfloat16: DG_DTYPE_BF16}.get(x.dtype)
+    if dtype is None:
+        raise ValueError("x must be float32 or bfloat16")
+    ld = dg_get_tma_aligned_size(m, 4)
+    if q is None:
+        q = torch.empty(xb.shape, dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty((b, k // 128, ld), dtype=torch.float32, device=x.device)
+    rc = load_library().dg_quantize_1x128(
+        _ptr(xb), dtype, b, m, k, k, _ptr(q), k, _ptr(sf), sf.shape[-1],
+        DG_SCALE_POW2 if pow2 else DG_SCALE_FP32, _stream(stream))
+    _check(rc, "dg_quantize_1x128")
+    if not batched:
+        return q.view(m, k), sf.view(k // 128, sf.shape[-1])
+    return q, sf
+
+
+def dg_quantize_128x128(w: torch.Tensor, pow2: bool = False, stream=None):
+    """128 x 128 quantization of w [N, K] or [G, N, K] float32.
+
+    Returns (q uint8 like w, sf float32 [ceil(N/128), K/128] or
+    [G, ceil(N/128), K/128])."""
+    _need_cuda(w)
+    if w.dtype != torch.float32:
+        raise ValueError("w must be float32")
+    grouped = w.dim() == 3
+    wb = w if grouped else w.unsqueeze(0)
+    g, n, k = wb.shape
+    q = torch.empty(wb.shape, dtype=torch.uint8, device=w.device)
+    sf = torch.empty((g, -(-n // 128), k // 128), dtype=torch.float32, device=w.device)
+    rc = load_library().dg_quantize_128x128(
+        _ptr(wb), g, n, k, _ptr(q), _ptr(sf),
+        DG_SCALE_POW2 if pow2 else DG_SCALE_FP32, _stream(stream))
+    _check(rc, "dg_quantize_128x128")
+    if not grouped:
+        return q[0], sf[0]
+    return q, sf
+
+
+# ------------------------------------------------------------------ GEMMs
+def dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """D = A * B^T with 1x128 (sfa, MN-major [K/128, ld]) and 128x128 (sfb)
+    scales; d is a preallocated bfloat16 [M, N] tensor, returned."""
+    _need_cuda(a, sfa, b, sfb, d)
+    m, k = a.shape
+    n = b.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load_library().dg_fp8_gemm_nt(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d), m, n, k,
+        _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dg_fp8_gemm_nt")
+    return d
+
+
+def dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices,
+                                        stream=None) -> torch.Tensor:
+    """Contiguous m-grouped GEMM: a [M_total, K], b [G, N, K], m_indices int32
+    [M_total] (-1 = padding); padding rows of d are not written."""
+    _need_cuda(a, sfa, b, sfb, d, m_indices)
+    m_total, k = a.shape
+    g, n, _ = b.shape
+    rc = load_library().dg_m_grouped_fp8_gemm_nt_contiguous(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d),
+        _ptr(m_indices), m_total, n, k, g, _stream(stream))
+    _check(rc, "dg_m_grouped_fp8_gemm_nt_contiguous")
+    return d
+
+
+def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m,
+                                    stream=None) -> torch.Tensor:
+    """Masked m-grouped GEMM: a [G, M_max, K], sfa [G, K/128, ld], b [G, N, K],
+    masked_m int32 [G] on the device; rows >= masked_m[g] of d untouched."""
+    _need_cuda(a, sfa, b, sfb, d, masked_m)
+    g, m_max, k = a.shape
+    n = b.shape[1]
+    rc = load_library().dg_m_grouped_fp8_gemm_nt_masked(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d),
+        _ptr(masked_m), g, m_max, n, k, _stream(stream))
+    _check(rc, "dg_m_grouped_fp8_gemm_nt_masked")
+    return d

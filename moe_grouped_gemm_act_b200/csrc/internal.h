@@ -1,0 +1,85 @@
+// internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "dg.h"
+
+namespace dg {
+
+// ---------------------------------------------------------------- quantizers
+int launch_quantize_1x128(const void *x, int x_dtype, int64_t batch, int64_t M,
+                          int64_t K, int64_t ld_x, uint8_t *q, int64_t ld_q,
+                          float *sf, int64_t ld_sf, int flags,
+                          cudaStream_t stream, int num_sms);
+
+int launch_quantize_128x128(const float *w, int64_t G, int64_t N, int64_t K,
+                            uint8_t *q, float *sf, int flags,
+                            cudaStream_t stream);
+
+// ---------------------------------------------------------------- GEMM
+enum Sched : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+
+// Kernel parameters besides the two tensor maps.  Row coordinates are inside
+// one "slab": the whole of A for dense and contiguous, one expert's M_max rows
+// for masked.
+struct GemmParams {
+  const float *sfa;      // MN-major alpha: [slab][K/128][ld_sfa]
+  int64_t ld_sfa;
+  const float *sfb;      // beta: [group][ceil(N/128)][K/128]
+  uint16_t *d;           // BF16 output [slab][rows][N]
+  const int32_t *m_indices;  // contiguous: expert per row (-1 = padding)
+  const int32_t *masked_m;   // masked: valid rows per expert
+  int *status;           // device status word (first error wins)
+  float *ws;             // split-K partials (nullptr: no split)
+  uint32_t *ws_ticket;   // split-K arrival counters, one per output tile
+  int rows;              // dense: M; contiguous: M_total; masked: M_max
+  int n, k;
+  int groups;            // experts (1 for dense)
+  int num_m_blocks;      // ceil(rows / 128)
+  int num_n_blocks;      // ceil(n / BN)
+  int num_k_blocks;      // k / 128
+  int splits;            // K splits (1 = none)
+};
+
+struct GemmConfig {
+  int block_n;
+  int stages;
+  int splits;
+  int num_sms;
+  int smem_bytes;
+};
+
+// Host entry of the GEMM: picks a config, encodes tensor maps, launches.
+int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B,
+                    GemmParams p, cudaStream_t stream, int num_sms,
+                    size_t ws_bytes, void *ws);
+
+size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int num_sms);
+
+// ---------------------------------------------------------------- device state
+struct DeviceInfo {
+  int ok;            // 1 when the device is usable (sm_100)
+  int num_sms;
+  int max_smem_optin;
+  int *status;       // device address of the status word
+};
+
+// Per-device properties (cached); returns nullptr on a CUDA error.
+const DeviceInfo *device_info();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t,
+                                  void *, const cuuint64_t *, const cuuint64_t *,
+                                  const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+int effective_num_sms();
+
+}  // namespace dg

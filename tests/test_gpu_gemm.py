@@ -1,0 +1,383 @@
+"""GPU parity of the three GEMM entry points against the oracle (through the
+C ABI): shapes spanning several tiles with ragged tails, every N-tile instance,
+split K, the exact-integer special case, untouched padding / masked rows,
+determinism and CUDA-graph replay of the masked call."""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import moe_grouped_gemm_act_b200 as dg
+from moe_grouped_gemm_act_b200 import inputs
+from oracle import bf16, e4m3, gemm, quant
+
+from _helpers import bits_of, check_gemm, dev, sfa_batched_to_device, sfa_to_device
+
+pytestmark = pytest.mark.gpu
+
+SENTINEL = 0x7FC1  # a NaN bit pattern no GEMM result can produce
+
+
+class env:
+    """Temporarily set library tuning variables (read at each call)."""
+
+    def __init__(self, **kv):
+        self.kv = {k: str(v) for k, v in kv.items()}
+
+    def __enter__(self):
+        self.old = {k: os.environ.get(k) for k in self.kv}
+        os.environ.update(self.kv)
+
+    def __exit__(self, *a):
+        for k, v in self.old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
+def dense_case(m, n, k, seed, outliers=True):
+    x = inputs.activations(m, k, seed=seed, outliers=outliers)
+    w = inputs.weights((n, k), seed=seed + 1)
+    qa, alpha = quant.quantize_1x128(x)
+    qb, beta = quant.quantize_128x128(w)
+    return qa, alpha, qb, beta
+
+
+def run_dense(qa, alpha, qb, beta, workspace=False):
+    m, n = qa.shape[0], qb.shape[0]
+    d = torch.full((m, n), 0, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    ws = None
+    if workspace:
+        nbytes = dg.dg_fp8_gemm_nt_workspace_size(m, n, qa.shape[1])
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
+    dg.dg_fp8_gemm_nt(dev(qa), sfa_to_device(alpha), dev(qb), dev(beta), d, workspace=ws)
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    return bits_of(d)
+
+
+# ------------------------------------------------------------------ dense
+def test_dense_parity_config():
+    c = inputs.DENSE_PARITY
+    x = inputs.activations(c["m"], c["k"], seed=c["seed_a"])
+    w = inputs.weights((c["n"], c["k"]), seed=c["seed_b"])
+    qa, alpha = quant.quantize_1x128(x)
+    qb, beta = quant.quantize_128x128(w)
+    got = run_dense(qa, alpha, qb, beta)
+    check_gemm(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), "128x256x512")
+
+
+@pytest.mark.parametrize("bn", [16, 32, 64, 128])
+@pytest.mark.parametrize("m,n,k", [(300, 392, 1024), (1, 136, 256), (129, 2112, 384)])
+def test_dense_ragged_every_block_n(bn, m, n, k):
+    qa, alpha, qb, beta = dense_case(m, n, k, seed=m + n + k)
+    with env(DG_BLOCK_N=bn):
+        got = run_dense(qa, alpha, qb, beta)
+    check_gemm(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"{m}x{n}x{k} BN={bn}")
+
+
+@pytest.mark.parametrize("splits", [2, 3, 8])
+@pytest.mark.parametrize("bn", [32, 128])
+def test_dense_split_k(splits, bn):
+    qa, alpha, qb, beta = dense_case(64, 528, 2048, seed=splits)
+    want = gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta)
+    with env(DG_BLOCK_N=bn, DG_SPLITS=splits):
+        a = run_dense(qa, alpha, qb, beta, workspace=True)
+        b = run_dense(qa, alpha, qb, beta, workspace=True)
+    check_gemm(a, want, f"split {splits}")
+    assert np.array_equal(a, b), "split-K result not deterministic"
+
+
+def test_dense_exact_integers_bit_exact():
+    # integer codes in [-4, 4] with unit scales: every 128-K partial and the
+    # FP32 running sum are exact, so D must equal BF16(exact) bit for bit
+    g = np.random.default_rng(1)
+    m, n, k = 256, 384, 7168
+    a = g.integers(-4, 5, size=(m, k)).astype(np.float32)
+    b = g.integers(-4, 5, size=(n, k)).astype(np.float32)
+    qa, qb = e4m3.encode_rne(a), e4m3.encode_rne(b)
+    alpha = np.ones((m, k // 128), np.float32)
+    beta = np.ones((-(-n // 128), k // 128), np.float32)
+    got = run_dense(qa, alpha, qb, beta)
+    exact = a.astype(np.int64) @ b.astype(np.int64).T
+    assert np.array_equal(got, bf16.to_bits(exact.astype(np.float64)))
+
+
+def test_dense_deterministic():
+    qa, alpha, qb, beta = dense_case(512, 1024, 2048, seed=3)
+    assert np.array_equal(run_dense(qa, alpha, qb, beta), run_dense(qa, alpha, qb, beta))
+
+
+def test_dense_lesson13_exercise_inputs():
+    # the worked exercise of Lesson 13 (integers in [-10, 10) are exact E4M3)
+    np.random.seed(42)
+    A = np.random.randint(-10, 10, size=(128, 256)).astype(np.float32)
+    B = np.random.randint(-10, 10, size=(256, 256)).astype(np.float32)
+    SA = np.random.uniform(0.01, 0.05, size=(128, 2)).astype(np.float32)
+    SB = np.random.uniform(0.01, 0.05, size=(2, 2)).astype(np.float32)
+    qa, qb = e4m3.encode_rne(A), e4m3.encode_rne(B)
+    got = run_dense(qa, SA, qb, SB)
+    check_gemm(got, gemm.fp8_gemm_nt_f64(qa, SA, qb, SB), "exercise")
+
+
+@pytest.mark.parametrize("n,k", inputs.PREFILL_NK)
+def test_dense_prefill_full_size_sampled_rows(n, k):
+    # full bench shape, launch configuration of the bench; all columns of a
+    # sampled row set (first/last row of every M tile + 2 random rows per tile)
+    m = inputs.PREFILL_M
+    x = inputs.activations(m, k, seed=inputs.PREFILL_SEEDS["seed_a"], outliers=True)
+    w = inputs.weights((n, k), seed=inputs.PREFILL_SEEDS["seed_b"])
+    qa_d, sfa_d = dg.dg_quantize_1x128(torch.from_numpy(x).cuda())
+    qb_d, sfb_d = dg.dg_quantize_128x128(torch.from_numpy(w).cuda())
+    d = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    dg.dg_fp8_gemm_nt(qa_d, sfa_d, qb_d, sfb_d, d)
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    g = np.random.default_rng(n + k)
+    rows = []
+    for t in range(m // 128):
+        rows += [128 * t, 128 * t + 127, *(128 * t + g.integers(1, 127, size=2))]
+    rows = np.array(sorted(set(rows)))
+    qa, alpha = quant.quantize_1x128(x[rows])
+    qb, beta = quant.quantize_128x128(w)
+    # the device quantizers are bit-exact; check that on the sampled rows too
+    assert np.array_equal(qa_d.cpu().numpy()[rows], qa)
+    want = gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta)
+    check_gemm(bits_of(d)[rows], want, f"prefill {n}x{k}")
+
+
+@pytest.mark.parametrize("m", inputs.DECODE_M)
+@pytest.mark.parametrize("n,k", inputs.PREFILL_NK)
+def test_dense_decode_full_size(m, n, k):
+    x = inputs.activations(m, k, seed=inputs.DECODE_SEEDS["seed_a"], outliers=True)
+    w = inputs.weights((n, k), seed=inputs.DECODE_SEEDS["seed_b"])
+    qb_d, sfb_d = dg.dg_quantize_128x128(torch.from_numpy(w).cuda())
+    qa, alpha = quant.quantize_1x128(x)
+    d = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    nbytes = dg.dg_fp8_gemm_nt_workspace_size(m, n, k)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
+    dg.dg_fp8_gemm_nt(dev(qa), sfa_to_device(alpha), qb_d, sfb_d, d, workspace=ws)
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    qb, beta = quant.quantize_128x128(w)
+    check_gemm(bits_of(d), gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"decode {m}x{n}x{k}")
+
+
+def test_dense_m_zero_is_noop():
+    d = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    a = torch.empty((0, 128), dtype=torch.uint8, device="cuda")
+    sfa = torch.empty((1, 4), dtype=torch.float32, device="cuda")
+    b = torch.zeros((128, 128), dtype=torch.uint8, device="cuda")
+    sfb = torch.zeros((1, 1), dtype=torch.float32, device="cuda")
+    dg.dg_fp8_gemm_nt(a, sfa, b, sfb, d)
+
+
+def test_dense_rejects_bad_shapes():
+    a = torch.zeros((128, 200), dtype=torch.uint8, device="cuda")
+    sfa = torch.zeros((2, 128), dtype=torch.float32, device="cuda")
+    b = torch.zeros((128, 200), dtype=torch.uint8, device="cuda")
+    sfb = torch.zeros((1, 2), dtype=torch.float32, device="cuda")
+    d = torch.empty((128, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(dg.DGError):
+        dg.dg_fp8_gemm_nt(a, sfa, b, sfb, d)   # K % 128 != 0
+
+
+# ------------------------------------------------------------------ contiguous
+def contiguous_case(tokens, groups, n, k, seed):
+    lay = inputs.contiguous_layout(tokens, groups, seed=seed)
+    x = inputs.activations(lay.m_total, k, seed=seed + 1, outliers=True)
+    w = inputs.weights((groups, n, k), seed=seed + 2)
+    qa, alpha = quant.quantize_1x128(x)
+    qb, beta = quant.quantize_128x128_grouped(w)
+    pad = lay.m_indices < 0
+    qa[pad] = 0x7F            # NaN codes on padding rows: must not leak
+    alpha[pad] = np.nan
+    return lay, qa, alpha, qb, beta
+
+
+def run_contiguous(lay, qa, alpha, qb, beta):
+    m_total, n = qa.shape[0], qb.shape[1]
+    d = torch.full((m_total, n), SENTINEL, dtype=torch.int16, device="cuda")
+    dg.dg_m_grouped_fp8_gemm_nt_contiguous(
+        dev(qa), sfa_to_device(alpha), dev(qb), dev(beta), d.view(torch.bfloat16),
+        dev(lay.m_indices))
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    return bits_of(d.view(torch.bfloat16))
+
+
+@pytest.mark.parametrize("bn", [16, 64, 128])
+def test_contiguous_parity_and_padding_untouched(bn):
+    lay, qa, alpha, qb, beta = contiguous_case(1000, 5, 264, 512, seed=60)
+    with env(DG_BLOCK_N=bn):
+        got = run_contiguous(lay, qa, alpha, qb, beta)
+    pad = lay.m_indices < 0
+    assert np.all(got[pad] == SENTINEL)
+    want = gemm.m_grouped_contiguous_f64(qa, alpha, qb, beta, lay.m_indices,
+                                         np.zeros(got.shape))
+    check_gemm(got[~pad], want[~pad], f"contiguous BN={bn}")
+
+
+def test_contiguous_empty_expert_and_padding_only_blocks():
+    # expert 1 has no tokens; an extra all-padding 128-row block at the end
+    lay, qa, alpha, qb, beta = contiguous_case(300, 3, 128, 256, seed=61)
+    lay.m_indices[lay.m_indices == 1] = -1
+    idx = np.concatenate([lay.m_indices, np.full(128, -1, np.int32)])
+    qa = np.concatenate([qa, np.full((128, qa.shape[1]), 0x7F, np.uint8)])
+    alpha = np.concatenate([alpha, np.full((128, alpha.shape[1]), np.nan, np.float32)])
+    lay2 = inputs.ContiguousLayout(lay.counts, idx, len(idx))
+    got = run_contiguous(lay2, qa, alpha, qb, beta)
+    pad = idx < 0
+    assert np.all(got[pad] == SENTINEL)
+    want = gemm.m_grouped_contiguous_f64(qa, alpha, qb, beta, idx, np.zeros(got.shape))
+    check_gemm(got[~pad], want[~pad], "contiguous sparse")
+
+
+def test_contiguous_bad_index_reports_status():
+    lay, qa, alpha, qb, beta = contiguous_case(256, 2, 128, 256, seed=62)
+    idx = lay.m_indices.copy()
+    idx[0] = 7                       # >= G
+    d = torch.full((qa.shape[0], 128), SENTINEL, dtype=torch.int16, device="cuda")
+    dg.dg_m_grouped_fp8_gemm_nt_contiguous(
+        dev(qa), sfa_to_device(alpha), dev(qb), dev(beta), d.view(torch.bfloat16), dev(idx))
+    assert dg.dg_get_device_status() == dg.DG_ERR_DEVICE_DATA
+    assert dg.dg_get_device_status() == 0   # read clears
+
+
+def test_contiguous_full_size_sampled_rows():
+    c = inputs.CONTIGUOUS
+    lay = inputs.contiguous_layout(c["tokens"], c["groups"], seed=c["seed"])
+    k, n, G = c["k"], c["n"], c["groups"]
+    x = inputs.activations(lay.m_total, k, seed=c["seed"] + 1, outliers=True)
+    w = inputs.weights((G, n, k), seed=c["seed"] + 2)
+    qa_d, sfa_d = dg.dg_quantize_1x128(torch.from_numpy(x).cuda())
+    qb_d, sfb_d = dg.dg_quantize_128x128(torch.from_numpy(w).cuda())
+    d = torch.full((lay.m_total, n), SENTINEL, dtype=torch.int16, device="cuda")
+    dg.dg_m_grouped_fp8_gemm_nt_contiguous(qa_d, sfa_d, qb_d, sfb_d,
+                                           d.view(torch.bfloat16), dev(lay.m_indices))
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    got = bits_of(d.view(torch.bfloat16))
+    pad = lay.m_indices < 0
+    assert np.all(got[pad] == SENTINEL)
+    g = np.random.default_rng(5)
+    rows = np.sort(g.choice(np.nonzero(~pad)[0], size=48, replace=False))
+    qa, alpha = quant.quantize_1x128(x[rows])
+    for e in range(G):
+        sel = rows[lay.m_indices[rows] == e]
+        if len(sel) == 0:
+            continue
+        qb, beta = quant.quantize_128x128(w[e])
+        i = np.searchsorted(rows, sel)
+        want = gemm.fp8_gemm_nt_f64(qa[i], alpha[i], qb, beta)
+        check_gemm(got[sel], want, f"contiguous expert {e}")
+
+
+# ------------------------------------------------------------------ masked
+def masked_case(G, m_max, n, k, seed, pow2=False):
+    x = inputs.activations(G * m_max, k, seed=seed, outliers=True).reshape(G, m_max, k)
+    w = inputs.weights((G, n, k), seed=seed + 1)
+    qa, alpha = zip(*(quant.quantize_1x128(x[e], pow2=pow2) for e in range(G)))
+    qa, alpha = np.stack(qa), np.stack(alpha)
+    qb, beta = quant.quantize_128x128_grouped(w, pow2=pow2)
+    return qa, alpha, qb, beta
+
+
+def run_masked(qa, alpha, qb, beta, masked_m):
+    G, m_max, _ = qa.shape
+    n = qb.shape[1]
+    d = torch.full((G, m_max, n), SENTINEL, dtype=torch.int16, device="cuda")
+    dg.dg_m_grouped_fp8_gemm_nt_masked(dev(qa), sfa_batched_to_device(alpha), dev(qb),
+                                       dev(beta), d.view(torch.bfloat16),
+                                       dev(np.asarray(masked_m, np.int32)))
+    torch.cuda.synchronize()
+    return bits_of(d.view(torch.bfloat16))
+
+
+def check_masked(got, qa, alpha, qb, beta, masked_m, what):
+    for e in range(qa.shape[0]):
+        m = int(min(max(masked_m[e], 0), qa.shape[1]))
+        assert np.all(got[e, m:] == SENTINEL), f"{what}: rows >= masked_m written"
+        if m:
+            check_gemm(got[e, :m], gemm.fp8_gemm_nt_f64(qa[e, :m], alpha[e, :m], qb[e], beta[e]),
+                       f"{what} expert {e}")
+
+
+@pytest.mark.parametrize("bn", [16, 128])
+def test_masked_parity_and_rows_untouched(bn):
+    qa, alpha, qb, beta = masked_case(5, 300, 264, 512, seed=70)
+    masked_m = [0, 300, 129, 1, 128]
+    with env(DG_BLOCK_N=bn):
+        got = run_masked(qa, alpha, qb, beta, masked_m)
+    assert dg.dg_get_device_status() == 0
+    check_masked(got, qa, alpha, qb, beta, masked_m, f"masked BN={bn}")
+
+
+def test_masked_pow2_scales():
+    qa, alpha, qb, beta = masked_case(4, 256, 512, 1024, seed=71, pow2=True)
+    masked_m = [256, 17, 0, 200]
+    got = run_masked(qa, alpha, qb, beta, masked_m)
+    check_masked(got, qa, alpha, qb, beta, masked_m, "masked pow2")
+
+
+def test_masked_out_of_range_counts_clamped_and_reported():
+    qa, alpha, qb, beta = masked_case(3, 128, 128, 256, seed=72)
+    masked_m = [-3, 500, 64]
+    got = run_masked(qa, alpha, qb, beta, masked_m)
+    assert dg.dg_get_device_status() == dg.DG_ERR_DEVICE_DATA
+    check_masked(got, qa, alpha, qb, beta, masked_m, "masked clamp")
+
+
+def test_masked_cuda_graph_replay():
+    G, m_max, n, k = 6, 256, 384, 1024
+    qa, alpha, qb, beta = masked_case(G, m_max, n, k, seed=73)
+    a, sfa, b, sfb = dev(qa), sfa_batched_to_device(alpha), dev(qb), dev(beta)
+    mm = torch.zeros(G, dtype=torch.int32, device="cuda")
+    d = torch.full((G, m_max, n), SENTINEL, dtype=torch.int16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        dg.dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d.view(torch.bfloat16), mm)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        dg.dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d.view(torch.bfloat16), mm)
+    rng = np.random.default_rng(3)
+    for _ in range(3):
+        counts = rng.integers(0, m_max + 1, size=G).astype(np.int32)
+        mm.copy_(torch.from_numpy(counts))
+        d.fill_(SENTINEL)
+        graph.replay()
+        torch.cuda.synchronize()
+        got = bits_of(d.view(torch.bfloat16))
+        check_masked(got, qa, alpha, qb, beta, counts, "graph replay")
+    assert dg.dg_get_device_status() == 0
+
+
+def test_masked_full_size_sampled():
+    c = inputs.MASKED
+    G, m_max, n, k = c["groups"], c["m_max"], c["n"], c["k"]
+    masked_m = inputs.masked_counts(G, m_max, seed=c["seed"])
+    x = inputs.activations(G * m_max, k, seed=c["seed"] + 1, outliers=True).reshape(G, m_max, k)
+    w = inputs.weights((G, n, k), seed=c["seed"] + 2)
+    qa_d, sfa_d = dg.dg_quantize_1x128(torch.from_numpy(x).cuda())
+    qb_d, sfb_d = dg.dg_quantize_128x128(torch.from_numpy(w).cuda())
+    d = torch.full((G, m_max, n), SENTINEL, dtype=torch.int16, device="cuda")
+    dg.dg_m_grouped_fp8_gemm_nt_masked(qa_d, sfa_d, qb_d, sfb_d, d.view(torch.bfloat16),
+                                       dev(masked_m))
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    got = bits_of(d.view(torch.bfloat16))
+    for e in range(G):
+        assert np.all(got[e, masked_m[e]:] == SENTINEL)
+    for e in [0, 5, 17, 31]:            # experts checked in full against the oracle
+        m = int(masked_m[e])
+        if not m:
+            continue
+        qa, alpha = quant.quantize_1x128(x[e, :m])
+        qb, beta = quant.quantize_128x128(w[e])
+        check_gemm(got[e, :m], gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"masked e{e}")
