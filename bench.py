@@ -93,7 +93,8 @@ def peaks() -> dict:
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples nvidia-smi every 200 ms while the timed region runs."""
+    """Samples nvidia-smi every 100 ms; ``summary`` keeps the samples taken
+    between ``mark_start`` and ``mark_stop`` (the timed region)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -102,26 +103,35 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.lines: list[str] = []
+        self.lines: list[tuple[float, str]] = []
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            time.sleep(0.3)  # let the first samples arrive
         except OSError:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_stop(self):
+        self.t1 = time.time()
 
     def __exit__(self, *a):
         if self.proc is not None:
+            time.sleep(0.15)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -131,7 +141,9 @@ class ClockSampler:
     def summary(self) -> dict:
         sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ts, ln in self.lines:
+            if self.t0 is not None and not (self.t0 <= ts <= (self.t1 or ts) + 0.1):
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -321,19 +333,21 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         torch.cuda.synchronize()
 
     # ------------------------------------------------ device-resident timing
-    for _ in range(args.warmup):
-        data.step()
     nshape = len(data.shapes)
     gemm_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(nshape)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
     with ClockSampler(local_rank) as clocks:
+        for _ in range(args.warmup):
+            data.step()
+        barrier()
+        clocks.mark_start()
         start.record()
         for i in range(args.steps):
             data.step(gemm_ev[i])
         stop.record()
         torch.cuda.synchronize()
+        clocks.mark_stop()
     barrier()
     total_ms = start.elapsed_time(stop)
     gemm_ms = [sum(e0.elapsed_time(e1) for e0, e1 in gemm_ev[i]) for i in range(args.steps)]
@@ -347,13 +361,14 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 25))  # PCIe-bound; fewer steps suffice
     e0.record()
-    for _ in range(args.steps):
+    for _ in range(e2e_steps):
         data.e2e_step(device)
     e1.record()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = e0.elapsed_time(e1) * args.steps / e2e_steps
 
     # ------------------------------------------------ max over ranks
     t = torch.tensor([total_ms, e2e_ms, sum(gemm_ms)], dtype=torch.float64, device=device)
@@ -420,8 +435,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="prefill",
                     choices=["prefill", "decode64", "decode128"])
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])

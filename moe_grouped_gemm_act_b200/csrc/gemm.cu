@@ -11,21 +11,26 @@
 // consumer pipeline).  The Hopper design on that page (TMA producer warpgroup,
 // WGMMA into registers, math warpgroups) is re-derived for Blackwell:
 //
-//   warp 0      TMA producer: one elected lane streams A [128 x 128] and
-//               B [BN x 128] K blocks into a STAGES-deep shared-memory ring
-//               (128-byte swizzle), completing on `full` mbarriers.
-//   warp 1      MMA issuer: one lane issues 4 tcgen05.mma (kind::f8f6f4,
-//               M=128, N=BN, K=32) per K block into one of two TMEM
-//               accumulator buffers, then tcgen05.commit frees the smem stage
-//               (`empty`) and publishes the buffer (`tmem_full`).  Each K
-//               block's product starts from zero (fresh partial sum).
-//   warps 4-11  promotion warpgroups: TMEM row i is read by the warp whose
-//               index mod 4 is i / 32; the two warpgroups split the BN
-//               columns.  Each thread owns one row and BN/2 columns: it loads
-//               the partial sum with tcgen05.ld, releases the TMEM buffer
-//               (`tmem_empty`) so the next block's MMA can start, and does
-//               acc += partial * (alpha_row * beta) in registers.  After the
-//               last K block it converts to BF16 and stores its row segment.
+//   warp 0      TMA producer: one lane streams A [128 x 128] and B [BN x 128]
+//               K blocks into a STAGES-deep shared-memory ring (128-byte
+//               swizzle), and the block's 128 row scales alpha (one 512-byte
+//               bulk copy from the MN-major scale array) into a separate ring
+//               of kAlphaSlots slots, all completing on mbarriers.
+//   warp 1      MMA issuer: allocates TMEM and, for each K block, issues 4
+//               tcgen05.mma (kind::f8f6f4, M=128, N=BN, K=32) into one of NBUF
+//               TMEM buffers (the first with accumulate off: a fresh partial
+//               sum per block), then tcgen05.commit frees the smem stage and
+//               publishes the buffer.  NBUF buffers let the tensor cores run
+//               up to NBUF blocks ahead of the promotion.
+//   warps 2-3   idle after set-up (warp 2 builds the masked prefix table);
+//               warps 0-3 form the control warpgroup, whose registers the
+//               promotion warpgroups take over for BN = 256.
+//   warps 4-11  promotion: warp w reads TMEM lanes 32 (w mod 4) .. +31; warps
+//               4-7 and 8-11 split the BN columns.  Each thread owns one row
+//               and BN/2 columns: it pulls the block's partial sum with
+//               tcgen05.ld, releases the buffer, and does acc += partial *
+//               (alpha_row * beta) in FP32 registers.  After the last K block
+//               it converts to BF16 and stores its row segment (valid rows).
 //
 // The kernel is persistent (one CTA per SM).  All roles walk the same tile
 // sequence produced by a scheduler that knows the three layouts:
@@ -55,17 +60,29 @@ namespace {
 
 constexpr int BM = 128;                 // rows per tile (one UMMA M)
 constexpr int BK = 128;                 // K per block = one scale group
-constexpr int kThreads = 384;           // 4 control warps + 2 promotion warpgroups
-constexpr int kPromoThreads = 256;
-constexpr int kPromoWarps = 8;
+constexpr int kControlWarps = 4;        // producer, MMA issuer, 2 helpers (one warpgroup)
+constexpr int kPromoWarps = 8;          // two column halves x four lane quarters
+constexpr int kPromoThreads = 32 * kPromoWarps;
+constexpr int kThreads = 32 * (kControlWarps + kPromoWarps);
+constexpr int kAlphaSlots = 16;         // alpha ring depth (>= STAGES + NBUF)
 constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 
-template <int BN>
+template <int BN, int STAGES, int NBUF>
 struct Layout {
   static constexpr uint32_t kBBytes = BN * BK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
+  static constexpr uint32_t kAlphaOff = STAGES * kStageBytes;
+  static constexpr uint32_t kBarOff = kAlphaOff + kAlphaSlots * BM * 4;
+  // full[S] empty[S] afull[A] aempty[A] tfull[NBUF] tempty[NBUF] drain
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAlphaSlots + 2 * NBUF + 1;
+  static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
+  static constexpr uint32_t kPrefixOff = kMiscOff + 16;
+  static constexpr uint32_t kCols = BN * NBUF;
+  static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64
+                                      : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
+  static_assert(kCols <= 512, "TMEM holds 512 columns");
+  static_assert(STAGES + NBUF <= kAlphaSlots, "alpha ring must cover the pipeline");
 };
 
 // ------------------------------------------------------------------ scheduler
@@ -76,15 +93,13 @@ struct Tile {
   int k_begin, k_end;  // K blocks of this unit
 };
 
-// Returns the number of work units for this launch (dense/contiguous: tiles x
-// splits; masked: from the prefix table in shared memory).
 __device__ __forceinline__ int num_units(const GemmParams &p, int sched,
                                          const int *s_prefix) {
   if (sched == kMasked) return s_prefix[p.groups];
   return p.num_m_blocks * p.num_n_blocks * p.splits;
 }
 
-// Maps unit u to a tile.  Contiguous expert lookup is done separately.
+// Maps unit u to a tile.  The contiguous expert lookup is done separately.
 __device__ __forceinline__ Tile unit_to_tile(const GemmParams &p, int sched,
                                              int u, const int *s_prefix,
                                              const int *s_mblocks) {
@@ -93,7 +108,8 @@ __device__ __forceinline__ Tile unit_to_tile(const GemmParams &p, int sched,
   t.slab = 0;
   t.group = 0;
   if (sched == kMasked) {
-    // largest e with prefix[e] <= u
+    // largest e with prefix[e] <= u; within an expert, the M blocks of one N
+    // block are adjacent so that they share B in L2
     int lo = 0, hi = p.groups - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -118,7 +134,6 @@ __device__ __forceinline__ Tile unit_to_tile(const GemmParams &p, int sched,
     t.m_blk = first_m + r % gm;
     t.n_blk = r / gm;
   }
-  // K range of this split: contiguous, balanced to within one block.
   const int kb = p.num_k_blocks, s = p.splits;
   t.k_begin = (kb * t.split) / s;
   t.k_end = (kb * (t.split + 1)) / s;
@@ -126,8 +141,8 @@ __device__ __forceinline__ Tile unit_to_tile(const GemmParams &p, int sched,
 }
 
 // Contiguous layout: the expert of a 128-row block, or -1 when the block holds
-// only padding.  Whole warp; every lane returns the same value.  When
-// `check` is set, a block mixing experts or holding an index >= groups records
+// only padding.  Whole warp; every lane returns the same value.  With `check`,
+// a block mixing experts or holding an index >= groups records
 // DG_ERR_DEVICE_DATA (rows of other experts are then not written).
 __device__ __forceinline__ int block_expert(const GemmParams &p, int m_blk,
                                             bool check) {
@@ -138,11 +153,9 @@ __device__ __forceinline__ int block_expert(const GemmParams &p, int m_blk,
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     if (vals[i] >= 0 && first == 0x7FFFFFFF) first = vals[i];
-  // lowest lane with a valid row holds the block's first valid index
   const unsigned any = __ballot_sync(0xffffffffu, first != 0x7FFFFFFF);
   if (!any) return -1;
-  const int src = __ffs(any) - 1;
-  const int e = __shfl_sync(0xffffffffu, first, src);
+  const int e = __shfl_sync(0xffffffffu, first, __ffs(any) - 1);
   if (check) {
     bool bad = false;
 #pragma unroll
@@ -153,16 +166,24 @@ __device__ __forceinline__ int block_expert(const GemmParams &p, int m_blk,
   return e < p.groups ? e : -1;
 }
 
+__device__ __forceinline__ int masked_rows(const GemmParams &p, int e) {
+  const int m = __ldg(p.masked_m + e);
+  return m < 0 ? 0 : (m > p.rows ? p.rows : m);
+}
+
 // ------------------------------------------------------------------ the kernel
-template <int BN, int STAGES, int SCHED>
+template <int BN, int STAGES, int NBUF, int SCHED>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
                 const GemmParams p) {
-  using L = Layout<BN>;
-  constexpr int W = BN / 2;  // columns per promotion thread
+  using L = Layout<BN, STAGES, NBUF>;
+  constexpr int W = BN / 2;                 // columns per promotion thread
+  // columns per TMEM load chunk: the whole slice up to 64; for BN = 256 the
+  // 128 accumulators leave room for 16-column chunks under 168 registers
+  constexpr int LW = W <= 64 ? W : 16;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
-  static_assert(W == 8 || W == 16 || W == 32 || W == 64, "TMEM load width");
+  static_assert(W % LW == 0 && (LW == 8 || LW == 16 || LW == 32 || LW == 64), "TMEM chunk");
 
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
@@ -170,18 +191,22 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t *smem = smem_raw + (base - raw);
 
-  const uint32_t bar_base = base + STAGES * L::kStageBytes;
-  auto full_bar = [&](int s) { return bar_base + 8u * s; };
-  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
-  auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
-  auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
-  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
-  uint8_t *misc = smem + STAGES * L::kStageBytes + 8 * (2 * STAGES + 5);
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(misc);
-  volatile int *s_abort = reinterpret_cast<volatile int *>(misc + 4);
-  int *s_flag = reinterpret_cast<int *>(misc + 8);
-  int *s_prefix = reinterpret_cast<int *>(misc + 16);          // [groups + 1]
-  int *s_mblocks = s_prefix + (SCHED == kMasked ? p.groups + 1 : 0);  // [groups]
+  const uint32_t bars = base + L::kBarOff;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
+  auto afull_bar = [&](int s) { return bars + 8u * (2 * STAGES + s); };
+  auto aempty_bar = [&](int s) { return bars + 8u * (2 * STAGES + kAlphaSlots + s); };
+  auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 * kAlphaSlots + b); };
+  auto tempty_bar = [&](int b) {
+    return bars + 8u * (2 * STAGES + 2 * kAlphaSlots + NBUF + b);
+  };
+  const uint32_t drain_bar = bars + 8u * (L::kNumBars - 1);
+  const float *s_alpha = reinterpret_cast<const float *>(smem + L::kAlphaOff);
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+  int *s_flag = reinterpret_cast<int *>(smem + L::kMiscOff + 8);
+  int *s_prefix = reinterpret_cast<int *>(smem + L::kPrefixOff);        // [groups + 1]
+  int *s_mblocks = s_prefix + (SCHED == kMasked ? p.groups + 1 : 0);   // [groups]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -194,7 +219,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int s = 0; s < kAlphaSlots; ++s) {
+      mbar_init(afull_bar(s), 1);
+      mbar_init(aempty_bar(s), kPromoWarps);
+    }
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(tfull_bar(b), 1);
       mbar_init(tempty_bar(b), kPromoWarps);
     }
@@ -209,21 +238,19 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   }
   if constexpr (SCHED == kMasked) {
     if (warp == 2) {
-      // prefix[e] = sum_{e' < e} ceil(clamp(masked_m[e'])/128) * n_blocks
+      // prefix[e] = sum_{e' < e} ceil(clamp(masked_m[e']) / 128) * n_blocks
       int running = 0;
       for (int e0 = 0; e0 < p.groups; e0 += 32) {
         const int e = e0 + lane;
         int mb = 0;
         if (e < p.groups) {
-          int m = __ldg(p.masked_m + e);
-          if (m < 0 || m > p.rows) {
-            record_status(p.status, DG_ERR_DEVICE_DATA);
-            m = m < 0 ? 0 : p.rows;
-          }
-          mb = (m + BM - 1) / BM;
+          const int m = __ldg(p.masked_m + e);
+          if (m < 0 || m > p.rows) record_status(p.status, DG_ERR_DEVICE_DATA);
+          mb = (masked_rows(p, e) + BM - 1) / BM;
           s_mblocks[e] = mb;
         }
-        int v = mb * p.num_n_blocks, incl = v;
+        const int v = mb * p.num_n_blocks;
+        int incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int t = __shfl_up_sync(0xffffffffu, incl, o);
@@ -240,6 +267,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int units = num_units(p, SCHED, s_prefix);
+  const int kg_total = p.num_k_blocks;
 
   if (warp == 0) {
     // ============================================================ producer
@@ -252,15 +280,26 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (t.group < 0) continue;
       }
       const int a_row = t.m_blk * BM, b_row = t.n_blk * BN;
+      // alpha slice of this M block: rows a_row .. a_row+127 of the MN-major
+      // array, clipped to the leading dimension (a multiple of 4 floats)
+      const int64_t a_avail = p.ld_sfa - a_row;
+      const uint32_t a_bytes = static_cast<uint32_t>(4 * (a_avail < BM ? a_avail : BM));
+      const float *a_src = p.sfa + static_cast<int64_t>(t.slab) * kg_total * p.ld_sfa + a_row;
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
+        const int as = it % kAlphaSlots;
+        const uint32_t aph = (it / kAlphaSlots) & 1;
         if (!mbar_wait(empty_bar(s), ph ^ 1, s_abort, p.status)) { alive = false; break; }
+        if (!mbar_wait(aempty_bar(as), aph ^ 1, s_abort, p.status)) { alive = false; break; }
         if (lane == 0) {
           const uint32_t sa = base + s * L::kStageBytes;
           mbar_arrive_expect_tx(full_bar(s), L::kStageBytes);
           tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, t.slab);
           tma_load_3d(sa + kABytes, &tmap_b, full_bar(s), kb * BK, b_row, t.group);
+          mbar_arrive_expect_tx(afull_bar(as), a_bytes);
+          bulk_load(base + L::kAlphaOff + as * (BM * 4), a_src + static_cast<int64_t>(kb) * p.ld_sfa,
+                    a_bytes, afull_bar(as));
         }
         __syncwarp();
       }
@@ -278,9 +317,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it, ++acc_it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        const int buf = acc_it & 1;
-        const uint32_t aph = (acc_it >> 1) & 1;
-        if (!mbar_wait(tempty_bar(buf), aph ^ 1, s_abort, p.status)) { alive = false; break; }
+        const int buf = acc_it % NBUF;
+        const uint32_t bph = (acc_it / NBUF) & 1;
+        if (!mbar_wait(tempty_bar(buf), bph ^ 1, s_abort, p.status)) { alive = false; break; }
         if (!mbar_wait(full_bar(s), ph, s_abort, p.status)) { alive = false; break; }
         tc_fence_after();
         if (lane == 0) {
@@ -300,22 +339,21 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         __syncwarp();
       }
     }
-    // make sure every MMA issued above has completed before TMEM is freed
-    // (bounded, and not cut short by the abort flag)
+    // every MMA issued above must complete before TMEM is freed (bounded, and
+    // not cut short by the abort flag)
     if (lane == 0) umma_commit(drain_bar);
     __syncwarp();
     volatile int never = 0;
     mbar_wait(drain_bar, 0, &never, p.status);
-  } else if (warp >= 4) {
+  } else if (warp >= kControlWarps) {
     // ============================================================ promotion
-    const int pw = warp - 4;           // 0..7
-    const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31
-    const int half = pw >> 2;          // column half of the tile
+    const int pw = warp - kControlWarps;   // 0..7
+    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
+    const int half = pw >> 2;              // column half of the tile
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
     const int nb_total = (p.n + 127) / 128;
-    const int kg_total = p.num_k_blocks;
-    int acc_it = 0;
+    int it = 0;
     bool alive = true;
     for (int u = blockIdx.x; u < units && alive; u += gridDim.x) {
       Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
@@ -326,16 +364,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (t.group < 0) continue;
         row_ok = row < p.rows && __ldg(p.m_indices + row) == t.group;
       } else if constexpr (SCHED == kMasked) {
-        int m = __ldg(p.masked_m + t.slab);
-        m = m < 0 ? 0 : (m > p.rows ? p.rows : m);
-        row_ok = row < m;
+        row_ok = row < masked_rows(p, t.slab);
       } else {
         row_ok = row < p.rows;
       }
       const int col0 = t.n_blk * BN + half * W;  // first column of this thread
-      const int row_c = row < p.rows ? row : p.rows - 1;
-      const float *sfa_ptr =
-          p.sfa + static_cast<int64_t>(t.slab) * kg_total * p.ld_sfa + row_c;
+      // a thread's W columns (W divides 128 or equals 128) lie in one beta block
       const int nb = min(col0, p.n - 1) / 128;
       const float *sfb_ptr =
           p.sfb + (static_cast<int64_t>(t.group) * nb_total + nb) * kg_total;
@@ -344,28 +378,39 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
       for (int c = 0; c < W; ++c) acc[c] = 0.0f;
 
-      float a_next = __ldg(sfa_ptr + static_cast<int64_t>(t.k_begin) * p.ld_sfa);
       float b_next = __ldg(sfb_ptr + t.k_begin);
-      for (int kb = t.k_begin; kb < t.k_end; ++kb, ++acc_it) {
-        const float a_cur = a_next, b_cur = b_next;
-        if (kb + 1 < t.k_end) {
-          a_next = __ldg(sfa_ptr + static_cast<int64_t>(kb + 1) * p.ld_sfa);
-          b_next = __ldg(sfb_ptr + kb + 1);
+      for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
+        const float b_cur = b_next;
+        if (kb + 1 < t.k_end) b_next = __ldg(sfb_ptr + kb + 1);
+        const int as = it % kAlphaSlots;
+        const int buf = it % NBUF;
+        if (!mbar_wait(afull_bar(as), (it / kAlphaSlots) & 1, s_abort, p.status)) {
+          alive = false;
+          break;
         }
-        const int buf = acc_it & 1;
-        const uint32_t aph = (acc_it >> 1) & 1;
-        if (!mbar_wait(tfull_bar(buf), aph, s_abort, p.status)) { alive = false; break; }
-        tc_fence_after();
-        uint32_t r[W];
-        tmem_ld<W>(tmem_base + t_lane + buf * BN + half * W, r);
-        tmem_wait_ld();
-        reg_barrier<W>(r);
-        tc_fence_before();
+        const float sc = s_alpha[as * BM + row_in_tile] * b_cur;
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(buf));
-        const float sc = a_cur * b_cur;
+        if (lane == 0) mbar_arrive(aempty_bar(as));
+        if (!mbar_wait(tfull_bar(buf), (it / NBUF) & 1, s_abort, p.status)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < W; ++c) acc[c] = fmaf(__uint_as_float(r[c]), sc, acc[c]);
+        for (int c0 = 0; c0 < W; c0 += LW) {
+          uint32_t r[LW];
+          tmem_ld<LW>(tmem_base + t_lane + buf * BN + half * W + c0, r);
+          tmem_wait_ld();
+          reg_barrier<LW>(r);
+          if (c0 + LW == W) {
+            // all of this buffer has been read: hand it back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(buf));
+          }
+#pragma unroll
+          for (int c = 0; c < LW; ++c) acc[c0 + c] = fmaf(__uint_as_float(r[c]), sc, acc[c0 + c]);
+        }
       }
       if (!alive) break;
 
@@ -382,7 +427,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                  make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
         __threadfence();
         asm volatile("bar.sync 1, %0;" ::"n"(kPromoThreads) : "memory");
-        if (threadIdx.x == 4 * 32) {
+        if (threadIdx.x == kControlWarps * 32) {
           const uint32_t prev = atomicAdd(p.ws_ticket + tile, 1u);
           const int last = prev == static_cast<uint32_t>(p.splits - 1);
           if (last) p.ws_ticket[tile] = 0;  // ready for the next call
@@ -430,24 +475,24 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 }
 
 // ------------------------------------------------------------------ host side
-template <int BN, int STAGES>
-constexpr int smem_bytes_for(int groups_extra) {
-  return 1024 + STAGES * Layout<BN>::kStageBytes + 8 * (2 * STAGES + 5) + 16 +
-         groups_extra;
+struct Candidate {
+  int bn, stages, nbuf;
+};
+// N tiles and their pipeline depths: 4-6 stages keep ~200 KB of operands in
+// flight; NBUF fills the 512 TMEM columns (at most 8 buffers).
+constexpr Candidate kCandidates[] = {
+    {256, 4, 2}, {128, 6, 4}, {64, 8, 8}, {32, 8, 8}, {16, 8, 8}};
+
+template <int BN, int STAGES, int NBUF>
+constexpr int smem_bytes_for(int extra) {
+  return 1024 + Layout<BN, STAGES, NBUF>::kPrefixOff + extra;
 }
 
-struct Candidate {
-  int bn;
-  int stages;
-};
-constexpr Candidate kCandidates[] = {{128, 6}, {64, 8}, {32, 8}, {16, 8}};
-
-template <int BN, int STAGES, int SCHED>
-int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb,
-                    const GemmParams &p, int grid, int extra_smem,
-                    cudaStream_t stream) {
-  const int smem = smem_bytes_for<BN, STAGES>(extra_smem);
-  auto kern = fp8_gemm_kernel<BN, STAGES, SCHED>;
+template <int BN, int STAGES, int NBUF, int SCHED>
+int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+                    int grid, int extra_smem, cudaStream_t stream) {
+  const int smem = smem_bytes_for<BN, STAGES, NBUF>(extra_smem);
+  auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED>;
   static int configured_smem[64] = {0};  // per device; grows only
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DG_ERR_CUDA;
@@ -462,27 +507,27 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb,
 }
 
 template <int SCHED>
-int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb,
-             const GemmParams &p, int grid, int extra, cudaStream_t st) {
+int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+             int grid, int extra, cudaStream_t st) {
   switch (bn) {
-    case 128: return launch_instance<128, 6, SCHED>(ta, tb, p, grid, extra, st);
-    case 64: return launch_instance<64, 8, SCHED>(ta, tb, p, grid, extra, st);
-    case 32: return launch_instance<32, 8, SCHED>(ta, tb, p, grid, extra, st);
-    case 16: return launch_instance<16, 8, SCHED>(ta, tb, p, grid, extra, st);
+    case 256: return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st);
+    case 128: return launch_instance<128, 6, 4, SCHED>(ta, tb, p, grid, extra, st);
+    case 64: return launch_instance<64, 8, 8, SCHED>(ta, tb, p, grid, extra, st);
+    case 32: return launch_instance<32, 8, 8, SCHED>(ta, tb, p, grid, extra, st);
+    case 16: return launch_instance<16, 8, 8, SCHED>(ta, tb, p, grid, extra, st);
     default: return DG_ERR_INVALID_ARG;
   }
 }
 
 // 3-D tensor map over an E4M3 tensor [dim2][dim1][K] with a box of
 // [1][box_rows][128] and the 128-byte swizzle.
-int make_tmap(CUtensorMap *m, const void *ptr, int64_t k, int64_t rows,
-              int64_t slabs, int box_rows) {
+int make_tmap(CUtensorMap *m, const void *ptr, int64_t k, int64_t rows, int64_t slabs,
+              int box_rows) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return DG_ERR_CUDA;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(slabs)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(k),
-                                 static_cast<cuuint64_t>(k * rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(k * rows)};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims,
@@ -493,49 +538,46 @@ int make_tmap(CUtensorMap *m, const void *ptr, int64_t k, int64_t rows,
 }
 
 bool print_configs() {
-  static const int v = [] {
-    const char *e = getenv("DG_PRINT_CONFIGS");
-    return (e && *e && *e != '0') ? 1 : 0;
-  }();
-  return v != 0;
+  const char *e = getenv("DG_PRINT_CONFIGS");
+  return e && *e && *e != '0';
 }
 
-// Estimated time (arbitrary units) of a config: waves x per-tile time, with
-// per-tile time the larger of tensor time and operand-feed time per K block,
-// and a floor from streaming every distinct byte once through HBM.
-double estimate(int64_t m_blocks, int64_t n, int64_t k, int bn, int splits,
-                int sms) {
+// Estimated time (SM cycles) of a config: waves x per-unit time, with per-unit
+// time the larger of tensor time and operand-feed time per K block plus a
+// fixed tile overhead, and a floor from streaming the distinct bytes once
+// through HBM.
+double estimate(int64_t m_blocks, int64_t n, int64_t k, int bn, int splits, int sms) {
   const int64_t n_blocks = (n + bn - 1) / bn;
   const int64_t units = m_blocks * n_blocks * splits;
   const int64_t waves = (units + sms - 1) / sms;
   const double kb = static_cast<double>(k / BK) / splits;
-  // cycles per K block: MMA 128 x bn x 128 at ~8192 MAC/clk; operand feed
-  // (16 KB + bn*128 B) at ~64 B/clk from L2; fixed ~120 cycles of latency.
-  const double mma = 2.0 * bn;
-  const double feed = (16384.0 + 128.0 * bn) / 64.0;
-  const double per_tile = kb * std::max(mma, feed) + 400.0 + 4.0 * bn;
-  double t = waves * per_tile;
-  // HBM floor: B once + A once, at ~23 B/clk/SM aggregated over all SMs
+  const double mma = 2.0 * bn;                             // 128 x bn x 128 / 8192 per clk
+  const double feed = (16384.0 + 128.0 * bn) / 96.0;       // smem fill rate from L2
+  const double per_unit = kb * std::max(mma, feed) + 800.0 + 4.0 * bn;
+  double t = waves * per_unit;
   const double bytes = static_cast<double>(n) * k + m_blocks * 128.0 * k;
-  t = std::max(t, bytes / (23.0 * sms));
-  if (splits > 1) t += 600.0;  // reduction pass and its latency
+  t = std::max(t, bytes / (23.0 * sms));                   // ~6.5 TB/s of HBM
+  if (splits > 1) t += 800.0;                              // reduction pass
   return t;
+}
+
+size_t split_ws_bytes(int64_t tiles, int splits, int bn) {
+  return static_cast<size_t>(tiles) * splits * BM * bn * 4 + tiles * 4;
 }
 
 }  // namespace
 
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int num_sms) {
   (void)num_sms;
+  (void)K;
   if (M <= 0 || M > 2 * BM) return 0;
-  // largest possible split-K footprint: BN 16, up to 8 splits
+  // largest split-K footprint over the candidates, up to 8 splits
   const int64_t m_blocks = (M + BM - 1) / BM;
   size_t best = 0;
   for (const Candidate &c : kCandidates) {
     const int64_t tiles = m_blocks * ((N + c.bn - 1) / c.bn);
-    const size_t bytes = static_cast<size_t>(tiles) * 8 * BM * c.bn * 4 + tiles * 4 + 16;
-    best = std::max(best, bytes);
+    best = std::max(best, split_ws_bytes(tiles, 8, c.bn) + 16);
   }
-  (void)K;
   return (best + 255) & ~static_cast<size_t>(255);
 }
 
@@ -548,19 +590,15 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   // ------------------------------------------------ choose BN (and splits)
   int bn = 128, splits = 1;
   double best = 1e300;
-  const int64_t m_blocks_eff = sched == kMasked ? p.num_m_blocks * p.groups : p.num_m_blocks;
-  const int64_t n_eff = sched == kDense ? n : n;  // B per expert
+  const int64_t m_blocks_eff =
+      sched == kMasked ? static_cast<int64_t>(p.num_m_blocks) * p.groups : p.num_m_blocks;
   for (const Candidate &c : kCandidates) {
     for (int s = 1; s <= 8; s *= 2) {
       if (s > 1 && (sched != kDense || ws == nullptr || p.num_m_blocks > 2)) break;
       if (s > p.num_k_blocks) break;
-      const int64_t tiles = p.num_m_blocks * ((n + c.bn - 1) / c.bn);
-      if (s > 1) {
-        const size_t need = static_cast<size_t>(tiles) * s * BM * c.bn * 4 + tiles * 4;
-        if (need > ws_bytes) break;
-      }
-      double e = estimate(m_blocks_eff, n_eff, k, c.bn, s, num_sms);
-      if (sched == kMasked) e = estimate(m_blocks_eff, n, k, c.bn, s, num_sms);
+      const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * ((n + c.bn - 1) / c.bn);
+      if (s > 1 && split_ws_bytes(tiles, s, c.bn) > ws_bytes) break;
+      const double e = estimate(m_blocks_eff, n, k, c.bn, s, num_sms);
       if (e < best * 0.97) {
         best = e;
         bn = c.bn;
@@ -579,8 +617,8 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
     const int v = atoi(e);
     if (v >= 1) {
       const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * ((n + bn - 1) / bn);
-      const size_t need = static_cast<size_t>(tiles) * v * BM * bn * 4 + tiles * 4;
-      if (v > 1 && (sched != kDense || ws == nullptr || need > ws_bytes || v > p.num_k_blocks))
+      if (v > 1 && (sched != kDense || ws == nullptr || split_ws_bytes(tiles, v, bn) > ws_bytes ||
+                    v > p.num_k_blocks))
         return DG_ERR_WORKSPACE;
       splits = v;
     }
@@ -600,8 +638,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
 
   // ------------------------------------------------ tensor maps
   CUtensorMap ta, tb;
-  const int64_t a_slabs = sched == kMasked ? p.groups : 1;
-  int rc = make_tmap(&ta, A, k, rows, a_slabs, BM);
+  int rc = make_tmap(&ta, A, k, rows, sched == kMasked ? p.groups : 1, BM);
   if (rc) return rc;
   rc = make_tmap(&tb, B, k, n, sched == kDense ? 1 : p.groups, bn);
   if (rc) return rc;
@@ -610,7 +647,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   int64_t units;
   int extra = 0;
   if (sched == kMasked) {
-    units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks * p.groups;  // upper bound
+    units = m_blocks_eff * p.num_n_blocks;  // upper bound; actual from masked_m
     extra = 8 * (p.groups + 1);
   } else {
     units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks * splits;
@@ -618,11 +655,10 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
   if (print_configs()) {
     fprintf(stderr,
-            "[dg] gemm sched=%d rows=%lld n=%lld k=%lld groups=%d: BN=%d splits=%d "
-            "grid=%d units=%lld\n",
+            "[dg] gemm sched=%d rows=%lld n=%lld k=%lld groups=%d: BN=%d splits=%d grid=%d "
+            "units=%lld\n",
             sched, static_cast<long long>(rows), static_cast<long long>(n),
-            static_cast<long long>(k), p.groups, bn, splits, grid,
-            static_cast<long long>(units));
+            static_cast<long long>(k), p.groups, bn, splits, grid, static_cast<long long>(units));
   }
   switch (sched) {
     case kDense: return dispatch<kDense>(bn, ta, tb, p, grid, extra, stream);

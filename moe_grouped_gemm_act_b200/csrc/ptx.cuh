@@ -114,6 +114,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap,
       : "memory");
 }
 
+// 1-D bulk copy global -> shared, completing on mbarrier `bar`.  Both
+// addresses 16-byte aligned, `bytes` a positive multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src,
+                                          uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], "
+      "[%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 // Allocates `ncols` TMEM columns (power of two >= 32); the base address is
 // written to shared memory at `dst`.  Whole warp.

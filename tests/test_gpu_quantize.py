@@ -48,6 +48,50 @@ def test_1x128_edge_cases_bit_exact(pow2):
     assert np.array_equal(sf.T.view(np.uint32), a0.view(np.uint32))
 
 
+def near_midpoint_rows(rows=64, k=1024, seed=0):
+    """Groups whose quotients x / alpha sit within a few float32 ulps of E4M3
+    rounding midpoints, for scales that are not powers of two: these decide
+    whether the device quotient is the correctly rounded one."""
+    from oracle import e4m3
+    g = np.random.default_rng(seed)
+    pos = e4m3.DECODE[:0x7F]
+    mids = ((pos[:-1] + pos[1:]) / 2)
+    out = np.zeros((rows, k), np.float32)
+    for r in range(rows):
+        for grp in range(k // 128):
+            amax = np.float32(g.uniform(0.5, 2.0) * 10.0 ** g.integers(-20, 20))
+            s = amax / np.float32(448.0)                    # float32 division, RN
+            m = g.choice(mids, size=127) * g.choice([-1, 1], size=127)
+            x = (m * np.float64(s)).astype(np.float32)       # near m * s
+            x = np.nextafter(x, np.float32(np.inf) * np.sign(x),
+                             dtype=np.float32) if r % 3 == 1 else x
+            x = np.nextafter(x, np.float32(0), dtype=np.float32) if r % 3 == 2 else x
+            x = np.clip(x, -amax, amax)
+            out[r, grp * 128] = amax
+            out[r, grp * 128 + 1:(grp + 1) * 128] = x
+    return out
+
+
+@pytest.mark.parametrize("pow2", [False, True])
+def test_1x128_near_midpoints_bit_exact(pow2):
+    x = near_midpoint_rows()
+    q, sf = run_1x128(x, pow2)
+    q0, a0 = quant.quantize_1x128(x, pow2=pow2)
+    assert np.array_equal(sf.T.view(np.uint32), a0.view(np.uint32))
+    assert np.array_equal(q, q0)
+
+
+def test_1x128_wide_dynamic_range_bit_exact():
+    x = inputs.activations(512, 1024, seed=21, outliers=True)
+    g = np.random.default_rng(4)
+    x *= (10.0 ** g.uniform(-38, 36, size=(512, 1))).astype(np.float32)
+    x[5, :128] *= np.float32(1e-10)              # subnormal inputs and scales
+    q, sf = run_1x128(x)
+    q0, a0 = quant.quantize_1x128(x)
+    assert np.array_equal(sf.T.view(np.uint32), a0.view(np.uint32))
+    assert np.array_equal(q, q0)
+
+
 @pytest.mark.parametrize("m,k", [(1, 128), (3, 384), (128, 512), (300, 1024), (1000, 7168)])
 @pytest.mark.parametrize("pow2", [False, True])
 def test_1x128_random_bit_exact(m, k, pow2):
