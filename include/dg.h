@@ -156,8 +156,10 @@ int dg_fp8_gemm_nt(const uint8_t *A, const float *sfa, int64_t ld_sfa,
                    int64_t N, int64_t K, void *workspace,
                    size_t workspace_bytes, dg_stream_t stream);
 
-/* Workspace size in bytes that lets dg_fp8_gemm_nt use its split-K path for
- * this shape (0 when the shape never splits).  16-byte aligned. */
+/* Workspace size in bytes with which dg_fp8_gemm_nt uses the K split its
+ * tile heuristic prefers for this shape on the current device (0 when that
+ * choice does not split K; the result depends on the SM count in effect,
+ * see dg_set_num_sms).  A multiple of 256 bytes. */
 size_t dg_fp8_gemm_nt_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*

@@ -162,7 +162,9 @@ int dg_quantize_128x128(const float *w, int64_t G, int64_t N, int64_t K, uint8_t
 
 size_t dg_fp8_gemm_nt_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
-  return gemm_workspace_size(M, N, K, 0);
+  int sms = effective_num_sms();
+  if (sms <= 0) sms = 148;  // no usable device: size for a full B200
+  return gemm_workspace_size(M, N, K, sms);
 }
 
 int dg_fp8_gemm_nt(const uint8_t *A, const float *sfa, int64_t ld_sfa, const uint8_t *B,

@@ -565,20 +565,45 @@ size_t split_ws_bytes(int64_t tiles, int splits, int bn) {
   return static_cast<size_t>(tiles) * splits * BM * bn * 4 + tiles * 4;
 }
 
+struct Choice {
+  int bn, splits;
+};
+
+// Tile width and K split for a launch.  Splitting K is considered for dense
+// shapes of at most two M blocks, and only when the workspace can hold the
+// split's FP32 partials (`ws_bytes`).
+Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, int num_sms,
+                     size_t ws_bytes) {
+  const int64_t m_blocks = (rows + BM - 1) / BM;
+  const int64_t k_blocks = k / BK;
+  const int64_t m_blocks_eff = sched == kMasked ? m_blocks * groups : m_blocks;
+  Choice c{128, 1};
+  double best = 1e300;
+  for (const Candidate &cand : kCandidates) {
+    for (int s = 1; s <= 8; s *= 2) {
+      if (s > 1 && (sched != kDense || m_blocks > 2)) break;
+      if (s > k_blocks) break;
+      const int64_t tiles = m_blocks * ((n + cand.bn - 1) / cand.bn);
+      if (s > 1 && split_ws_bytes(tiles, s, cand.bn) > ws_bytes) break;
+      const double e = estimate(m_blocks_eff, n, k, cand.bn, s, num_sms);
+      if (e < best * 0.97) {
+        best = e;
+        c = {cand.bn, s};
+      }
+    }
+  }
+  return c;
+}
+
 }  // namespace
 
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int num_sms) {
-  (void)num_sms;
-  (void)K;
-  if (M <= 0 || M > 2 * BM) return 0;
-  // largest split-K footprint over the candidates, up to 8 splits
-  const int64_t m_blocks = (M + BM - 1) / BM;
-  size_t best = 0;
-  for (const Candidate &c : kCandidates) {
-    const int64_t tiles = m_blocks * ((N + c.bn - 1) / c.bn);
-    best = std::max(best, split_ws_bytes(tiles, 8, c.bn) + 16);
-  }
-  return (best + 255) & ~static_cast<size_t>(255);
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  // the split the heuristic picks when the workspace is not a constraint
+  const Choice c = choose_config(kDense, M, N, K, 1, num_sms, ~static_cast<size_t>(0));
+  if (c.splits <= 1) return 0;
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + c.bn - 1) / c.bn);
+  return (split_ws_bytes(tiles, c.splits, c.bn) + 255) & ~static_cast<size_t>(255);
 }
 
 int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
@@ -586,26 +611,13 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   const int64_t rows = p.rows, n = p.n, k = p.k;
   p.num_m_blocks = static_cast<int>((rows + BM - 1) / BM);
   p.num_k_blocks = static_cast<int>(k / BK);
-
-  // ------------------------------------------------ choose BN (and splits)
-  int bn = 128, splits = 1;
-  double best = 1e300;
+  if (ws == nullptr) ws_bytes = 0;
   const int64_t m_blocks_eff =
       sched == kMasked ? static_cast<int64_t>(p.num_m_blocks) * p.groups : p.num_m_blocks;
-  for (const Candidate &c : kCandidates) {
-    for (int s = 1; s <= 8; s *= 2) {
-      if (s > 1 && (sched != kDense || ws == nullptr || p.num_m_blocks > 2)) break;
-      if (s > p.num_k_blocks) break;
-      const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * ((n + c.bn - 1) / c.bn);
-      if (s > 1 && split_ws_bytes(tiles, s, c.bn) > ws_bytes) break;
-      const double e = estimate(m_blocks_eff, n, k, c.bn, s, num_sms);
-      if (e < best * 0.97) {
-        best = e;
-        bn = c.bn;
-        splits = s;
-      }
-    }
-  }
+
+  // ------------------------------------------------ choose BN (and splits)
+  const Choice choice = choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes);
+  int bn = choice.bn, splits = choice.splits;
   // Tuning / test overrides: DG_BLOCK_N forces the N tile, DG_SPLITS the K
   // split (dense only; needs enough workspace).
   if (const char *e = getenv("DG_BLOCK_N")) {

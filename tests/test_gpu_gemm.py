@@ -51,8 +51,10 @@ def run_dense(qa, alpha, qb, beta, workspace=False):
     d = torch.full((m, n), 0, dtype=torch.int16, device="cuda").view(torch.bfloat16)
     ws = None
     if workspace:
-        nbytes = dg.dg_fp8_gemm_nt_workspace_size(m, n, qa.shape[1])
-        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
+        # room for any forced split (tiles x splits x 128 x BN FP32 + tickets)
+        nbytes = max(dg.dg_fp8_gemm_nt_workspace_size(m, n, qa.shape[1]),
+                     -(-m // 128) * (n + 256) * 8 * 128 * 4 + (1 << 16))
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     dg.dg_fp8_gemm_nt(dev(qa), sfa_to_device(alpha), dev(qb), dev(beta), d, workspace=ws)
     torch.cuda.synchronize()
     assert dg.dg_get_device_status() == 0
