@@ -163,6 +163,35 @@ int dg_fp8_gemm_nt(const uint8_t *A, const float *sfa, int64_t ld_sfa,
 size_t dg_fp8_gemm_nt_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
+ * dg_fp8_gemm_nt_noalloc -- dg_fp8_gemm_nt for callers that cannot allocate
+ * device memory.  The pages have no counterpart to this entry point.
+ *
+ * Who needs it: a runtime that reserves all device memory at start-up and
+ * forbids later allocation, a plugin whose host framework owns every buffer
+ * and passes in only inputs and outputs, or a latency-critical loop that
+ * cannot pay for cudaMalloc's implicit device-wide synchronisation.  Such a
+ * caller cannot supply the split-K workspace dg_fp8_gemm_nt takes; here the
+ * scratch is a fixed 32 MiB array inside the library, placed on each device
+ * that loads the library's code and kept there until the process exits.
+ *
+ * Same computation, arguments, layouts and errors as dg_fp8_gemm_nt, minus
+ * the workspace.  Nothing is allocated and no allocating routine is called.
+ *   - Returns DG_ERR_WORKSPACE (nothing launched) when the shape's preferred
+ *     K split needs more than 32 MiB, i.e. when
+ *     dg_fp8_gemm_nt_workspace_size(M, N, K) > 32 MiB.
+ *   - The first call on a device looks up the array's device address (and
+ *     loads that code on the device); make that first call before any stream
+ *     capture.
+ *   - All calls share the one array and leave their partial sums in it; each
+ *     call clears the part that must start at zero before its kernel runs.
+ *     Calls whose kernels overlap on the GPU (unordered streams) race on the
+ *     array: order them.
+ */
+int dg_fp8_gemm_nt_noalloc(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                           const uint8_t *B, const float *sfb, void *D, int64_t M,
+                           int64_t N, int64_t K, dg_stream_t stream);
+
+/*
  * dg_m_grouped_fp8_gemm_nt_contiguous -- MoE m-grouped GEMM, contiguous
  * layout (Lesson 13, Fig. 13-3 "contiguous"; Deep dive, section 3).
  *

@@ -41,7 +41,8 @@ EXPORTS = [
     "dg_status_string", "dg_get_mk_alignment_for_contiguous_layout",
     "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms",
     "dg_quantize_1x128", "dg_quantize_128x128", "dg_fp8_gemm_nt",
-    "dg_fp8_gemm_nt_workspace_size", "dg_m_grouped_fp8_gemm_nt_contiguous",
+    "dg_fp8_gemm_nt_workspace_size", "dg_fp8_gemm_nt_noalloc",
+    "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_get_device_status",
 ]
 
@@ -74,6 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_quantize_128x128": (I, [P, I64, I64, I64, P, P, I, P]),
         "dg_fp8_gemm_nt": (I, [P, P, I64, P, P, P, I64, I64, I64, P, SZ, P]),
         "dg_fp8_gemm_nt_workspace_size": (SZ, [I64, I64, I64]),
+        "dg_fp8_gemm_nt_noalloc": (I, [P, P, I64, P, P, P, I64, I64, I64, P]),
         "dg_m_grouped_fp8_gemm_nt_contiguous":
             (I, [P, P, I64, P, P, P, P, I64, I64, I64, I, P]),
         "dg_m_grouped_fp8_gemm_nt_masked":
@@ -208,6 +210,22 @@ def dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace: torch.Tensor | None = None,
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d), m, n, k,
         _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "dg_fp8_gemm_nt")
+    return d
+
+
+def dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, d, stream=None) -> torch.Tensor:
+    """dg_fp8_gemm_nt without a caller-provided workspace, for callers that
+    cannot allocate device memory (see include/dg.h): the split-K scratch is
+    the library's own fixed 32 MiB per-device array.  Shapes whose preferred
+    split needs more raise DGError (DG_ERR_WORKSPACE).  Calls that overlap on
+    the GPU share that array and must be ordered."""
+    _need_cuda(a, sfa, b, sfb, d)
+    m, k = a.shape
+    n = b.shape[0]
+    rc = load_library().dg_fp8_gemm_nt_noalloc(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d), m, n, k,
+        _stream(stream))
+    _check(rc, "dg_fp8_gemm_nt_noalloc")
     return d
 
 
