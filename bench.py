@@ -197,15 +197,37 @@ class DenseData:
                 4 * (-(-n // 128)) * (k // 128) + 2 * self.m * n
         return tot
 
-    def step(self, gemm_events=None):
-        dg = self.dg
-        for i, s in enumerate(self.shapes):
-            dg.dg_quantize_1x128(s["a32"], q=s["qa"], sf=s["sfa"])
-            if gemm_events is not None:
-                gemm_events[i][0].record()
-            dg.dg_fp8_gemm_nt(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"], workspace=s["ws"])
-            if gemm_events is not None:
-                gemm_events[i][1].record()
+    def gemm(self, s):
+        self.dg.dg_fp8_gemm_nt(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"], workspace=s["ws"])
+
+    def step(self):
+        """One pass of the hot path: for every shape, quantize A, then GEMM."""
+        for s in self.shapes:
+            self.dg.dg_quantize_1x128(s["a32"], q=s["qa"], sf=s["sfa"])
+            self.gemm(s)
+
+    def capture(self):
+        """CUDA graphs of one step and of each shape's GEMM alone.  The
+        library is called once eagerly first (its per-device set-up must not
+        happen inside a capture); replaying removes host launch overhead, as a
+        serving loop would."""
+        import torch
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.step_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.step_graph):
+            self.step()
+        self.gemm_graphs = []
+        for s in self.shapes:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.gemm(s)
+            self.gemm_graphs.append(g)
+        torch.cuda.synchronize()
 
     def launches_per_step(self) -> int:
         return 2 * len(self.shapes)
@@ -333,26 +355,39 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         torch.cuda.synchronize()
 
     # ------------------------------------------------ device-resident timing
+    # Each step replays a CUDA graph of the whole step (quantize + GEMM for
+    # every shape); events on the replay stream bracket exactly K steps.
+    data.capture()
     nshape = len(data.shapes)
-    gemm_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(nshape)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clocks:
         for _ in range(args.warmup):
-            data.step()
+            data.step_graph.replay()
         barrier()
         clocks.mark_start()
         start.record()
-        for i in range(args.steps):
-            data.step(gemm_ev[i])
+        for _ in range(args.steps):
+            data.step_graph.replay()
         stop.record()
         torch.cuda.synchronize()
         clocks.mark_stop()
     barrier()
     total_ms = start.elapsed_time(stop)
-    gemm_ms = [sum(e0.elapsed_time(e1) for e0, e1 in gemm_ev[i]) for i in range(args.steps)]
-    per_shape_ms = [statistics.mean(gemm_ev[i][j][0].elapsed_time(gemm_ev[i][j][1])
-                                    for i in range(args.steps)) for j in range(nshape)]
+    # The dominant kernel alone: the shapes' GEMM graphs replayed round-robin
+    # (so each launch finds the other shapes' operands, not its own, in L2),
+    # as many launches per shape as timed steps, one event pair per launch.
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)] for _ in range(nshape)]
+    for g in data.gemm_graphs:
+        g.replay()
+    for i in range(args.steps):
+        for j, g in enumerate(data.gemm_graphs):
+            ev[j][i][0].record()
+            g.replay()
+            ev[j][i][1].record()
+    torch.cuda.synchronize()
+    per_shape_ms = [statistics.mean(a.elapsed_time(b) for a, b in ev[j]) for j in range(nshape)]
+    gemm_ms = [sum(per_shape_ms)] * args.steps
 
     # ------------------------------------------------ end-to-end timing
     data.make_host()

@@ -39,8 +39,10 @@
 //               from the per-row index; blocks holding only padding skipped;
 //   masked      per expert g, ceil(masked_m[g] / 128) row blocks x N blocks,
 //               counts read on the device (launch shape independent of them).
-// Dense small-M shapes may split K (units = tile x split); FP32 partials go to
-// a workspace and the last-arriving CTA of a tile reduces them in split order.
+// Dense small-M shapes may split K (units = tile x split, one unit per CTA,
+// cooperative launch): FP32 partials go to a workspace, the splits of a tile
+// wait for each other on an arrival counter and each reduces a share of the
+// tile in split order.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -68,9 +70,10 @@ constexpr int kAlphaSlots = 16;         // alpha ring depth (>= STAGES + NBUF)
 constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 
-template <int BN, int STAGES, int NBUF>
+template <int BN, int STAGES, int NBUF, bool PAIR>
 struct Layout {
-  static constexpr uint32_t kBBytes = BN * BK;
+  // the pair form keeps half of the B tile (BN/2 rows) in each CTA
+  static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kAlphaOff = STAGES * kStageBytes;
   static constexpr uint32_t kBarOff = kAlphaOff + kAlphaSlots * BM * 4;
@@ -172,12 +175,22 @@ __device__ __forceinline__ int masked_rows(const GemmParams &p, int e) {
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int BN, int STAGES, int NBUF, int SCHED>
+//
+// PAIR: a 2-CTA cluster computes a 256 x BN tile with cta_group::2 MMAs
+// (M = 256).  Each CTA loads its own 128 rows of A and half of the B tile
+// (BN/2 rows), so every SM pulls half of B from L2 instead of all of it; both
+// CTAs' TMA loads complete on rank 0's `full` barrier, rank 0 issues the MMAs
+// and commits to the `empty` / `tmem_full` barriers of both CTAs, and the
+// promotion warps of both CTAs release TMEM buffers on rank 0's `tmem_empty`
+// barrier.  Each CTA promotes and stores its own 128 rows.
+template <int BN, int STAGES, int NBUF, int SCHED, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
                 const GemmParams p) {
-  using L = Layout<BN, STAGES, NBUF>;
+  using L = Layout<BN, STAGES, NBUF, PAIR>;
+  constexpr int TM = PAIR ? 2 * BM : BM;   // rows per tile
+  static_assert(!PAIR || SCHED == kDense, "the pair form serves dense GEMMs");
   constexpr int W = BN / 2;                 // columns per promotion thread
   // columns per TMEM load chunk: the whole slice up to 64; for BN = 256 the
   // 128 accumulators leave room for 16-column chunks under 168 registers
@@ -210,6 +223,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0;   // 0 issues the pair's MMAs
+  const int u_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int u_stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   // ---------------------------------------------------------------- setup
   if (warp == 0 && lane == 0) {
@@ -225,7 +241,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), kPromoWarps);
+      mbar_init(tempty_bar(b), PAIR ? 2 * kPromoWarps : kPromoWarps);
     }
     mbar_init(drain_bar, 1);
     *s_abort = 0;
@@ -233,8 +249,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(s_tmem), L::kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(s_tmem), L::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(s_tmem), L::kTmemCols);
+      tmem_relinquish();
+    }
   }
   if constexpr (SCHED == kMasked) {
     if (warp == 2) {
@@ -264,6 +285,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int units = num_units(p, SCHED, s_prefix);
@@ -271,20 +293,29 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
   if (warp == 0) {
     // ============================================================ producer
+    // bytes per stage: the A box (128 rows, or 64 when M <= 64: the MMA then
+    // reads stale rows 64-127, which only reach output rows that are never
+    // stored) and the B box
+    const uint32_t stage_tx = static_cast<uint32_t>(p.a_box_rows) * BK + L::kBBytes;
     int it = 0;
     bool alive = true;
-    for (int u = blockIdx.x; u < units && alive; u += gridDim.x) {
+    for (int u = u_first; u < units && alive; u += u_stride) {
       Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
       if constexpr (SCHED == kContiguous) {
         t.group = block_expert(p, t.m_blk, true);
         if (t.group < 0) continue;
       }
-      const int a_row = t.m_blk * BM, b_row = t.n_blk * BN;
+      const int a_row = t.m_blk * TM + static_cast<int>(rank) * BM;
+      const int b_row = t.n_blk * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
       // alpha slice of this M block: rows a_row .. a_row+127 of the MN-major
-      // array, clipped to the leading dimension (a multiple of 4 floats)
-      const int64_t a_avail = p.ld_sfa - a_row;
+      // array, clipped to the leading dimension (a multiple of 4 floats).  In
+      // the pair form rank 1's rows may all lie past the end; it then copies
+      // the last 4 scales instead (its rows are never stored), keeping the
+      // copy inside the array and at least 16 bytes long.
+      const int64_t a_start = a_row <= p.ld_sfa - 4 ? a_row : p.ld_sfa - 4;
+      const int64_t a_avail = p.ld_sfa - a_start;
       const uint32_t a_bytes = static_cast<uint32_t>(4 * (a_avail < BM ? a_avail : BM));
-      const float *a_src = p.sfa + static_cast<int64_t>(t.slab) * kg_total * p.ld_sfa + a_row;
+      const float *a_src = p.sfa + static_cast<int64_t>(t.slab) * kg_total * p.ld_sfa + a_start;
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -294,9 +325,18 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (!mbar_wait(aempty_bar(as), aph ^ 1, s_abort, p.status)) { alive = false; break; }
         if (lane == 0) {
           const uint32_t sa = base + s * L::kStageBytes;
-          mbar_arrive_expect_tx(full_bar(s), L::kStageBytes);
-          tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, t.slab);
-          tma_load_3d(sa + kABytes, &tmap_b, full_bar(s), kb * BK, b_row, t.group);
+          if constexpr (PAIR) {
+            // both CTAs' stage bytes complete on rank 0's full barrier, whose
+            // single arrival (with the pair's byte count) comes from rank 0
+            const uint32_t fb = mapa_shared(full_bar(s), 0);
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2 * stage_tx);
+            tma_load_3d_pair(sa, &tmap_a, fb, kb * BK, a_row, t.slab);
+            tma_load_3d_pair(sa + kABytes, &tmap_b, fb, kb * BK, b_row, t.group);
+          } else {
+            mbar_arrive_expect_tx(full_bar(s), stage_tx);
+            tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, t.slab);
+            tma_load_3d(sa + kABytes, &tmap_b, full_bar(s), kb * BK, b_row, t.group);
+          }
           mbar_arrive_expect_tx(afull_bar(as), a_bytes);
           bulk_load(base + L::kAlphaOff + as * (BM * 4), a_src + static_cast<int64_t>(kb) * p.ld_sfa,
                     a_bytes, afull_bar(as));
@@ -306,10 +346,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+    // (in the pair form only rank 0 issues; rank 1's warp 1 idles)
+    constexpr uint32_t idesc = idesc_e4m3_f32(TM, BN);
     int it = 0, acc_it = 0;
-    bool alive = true;
-    for (int u = blockIdx.x; u < units && alive; u += gridDim.x) {
+    bool alive = rank == 0;
+    for (int u = u_first; u < units && alive; u += u_stride) {
       Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
       if constexpr (SCHED == kContiguous) {
         if (block_expert(p, t.m_blk, false) < 0) continue;
@@ -331,20 +372,40 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           for (int k = 0; k < BK / 32; ++k) {
             // +32 bytes along K inside the swizzled 128-byte row = +2 in the
             // descriptor's 16-byte address field
-            umma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+            if constexpr (PAIR) {
+              umma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+            } else {
+              umma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+            }
           }
-          umma_commit(empty_bar(s));
-          umma_commit(tfull_bar(buf));
+          if constexpr (PAIR) {
+            // free the stage and publish the buffer in both CTAs
+            umma_commit_pair(mapa_shared(empty_bar(s), 0));
+            umma_commit_pair(mapa_shared(empty_bar(s), 1));
+            umma_commit_pair(mapa_shared(tfull_bar(buf), 0));
+            umma_commit_pair(mapa_shared(tfull_bar(buf), 1));
+          } else {
+            umma_commit(empty_bar(s));
+            umma_commit(tfull_bar(buf));
+          }
         }
         __syncwarp();
       }
     }
-    // every MMA issued above must complete before TMEM is freed (bounded, and
-    // not cut short by the abort flag)
-    if (lane == 0) umma_commit(drain_bar);
-    __syncwarp();
-    volatile int never = 0;
-    mbar_wait(drain_bar, 0, &never, p.status);
+    if (rank == 0) {
+      // every MMA issued above must complete before TMEM is freed (bounded,
+      // and not cut short by the abort flag)
+      if (lane == 0) {
+        if constexpr (PAIR) {
+          umma_commit_pair(mapa_shared(drain_bar, 0));
+        } else {
+          umma_commit(drain_bar);
+        }
+      }
+      __syncwarp();
+      volatile int never = 0;
+      mbar_wait(drain_bar, 0, &never, p.status);
+    }
   } else if (warp >= kControlWarps) {
     // ============================================================ promotion
     const int pw = warp - kControlWarps;   // 0..7
@@ -353,11 +414,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
     const int nb_total = (p.n + 127) / 128;
+    // TMEM buffers are handed back on rank 0's barrier (the MMA issuer's)
+    const uint32_t tempty_target0 = PAIR ? mapa_shared(tempty_bar(0), 0) : tempty_bar(0);
     int it = 0;
     bool alive = true;
-    for (int u = blockIdx.x; u < units && alive; u += gridDim.x) {
+    for (int u = u_first; u < units && alive; u += u_stride) {
       Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
-      const int row = t.m_blk * BM + row_in_tile;
+      const int row = t.m_blk * TM + static_cast<int>(rank) * BM + row_in_tile;
       bool row_ok;
       if constexpr (SCHED == kContiguous) {
         t.group = block_expert(p, t.m_blk, false);
@@ -406,7 +469,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             // all of this buffer has been read: hand it back to the MMA warp
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(buf));
+            if (lane == 0) {
+              if constexpr (PAIR) {
+                mbar_arrive_cluster(tempty_target0 + 8u * buf);
+              } else {
+                mbar_arrive(tempty_bar(buf));
+              }
+            }
           }
 #pragma unroll
           for (int c = 0; c < LW; ++c) acc[c0 + c] = fmaf(__uint_as_float(r[c]), sc, acc[c0 + c]);
@@ -417,36 +486,71 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       // ---------------------------------------------------------- epilogue
       if (p.splits > 1) {
         if (*s_abort) break;
-        // write this split's FP32 partial; the last arriving CTA reduces
+        // Split K: every CTA of the tile writes its FP32 partial (valid rows
+        // only, as float4 slots [column / 4][row] so that a warp's 32 rows
+        // write 512 contiguous bytes), counts itself in on the tile's
+        // arrival counter and waits for all splits (the launch is
+        // cooperative, so they are all resident); then each split reduces its
+        // own 1/S share of the tile's slots, summing splits 0, 1, ... in
+        // order (deterministic), and stores that share as BF16.
         const int tile = u / p.splits;
-        float *mine = p.ws + ((static_cast<int64_t>(tile) * p.splits + t.split) * BM +
-                              row_in_tile) * BN + half * W;
+        constexpr int kTileSlots = BM * BN / 4;
+        float4 *part = reinterpret_cast<float4 *>(p.ws) +
+                       static_cast<int64_t>(tile) * p.splits * kTileSlots;
+        if (row_ok) {
 #pragma unroll
-        for (int c = 0; c < W; c += 4)
-          __stcg(reinterpret_cast<float4 *>(mine + c),
-                 make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
+          for (int c = 0; c < W; c += 4)
+            __stcg(part + static_cast<int64_t>(t.split) * kTileSlots +
+                       ((half * W + c) / 4) * BM + row_in_tile,
+                   make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
+        }
         __threadfence();
         asm volatile("bar.sync 1, %0;" ::"n"(kPromoThreads) : "memory");
-        if (threadIdx.x == kControlWarps * 32) {
-          const uint32_t prev = atomicAdd(p.ws_ticket + tile, 1u);
-          const int last = prev == static_cast<uint32_t>(p.splits - 1);
-          if (last) p.ws_ticket[tile] = 0;  // ready for the next call
-          *s_flag = last;
+        const int ptid = threadIdx.x - kControlWarps * 32;
+        if (ptid == 0) {
+          atomicAdd(p.ws_ticket + tile, 1u);
+          if (!wait_counter(p.ws_ticket + tile, static_cast<uint32_t>(p.splits), p.status))
+            *s_abort = 1;
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kPromoThreads) : "memory");
-        if (!*s_flag) continue;
+        if (*s_abort) break;
         __threadfence();
-#pragma unroll
-        for (int c = 0; c < W; ++c) acc[c] = 0.0f;
-        for (int s = 0; s < p.splits; ++s) {
-          const float *src = p.ws + ((static_cast<int64_t>(tile) * p.splits + s) * BM +
-                                     row_in_tile) * BN + half * W;
-#pragma unroll
-          for (int c = 0; c < W; c += 4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + c));
-            acc[c] += v.x; acc[c + 1] += v.y; acc[c + 2] += v.z; acc[c + 3] += v.w;
+        const int row0 = t.m_blk * TM + static_cast<int>(rank) * BM;
+        const int valid = min(BM, p.rows - row0);
+        const int slots = valid * (BN / 4);
+        const int share = (slots + p.splits - 1) / p.splits;
+        const int f_end = min(slots, (t.split + 1) * share);
+        for (int f = t.split * share + ptid; f < f_end; f += kPromoThreads) {
+          const int c4 = f / valid, r = f - c4 * valid;
+          const float4 *src = part + c4 * BM + r;
+          float4 sum = __ldcg(src);
+          int s = 1;
+          for (; s + 3 < p.splits; s += 4) {
+            // four independent loads in flight, added in split order
+            const float4 v0 = __ldcg(src + static_cast<int64_t>(s) * kTileSlots);
+            const float4 v1 = __ldcg(src + static_cast<int64_t>(s + 1) * kTileSlots);
+            const float4 v2 = __ldcg(src + static_cast<int64_t>(s + 2) * kTileSlots);
+            const float4 v3 = __ldcg(src + static_cast<int64_t>(s + 3) * kTileSlots);
+            sum.x += v0.x; sum.y += v0.y; sum.z += v0.z; sum.w += v0.w;
+            sum.x += v1.x; sum.y += v1.y; sum.z += v1.z; sum.w += v1.w;
+            sum.x += v2.x; sum.y += v2.y; sum.z += v2.z; sum.w += v2.w;
+            sum.x += v3.x; sum.y += v3.y; sum.z += v3.z; sum.w += v3.w;
+          }
+          for (; s < p.splits; ++s) {
+            const float4 v = __ldcg(src + static_cast<int64_t>(s) * kTileSlots);
+            sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+          }
+          const int col = t.n_blk * BN + 4 * c4;
+          if (col < p.n) {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z, sum.w);
+            uint2 v;
+            v.x = *reinterpret_cast<const uint32_t *>(&lo);
+            v.y = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(p.d + static_cast<int64_t>(row0 + r) * p.n + col) = v;
           }
         }
+        continue;  // this split's share of D is written
       }
       if (row_ok) {
         uint16_t *drow = p.d + (static_cast<int64_t>(t.slab) * p.rows + row) * p.n;
@@ -470,8 +574,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
+  // in the pair form neither CTA leaves (or frees TMEM) while rank 0's MMAs
+  // may still read the peer's shared memory: rank 0 drained them above
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, L::kTmemCols);
+  if (warp == 1) {
+    if constexpr (PAIR) {
+      tmem_dealloc_pair(tmem_base, L::kTmemCols);
+    } else {
+      tmem_dealloc(tmem_base, L::kTmemCols);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -482,17 +595,19 @@ struct Candidate {
 // flight; NBUF fills the 512 TMEM columns (at most 8 buffers).
 constexpr Candidate kCandidates[] = {
     {256, 4, 2}, {128, 6, 4}, {64, 8, 8}, {32, 8, 8}, {16, 8, 8}};
+// The pair form: 256 x 256 tiles, half of B per CTA (32 KB stages).
+constexpr Candidate kPairCandidate = {256, 6, 2};
 
-template <int BN, int STAGES, int NBUF>
+template <int BN, int STAGES, int NBUF, bool PAIR>
 constexpr int smem_bytes_for(int extra) {
-  return 1024 + Layout<BN, STAGES, NBUF>::kPrefixOff + extra;
+  return 1024 + Layout<BN, STAGES, NBUF, PAIR>::kPrefixOff + extra;
 }
 
-template <int BN, int STAGES, int NBUF, int SCHED>
+template <int BN, int STAGES, int NBUF, int SCHED, bool PAIR>
 int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
-                    int grid, int extra_smem, cudaStream_t stream) {
-  const int smem = smem_bytes_for<BN, STAGES, NBUF>(extra_smem);
-  auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED>;
+                    int grid, int extra_smem, cudaStream_t stream, bool coop) {
+  const int smem = smem_bytes_for<BN, STAGES, NBUF, PAIR>(extra_smem);
+  auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED, PAIR>;
   static int configured_smem[64] = {0};  // per device; grows only
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DG_ERR_CUDA;
@@ -502,19 +617,56 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
       return DG_ERR_CUDA;
     configured_smem[dev] = smem;
   }
-  kern<<<grid, kThreads, smem, stream>>>(ta, tb, p);
+  if (coop) {
+    // the splits of a tile wait for each other: all CTAs must be resident
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return DG_ERR_CUDA;
+  } else if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return DG_ERR_CUDA;
+  } else {
+    kern<<<grid, kThreads, smem, stream>>>(ta, tb, p);
+  }
   return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
 template <int SCHED>
-int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
-             int grid, int extra, cudaStream_t st) {
+int dispatch(int bn, bool pair, const CUtensorMap &ta, const CUtensorMap &tb,
+             const GemmParams &p, int grid, int extra, cudaStream_t st) {
+  const bool coop = p.splits > 1;
+  if (pair) {
+    if constexpr (SCHED == kDense) {
+      return launch_instance<kPairCandidate.bn, kPairCandidate.stages, kPairCandidate.nbuf,
+                             SCHED, true>(ta, tb, p, grid, extra, st, false);
+    }
+    return DG_ERR_INVALID_ARG;
+  }
   switch (bn) {
-    case 256: return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st);
-    case 128: return launch_instance<128, 6, 4, SCHED>(ta, tb, p, grid, extra, st);
-    case 64: return launch_instance<64, 8, 8, SCHED>(ta, tb, p, grid, extra, st);
-    case 32: return launch_instance<32, 8, 8, SCHED>(ta, tb, p, grid, extra, st);
-    case 16: return launch_instance<16, 8, 8, SCHED>(ta, tb, p, grid, extra, st);
+    case 256: return launch_instance<256, 4, 2, SCHED, false>(ta, tb, p, grid, extra, st, coop);
+    case 128: return launch_instance<128, 6, 4, SCHED, false>(ta, tb, p, grid, extra, st, coop);
+    case 64: return launch_instance<64, 8, 8, SCHED, false>(ta, tb, p, grid, extra, st, coop);
+    case 32: return launch_instance<32, 8, 8, SCHED, false>(ta, tb, p, grid, extra, st, coop);
+    case 16: return launch_instance<16, 8, 8, SCHED, false>(ta, tb, p, grid, extra, st, coop);
     default: return DG_ERR_INVALID_ARG;
   }
 }
@@ -542,23 +694,32 @@ bool print_configs() {
   return e && *e && *e != '0';
 }
 
-// Estimated time (SM cycles) of a config: waves x per-unit time, with per-unit
-// time the larger of tensor time and operand-feed time per K block plus a
-// fixed tile overhead, and a floor from streaming the distinct bytes once
-// through HBM.
+// Cycles one CTA spends per 128-K block of a unit, measured on B200.  The
+// tensor cores take ~540 cycles per block for any N up to 256 (one
+// 128 x N x 32 MMA per ~135 cycles), so narrow tiles waste them; the
+// MMA -> promotion -> MMA round trip through the TMEM buffers sets the rest.
+double kb_cycles(int bn) {
+  switch (bn) {
+    case 256: return 1240.0;
+    case 128: return 900.0;
+    case 64: return 770.0;
+    default: return 750.0;
+  }
+}
+
+// Estimated time (SM cycles) of a config: waves x per-unit time (K blocks x
+// kb_cycles + pipeline fill and epilogue + split-K reduction), floored by
+// streaming the distinct operand bytes once through HBM (~23 B/cycle/SM).
 double estimate(int64_t m_blocks, int64_t n, int64_t k, int bn, int splits, int sms) {
   const int64_t n_blocks = (n + bn - 1) / bn;
   const int64_t units = m_blocks * n_blocks * splits;
   const int64_t waves = (units + sms - 1) / sms;
-  const double kb = static_cast<double>(k / BK) / splits;
-  const double mma = 2.0 * bn;                             // 128 x bn x 128 / 8192 per clk
-  const double feed = (16384.0 + 128.0 * bn) / 96.0;       // smem fill rate from L2
-  const double per_unit = kb * std::max(mma, feed) + 800.0 + 4.0 * bn;
-  double t = waves * per_unit;
+  const int64_t kb = (k / BK + splits - 1) / splits;
+  double per_unit = kb * kb_cycles(bn) + 2500.0;
+  if (splits > 1) per_unit += 1500.0 + 300.0 * splits;
+  const double t = waves * per_unit;
   const double bytes = static_cast<double>(n) * k + m_blocks * 128.0 * k;
-  t = std::max(t, bytes / (23.0 * sms));                   // ~6.5 TB/s of HBM
-  if (splits > 1) t += 800.0;                              // reduction pass
-  return t;
+  return std::max(t, bytes / (23.0 * sms));
 }
 
 size_t split_ws_bytes(int64_t tiles, int splits, int bn) {
@@ -567,28 +728,34 @@ size_t split_ws_bytes(int64_t tiles, int splits, int bn) {
 
 struct Choice {
   int bn, splits;
+  bool pair;
 };
 
-// Tile width and K split for a launch.  Splitting K is considered for dense
-// shapes of at most two M blocks, and only when the workspace can hold the
-// split's FP32 partials (`ws_bytes`).
+// Tile form for a launch: a tile width and K split from the cost model.
+// Splitting K is considered for dense shapes of at most two M blocks, only
+// while all units fit in one wave of CTAs, and only when the workspace can
+// hold the split's FP32 partials
+// (`ws_bytes`).  The pair form (2-CTA clusters) is opt-in (DG_PAIR=1): on
+// B200 it halves each SM's B traffic but measured no faster than the single-
+// CTA 256-wide tile, both being bound by the TMEM round trip.
 Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, int num_sms,
                      size_t ws_bytes) {
   const int64_t m_blocks = (rows + BM - 1) / BM;
   const int64_t k_blocks = k / BK;
   const int64_t m_blocks_eff = sched == kMasked ? m_blocks * groups : m_blocks;
-  Choice c{128, 1};
+  Choice c{128, 1, false};
   double best = 1e300;
   for (const Candidate &cand : kCandidates) {
-    for (int s = 1; s <= 8; s *= 2) {
+    for (int s = 1; s <= 16; ++s) {
       if (s > 1 && (sched != kDense || m_blocks > 2)) break;
       if (s > k_blocks) break;
       const int64_t tiles = m_blocks * ((n + cand.bn - 1) / cand.bn);
+      if (s > 1 && tiles * s > num_sms) break;
       if (s > 1 && split_ws_bytes(tiles, s, cand.bn) > ws_bytes) break;
       const double e = estimate(m_blocks_eff, n, k, cand.bn, s, num_sms);
       if (e < best * 0.97) {
         best = e;
-        c = {cand.bn, s};
+        c = {cand.bn, s, false};
       }
     }
   }
@@ -609,32 +776,46 @@ size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int num_sms) {
 int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
                     cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws) {
   const int64_t rows = p.rows, n = p.n, k = p.k;
-  p.num_m_blocks = static_cast<int>((rows + BM - 1) / BM);
   p.num_k_blocks = static_cast<int>(k / BK);
   if (ws == nullptr) ws_bytes = 0;
-  const int64_t m_blocks_eff =
-      sched == kMasked ? static_cast<int64_t>(p.num_m_blocks) * p.groups : p.num_m_blocks;
 
-  // ------------------------------------------------ choose BN (and splits)
+  // ------------------------------------------------ choose the tile form
   const Choice choice = choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes);
   int bn = choice.bn, splits = choice.splits;
-  // Tuning / test overrides: DG_BLOCK_N forces the N tile, DG_SPLITS the K
-  // split (dense only; needs enough workspace).
+  bool pair = choice.pair;
+  // Tuning / test overrides: DG_PAIR=0/1 disables / forces the pair form
+  // (dense only), DG_BLOCK_N forces the N tile of the single-CTA form,
+  // DG_SPLITS the K split (dense, single-CTA; needs enough workspace).
+  if (const char *e = getenv("DG_PAIR")) {
+    if (*e == '0') {
+      if (pair) {
+        pair = false;
+        bn = 256;
+      }
+    } else if (*e == '1' && sched == kDense && num_sms >= 2) {
+      pair = true;
+      bn = kPairCandidate.bn;
+      splits = 1;
+    }
+  }
   if (const char *e = getenv("DG_BLOCK_N")) {
     const int v = atoi(e);
     for (const Candidate &c : kCandidates)
-      if (c.bn == v) bn = v;
+      if (c.bn == v && !pair) bn = v;
   }
   if (const char *e = getenv("DG_SPLITS")) {
     const int v = atoi(e);
-    if (v >= 1) {
-      const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * ((n + bn - 1) / bn);
+    if (v >= 1 && !pair) {
+      const int64_t tiles = ((rows + BM - 1) / BM) * ((n + bn - 1) / bn);
       if (v > 1 && (sched != kDense || ws == nullptr || split_ws_bytes(tiles, v, bn) > ws_bytes ||
                     v > p.num_k_blocks))
         return DG_ERR_WORKSPACE;
+      if (v > 1 && tiles * v > num_sms) return DG_ERR_INVALID_ARG;  // one unit per CTA
       splits = v;
     }
   }
+  const int tile_rows = pair ? 2 * BM : BM;
+  p.num_m_blocks = static_cast<int>((rows + tile_rows - 1) / tile_rows);
   p.num_n_blocks = static_cast<int>((n + bn - 1) / bn);
   p.splits = splits;
   if (splits > 1) {
@@ -650,32 +831,40 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
 
   // ------------------------------------------------ tensor maps
   CUtensorMap ta, tb;
-  int rc = make_tmap(&ta, A, k, rows, sched == kMasked ? p.groups : 1, BM);
+  p.a_box_rows = (sched == kDense && !pair && rows <= BM / 2) ? BM / 2 : BM;
+  int rc = make_tmap(&ta, A, k, rows, sched == kMasked ? p.groups : 1, p.a_box_rows);
   if (rc) return rc;
-  rc = make_tmap(&tb, B, k, n, sched == kDense ? 1 : p.groups, bn);
+  rc = make_tmap(&tb, B, k, n, sched == kDense ? 1 : p.groups, pair ? bn / 2 : bn);
   if (rc) return rc;
 
   // ------------------------------------------------ grid
   int64_t units;
   int extra = 0;
   if (sched == kMasked) {
-    units = m_blocks_eff * p.num_n_blocks;  // upper bound; actual from masked_m
+    // upper bound; the kernel reads the actual count from masked_m
+    units = static_cast<int64_t>(p.num_m_blocks) * p.groups * p.num_n_blocks;
     extra = 8 * (p.groups + 1);
   } else {
     units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks * splits;
   }
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
+  int grid;
+  if (pair) {
+    grid = 2 * static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms / 2)));
+  } else {
+    grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
+  }
   if (print_configs()) {
     fprintf(stderr,
-            "[dg] gemm sched=%d rows=%lld n=%lld k=%lld groups=%d: BN=%d splits=%d grid=%d "
+            "[dg] gemm sched=%d rows=%lld n=%lld k=%lld groups=%d: %s BN=%d splits=%d grid=%d "
             "units=%lld\n",
             sched, static_cast<long long>(rows), static_cast<long long>(n),
-            static_cast<long long>(k), p.groups, bn, splits, grid, static_cast<long long>(units));
+            static_cast<long long>(k), p.groups, pair ? "pair" : "single", bn, splits, grid,
+            static_cast<long long>(units));
   }
   switch (sched) {
-    case kDense: return dispatch<kDense>(bn, ta, tb, p, grid, extra, stream);
-    case kContiguous: return dispatch<kContiguous>(bn, ta, tb, p, grid, extra, stream);
-    case kMasked: return dispatch<kMasked>(bn, ta, tb, p, grid, extra, stream);
+    case kDense: return dispatch<kDense>(bn, pair, ta, tb, p, grid, extra, stream);
+    case kContiguous: return dispatch<kContiguous>(bn, false, ta, tb, p, grid, extra, stream);
+    case kMasked: return dispatch<kMasked>(bn, false, ta, tb, p, grid, extra, stream);
     default: return DG_ERR_INVALID_ARG;
   }
 }

@@ -43,6 +43,7 @@ struct GemmParams {
   int num_n_blocks;      // ceil(n / BN)
   int num_k_blocks;      // k / 128
   int splits;            // K splits (1 = none)
+  int a_box_rows;        // rows of A per TMA load: 128, or 64 when M <= 64
 };
 
 struct GemmConfig {

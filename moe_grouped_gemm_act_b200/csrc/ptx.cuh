@@ -97,6 +97,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Spins until *counter >= target (acquire).  Returns false, recording
+// DG_ERR_TIMEOUT, after kWaitLimitNs.
+__device__ __forceinline__ bool wait_counter(const uint32_t *counter, uint32_t target,
+                                             int *status) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const uint64_t t0 = globaltimer();
+  while (ld_acquire_gpu(counter) < target) {
+    __nanosleep(64);
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      record_status(status, DG_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
@@ -240,6 +262,99 @@ template <int N>
 __device__ __forceinline__ void reg_barrier(uint32_t *r) {
 #pragma unroll
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i])::"memory");
+}
+
+// ------------------------------------------------------------------ CTA pairs
+// The pair form: two CTAs of a 2-CTA cluster (ranks 0 and 1) run one
+// cta_group::2 MMA of M = 256; rank 0 issues it.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// All threads of both CTAs of the cluster.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address in the cluster shared window of the same shared-memory offset in
+// CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier given by its cluster-window address (possibly in the
+// peer CTA).  Default (release, CTA-scope) semantics: the arrive only has to
+// follow this thread's completed TMEM reads, which tcgen05.wait::ld and
+// tcgen05.fence::before_thread_sync already order; a cluster-scope release
+// would add a full fence to the promotion's critical path.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// 3-D TMA load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (`bar` is a cluster-window address).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void *tmap,
+                                                 uint32_t bar, int32_t c0,
+                                                 int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
+  asm volatile(
+      "tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+          dst),
+      "r"(ncols)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::
+                   : "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile(
+      "tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr),
+      "r"(ncols)
+      : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A * B^T with M = 256: rows 0-127 of A and D in
+// rank 0, rows 128-255 in rank 1; B split along N between the two CTAs'
+// shared memory at the same offsets.  Issued by one thread of rank 0.
+__device__ __forceinline__ void umma_f8_pair(uint32_t d_tmem, uint64_t a_desc,
+                                             uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, "
+      "%8, %9, %10, %11, %12}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z),
+      "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z)
+      : "memory");
+}
+
+// Arrives once on the mbarrier at cluster-window address `bar` (this CTA's or
+// the peer's) when all tcgen05 operations issued so far by this thread have
+// completed.  Pair form; one call per target barrier.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 "
+      "[%0];" ::"r"(bar)
+      : "memory");
 }
 
 // ------------------------------------------------------------------ UMMA descriptors

@@ -81,6 +81,30 @@ def test_dense_ragged_every_block_n(bn, m, n, k):
     check_gemm(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"{m}x{n}x{k} BN={bn}")
 
 
+@pytest.mark.parametrize("pair", [0, 1])
+@pytest.mark.parametrize("m,n,k", [(300, 392, 1024), (1000, 2112, 384), (513, 256, 256),
+                                   (256, 4096, 2048)])
+def test_dense_pair_and_single_cta_forms(pair, m, n, k):
+    # the 2-CTA (cta_group::2, 256 x 256 tiles) form and the single-CTA form
+    qa, alpha, qb, beta = dense_case(m, n, k, seed=m + 7 * n + k)
+    with env(DG_PAIR=pair):
+        got = run_dense(qa, alpha, qb, beta)
+    check_gemm(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"{m}x{n}x{k} pair={pair}")
+
+
+def test_dense_pair_exact_integers_bit_exact():
+    g = np.random.default_rng(2)
+    m, n, k = 512, 512, 2048
+    a = g.integers(-4, 5, size=(m, k)).astype(np.float32)
+    b = g.integers(-4, 5, size=(n, k)).astype(np.float32)
+    qa, qb = e4m3.encode_rne(a), e4m3.encode_rne(b)
+    with env(DG_PAIR=1):
+        got = run_dense(qa, np.ones((m, k // 128), np.float32), qb,
+                        np.ones((n // 128, k // 128), np.float32))
+    exact = a.astype(np.int64) @ b.astype(np.int64).T
+    assert np.array_equal(got, bf16.to_bits(exact.astype(np.float64)))
+
+
 @pytest.mark.parametrize("splits", [2, 3, 8])
 @pytest.mark.parametrize("bn", [32, 128])
 def test_dense_split_k(splits, bn):
