@@ -53,6 +53,38 @@ from moe_grouped_gemm_act_b200 import inputs  # noqa: E402
 METRIC = "FP8 block-scaled GEMM TFLOPS & % of B200 FP8 peak / HBM roofline, per shape"
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per GEMM launch,
+# averaged over the workload's launches, from ncu captures of this bench
+# (profiles/fp8_gemm_*.md give the commands).  Valid only for the GEMM
+# sources they were taken on: `source` is the first 16 hex digits of the
+# SHA-256 of csrc/gemm.cu + csrc/ptx.cuh + csrc/internal.h; on a mismatch the
+# bench reports null.
+GEMM_TRAFFIC = {
+    "source": "dd79907dc2e955a3",
+    "prefill": 201.7e6,
+    "decode64": 51.8e6,
+    "masked": 540.1e6,
+    "contiguous": 987.9e6,
+}
+
+
+def gemm_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "ptx.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "moe_grouped_gemm_act_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    try:
+        if gemm_source_hash() != GEMM_TRAFFIC["source"]:
+            return None
+    except OSError:
+        return None
+    return GEMM_TRAFFIC.get(workload)
+
 
 # ---------------------------------------------------------------- workloads
 def workload_spec(name: str) -> dict:
@@ -230,6 +262,8 @@ class DenseData:
         torch.cuda.synchronize()
 
     def launches_per_step(self) -> int:
+        # this library's kernels per step: one quantizer and one GEMM per
+        # shape (a split-K call also enqueues a runtime memset, not counted)
         return 2 * len(self.shapes)
 
     # end-to-end through the public API from pinned host buffers
@@ -254,6 +288,97 @@ class DenseData:
             qa, sfa = dg.dg_quantize_1x128(a)
             dg.dg_fp8_gemm_nt(qa, sfa, qb, sfb, s["d"], workspace=s["ws"])
             h["d"].copy_(s["d"], non_blocking=True)
+
+
+class GroupedData(DenseData):
+    """The MoE layouts: one grouped GEMM per step (quantize all activation
+    rows of the fixed buffer, then the contiguous or masked GEMM).  FLOPs
+    and algorithmic bytes count valid rows and active experts only."""
+
+    def __init__(self, spec, device):
+        import torch
+        import moe_grouped_gemm_act_b200 as dg
+        self.dg = dg
+        self.kind = spec["kind"]
+        G, n, k = spec["groups"], spec["n"], spec["k"]
+        if self.kind == "masked":
+            m_max = spec["m_max"]
+            counts = inputs.masked_counts(G, m_max, seed=spec["seed"])
+            x = inputs.activations(G * m_max, k, seed=spec["seed"] + 1,
+                                   outliers=True).reshape(G, m_max, k)
+            index = torch.from_numpy(counts).to(device)
+            rows_valid = int(counts.sum())
+            active = int((counts > 0).sum())
+            d_shape = (G, m_max, n)
+            self.rows_total = G * m_max
+        else:
+            lay = inputs.contiguous_layout(spec["tokens"], G, seed=spec["seed"])
+            x = inputs.activations(lay.m_total, k, seed=spec["seed"] + 1, outliers=True)
+            x[lay.m_indices < 0] = 0.0   # padding rows (their content is never read back)
+            index = torch.from_numpy(lay.m_indices).to(device)
+            rows_valid = int((lay.m_indices >= 0).sum())
+            active = int(len(np.unique(lay.m_indices[lay.m_indices >= 0])))
+            d_shape = (lay.m_total, n)
+            self.rows_total = lay.m_total
+        w = inputs.weights((G, n, k), seed=spec["seed"] + 2)
+        a32 = torch.from_numpy(x).to(device)
+        qb, sfb = dg.dg_quantize_128x128(torch.from_numpy(w).to(device))
+        del w
+        qa, sfa = dg.dg_quantize_1x128(a32)
+        d = torch.empty(d_shape, dtype=torch.bfloat16, device=device)
+        self.m = rows_valid
+        self.active = active
+        self.groups = G
+        self.shapes = [dict(n=n, k=k, a32=a32, qb=qb, sfb=sfb, qa=qa, sfa=sfa, d=d, ws=None,
+                            index=index, x_host=x)]
+        torch.cuda.synchronize()
+
+    def gemm_bytes(self) -> float:
+        s = self.shapes[0]
+        n, k, v = s["n"], s["k"], self.m
+        return (v * k + 4 * v * (k // 128) + self.active * (n * k + 4 * (-(-n // 128)) * (k // 128))
+                + 2 * v * n + 4 * s["index"].numel())
+
+    def gemm(self, s):
+        if self.kind == "masked":
+            self.dg.dg_m_grouped_fp8_gemm_nt_masked(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"],
+                                                    s["index"])
+        else:
+            self.dg.dg_m_grouped_fp8_gemm_nt_contiguous(s["qa"], s["sfa"], s["qb"], s["sfb"],
+                                                        s["d"], s["index"])
+
+    def make_host(self):
+        s = self.shapes[0]
+        self.host = [dict(a=torch_pin(s["x_host"]), qb=s["qb"].cpu().pin_memory(),
+                          sfb=s["sfb"].cpu().pin_memory(), index=s["index"].cpu().pin_memory(),
+                          d=torch_empty_pinned(s["d"]))]
+        h = self.host[0]
+        self.h2d = (h["a"].numel() * 4 + h["qb"].numel() + h["sfb"].numel() * 4
+                    + h["index"].numel() * 4)
+        self.d2h = h["d"].numel() * 2
+
+    def e2e_step(self, device):
+        s, h = self.shapes[0], self.host[0]
+        a = h["a"].to(device, non_blocking=True)
+        qb = h["qb"].to(device, non_blocking=True)
+        sfb = h["sfb"].to(device, non_blocking=True)
+        index = h["index"].to(device, non_blocking=True)
+        qa, sfa = self.dg.dg_quantize_1x128(a)
+        if self.kind == "masked":
+            self.dg.dg_m_grouped_fp8_gemm_nt_masked(qa, sfa, qb, sfb, s["d"], index)
+        else:
+            self.dg.dg_m_grouped_fp8_gemm_nt_contiguous(qa, sfa, qb, sfb, s["d"], index)
+        h["d"].copy_(s["d"], non_blocking=True)
+
+
+def torch_pin(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+
+
+def torch_empty_pinned(t):
+    import torch
+    return torch.empty(t.shape, dtype=t.dtype).pin_memory()
 
 
 class OracleSample:
@@ -344,10 +469,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     torch.cuda.set_device(device)
     dg.load_library()
     spec = workload_spec(args.workload)
-    if spec["kind"] != "dense":
-        raise SystemExit("the GPU arm of bench.py times the dense workloads; "
-                         "grouped layouts are covered by bench_grouped in the tests")
-    data = DenseData(spec, device)
+    data = DenseData(spec, device) if spec["kind"] == "dense" else GroupedData(spec, device)
 
     def barrier():
         if world > 1:
@@ -429,13 +551,14 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         peak = pk["hbm"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{pk['source']} copy bandwidth"}
-    roof["traffic"] = args.traffic
+    roof["traffic"] = args.traffic if args.traffic is not None else measured_traffic(args.workload)
+    roof["traffic_unit"] = "bytes per GEMM launch (ncu dram read + write)"
     per_shape = [{"n": s["n"], "k": s["k"], "gemm_us": 1e3 * ms,
                   "tflops": 2.0 * data.m * s["n"] * s["k"] / (ms * 1e-3) / 1e12}
                  for s, ms in zip(data.shapes, per_shape_ms)]
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and spec["kind"] == "dense":
         sampler = OracleSample(spec, args.ref_rows, args.ref_cols)
         sampler.run()
         secs, fl = 0.0, 0.0
@@ -450,7 +573,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3", "data": "synthetic",
-        "config": {"workload": spec["desc"], "m": data.m,
+        "config": {"workload": spec["desc"], "m" if spec["kind"] == "dense" else "valid_rows": data.m,
                    "nk": [[s["n"], s["k"]] for s in data.shapes],
                    "l2": "not flushed: each step streams %.0f MB of inputs (> 126 MB L2)"
                          % ((sum(s["a32"].numel() * 4 + s["qb"].numel() for s in data.shapes))
@@ -473,7 +596,7 @@ def main():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="prefill",
-                    choices=["prefill", "decode64", "decode128"])
+                    choices=["prefill", "decode64", "decode128", "contiguous", "masked"])
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--ref-rows", type=int, default=16,
                     help="rows of A per shape in the oracle's timed sample")
