@@ -13,9 +13,7 @@
 //
 //   warp 0      TMA producer: one lane streams A [128 x 128] and B [BN x 128]
 //               K blocks into a STAGES-deep shared-memory ring (128-byte
-//               swizzle), and the block's 128 row scales alpha (one 512-byte
-//               bulk copy from the MN-major scale array) into a separate ring
-//               of kAlphaSlots slots, all completing on mbarriers.
+//               swizzle), completing on mbarriers.
 //   warp 1      MMA issuer: allocates TMEM and, for each K block, issues 4
 //               tcgen05.mma (kind::f8f6f4, M=128, N=BN, K=32) into one of NBUF
 //               TMEM buffers (the first with accumulate off: a fresh partial
@@ -29,8 +27,10 @@
 //               4-7 and 8-11 split the BN columns.  Each thread owns one row
 //               and BN/2 columns: it pulls the block's partial sum with
 //               tcgen05.ld, releases the buffer, and does acc += partial *
-//               (alpha_row * beta) in FP32 registers.  After the last K block
-//               it converts to BF16 and stores its row segment (valid rows).
+//               (alpha_row * beta) in FP32 registers.  Its row scale alpha
+//               comes from its own async-copy ring, filled kAlphaAhead K
+//               blocks ahead.  After the last K block it converts to BF16 and
+//               stores its row segment (valid rows).
 //
 // The kernel is persistent (one CTA per SM).  All roles walk the same tile
 // sequence produced by a scheduler that knows the three layouts:
@@ -66,7 +66,8 @@ constexpr int kControlWarps = 4;        // producer, MMA issuer, 2 helpers (one 
 constexpr int kPromoWarps = 8;          // two column halves x four lane quarters
 constexpr int kPromoThreads = 32 * kPromoWarps;
 constexpr int kThreads = 32 * (kControlWarps + kPromoWarps);
-constexpr int kAlphaSlots = 16;         // alpha ring depth (>= STAGES + NBUF)
+constexpr int kAlphaAhead = 8;          // alpha prefetch lead, in K blocks
+constexpr int kAlphaRing = kAlphaAhead + 1;  // slots per promotion thread
 constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 
@@ -76,16 +77,15 @@ struct Layout {
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kAlphaOff = STAGES * kStageBytes;
-  static constexpr uint32_t kBarOff = kAlphaOff + kAlphaSlots * BM * 4;
-  // full[S] empty[S] afull[A] aempty[A] tfull[NBUF] tempty[NBUF] drain
-  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * kAlphaSlots + 2 * NBUF + 1;
+  static constexpr uint32_t kBarOff = kAlphaOff + kAlphaRing * kPromoThreads * 4;
+  // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 1;
   static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
   static constexpr uint32_t kPrefixOff = kMiscOff + 16;
   static constexpr uint32_t kCols = BN * NBUF;
   static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64
                                       : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
   static_assert(kCols <= 512, "TMEM holds 512 columns");
-  static_assert(STAGES + NBUF <= kAlphaSlots, "alpha ring must cover the pipeline");
 };
 
 // ------------------------------------------------------------------ scheduler
@@ -207,14 +207,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   const uint32_t bars = base + L::kBarOff;
   auto full_bar = [&](int s) { return bars + 8u * s; };
   auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
-  auto afull_bar = [&](int s) { return bars + 8u * (2 * STAGES + s); };
-  auto aempty_bar = [&](int s) { return bars + 8u * (2 * STAGES + kAlphaSlots + s); };
-  auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 * kAlphaSlots + b); };
-  auto tempty_bar = [&](int b) {
-    return bars + 8u * (2 * STAGES + 2 * kAlphaSlots + NBUF + b);
-  };
+  auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bars + 8u * (2 * STAGES + NBUF + b); };
   const uint32_t drain_bar = bars + 8u * (L::kNumBars - 1);
+  // per-thread alpha rings: [kAlphaRing][kPromoThreads] floats
   const float *s_alpha = reinterpret_cast<const float *>(smem + L::kAlphaOff);
+  const uint32_t s_alpha_u32 = base + L::kAlphaOff;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *s_flag = reinterpret_cast<int *>(smem + L::kMiscOff + 8);
@@ -234,10 +232,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
-    }
-    for (int s = 0; s < kAlphaSlots; ++s) {
-      mbar_init(afull_bar(s), 1);
-      mbar_init(aempty_bar(s), kPromoWarps);
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(tfull_bar(b), 1);
@@ -307,22 +301,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       }
       const int a_row = t.m_blk * TM + static_cast<int>(rank) * BM;
       const int b_row = t.n_blk * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
-      // alpha slice of this M block: rows a_row .. a_row+127 of the MN-major
-      // array, clipped to the leading dimension (a multiple of 4 floats).  In
-      // the pair form rank 1's rows may all lie past the end; it then copies
-      // the last 4 scales instead (its rows are never stored), keeping the
-      // copy inside the array and at least 16 bytes long.
-      const int64_t a_start = a_row <= p.ld_sfa - 4 ? a_row : p.ld_sfa - 4;
-      const int64_t a_avail = p.ld_sfa - a_start;
-      const uint32_t a_bytes = static_cast<uint32_t>(4 * (a_avail < BM ? a_avail : BM));
-      const float *a_src = p.sfa + static_cast<int64_t>(t.slab) * kg_total * p.ld_sfa + a_start;
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        const int as = it % kAlphaSlots;
-        const uint32_t aph = (it / kAlphaSlots) & 1;
         if (!mbar_wait(empty_bar(s), ph ^ 1, s_abort, p.status)) { alive = false; break; }
-        if (!mbar_wait(aempty_bar(as), aph ^ 1, s_abort, p.status)) { alive = false; break; }
         if (lane == 0) {
           const uint32_t sa = base + s * L::kStageBytes;
           if constexpr (PAIR) {
@@ -337,9 +319,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, t.slab);
             tma_load_3d(sa + kABytes, &tmap_b, full_bar(s), kb * BK, b_row, t.group);
           }
-          mbar_arrive_expect_tx(afull_bar(as), a_bytes);
-          bulk_load(base + L::kAlphaOff + as * (BM * 4), a_src + static_cast<int64_t>(kb) * p.ld_sfa,
-                    a_bytes, afull_bar(as));
         }
         __syncwarp();
       }
@@ -441,19 +420,34 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
       for (int c = 0; c < W; ++c) acc[c] = 0.0f;
 
+      // This thread's row scale alpha is prefetched kAlphaAhead K blocks
+      // ahead with per-thread 4-byte async copies into its own slots of a
+      // shared-memory ring (one commit group per K block, empty groups past
+      // the end of the unit), so no other thread is involved.  Rows past the
+      // end read the last row's scale (they are never stored).
+      const float *a_src = p.sfa + static_cast<int64_t>(t.slab) * kg_total * p.ld_sfa +
+                           min(row, p.rows - 1);
+      const int ptid = threadIdx.x - kControlWarps * 32;
+#pragma unroll
+      for (int d = 0; d < kAlphaAhead; ++d) {
+        if (t.k_begin + d < t.k_end)
+          cp_async4(s_alpha_u32 + 4u * (((it + d) % kAlphaRing) * kPromoThreads + ptid),
+                    a_src + static_cast<int64_t>(t.k_begin + d) * p.ld_sfa);
+        cp_async_commit();
+      }
       float b_next = __ldg(sfb_ptr + t.k_begin);
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
         const float b_cur = b_next;
         if (kb + 1 < t.k_end) b_next = __ldg(sfb_ptr + kb + 1);
-        const int as = it % kAlphaSlots;
         const int buf = it % NBUF;
-        if (!mbar_wait(afull_bar(as), (it / kAlphaSlots) & 1, s_abort, p.status)) {
-          alive = false;
-          break;
-        }
-        const float sc = s_alpha[as * BM + row_in_tile] * b_cur;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(aempty_bar(as));
+        cp_async_wait<kAlphaAhead - 1>();  // this block's alpha has landed
+        const float sc = s_alpha[(it % kAlphaRing) * kPromoThreads + ptid] * b_cur;
+        // refill the slot read one block ago (the ring is one slot deeper
+        // than the lead, so the slot just read is not overwritten)
+        if (kb + kAlphaAhead < t.k_end)
+          cp_async4(s_alpha_u32 + 4u * (((it + kAlphaAhead) % kAlphaRing) * kPromoThreads + ptid),
+                    a_src + static_cast<int64_t>(kb + kAlphaAhead) * p.ld_sfa);
+        cp_async_commit();
         if (!mbar_wait(tfull_bar(buf), (it / NBUF) & 1, s_abort, p.status)) {
           alive = false;
           break;

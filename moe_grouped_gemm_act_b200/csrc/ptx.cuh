@@ -147,6 +147,22 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src,
       : "memory");
 }
 
+// Per-thread 4-byte asynchronous copy global -> shared (completion tracked
+// per thread with commit / wait groups).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Waits until at most N of this thread's committed groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 // Allocates `ncols` TMEM columns (power of two >= 32); the base address is
 // written to shared memory at `dst`.  Whole warp.
