@@ -27,10 +27,10 @@
 //               4-7 and 8-11 split the BN columns.  Each thread owns one row
 //               and BN/2 columns: it pulls the block's partial sum with
 //               tcgen05.ld, releases the buffer, and does acc += partial *
-//               (alpha_row * beta) in FP32 registers.  Its row scale alpha
-//               comes from its own async-copy ring, filled kAlphaAhead K
-//               blocks ahead.  After the last K block it converts to BF16 and
-//               stores its row segment (valid rows).
+//               (alpha_row * beta) in FP32 registers, two columns per packed
+//               f32x2 FMA.  Its row scale alpha is loaded into registers two
+//               K blocks ahead.  After the last K block it converts to BF16
+//               and stores its row segment (valid rows).
 //
 // The kernel is persistent (one CTA per SM).  All roles walk the same tile
 // sequence produced by a scheduler that knows the three layouts:
@@ -66,8 +66,6 @@ constexpr int kControlWarps = 4;        // producer, MMA issuer, 2 helpers (one 
 constexpr int kPromoWarps = 8;          // two column halves x four lane quarters
 constexpr int kPromoThreads = 32 * kPromoWarps;
 constexpr int kThreads = 32 * (kControlWarps + kPromoWarps);
-constexpr int kAlphaAhead = 8;          // alpha prefetch lead, in K blocks
-constexpr int kAlphaRing = kAlphaAhead + 1;  // slots per promotion thread
 constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 
@@ -76,8 +74,7 @@ struct Layout {
   // the pair form keeps half of the B tile (BN/2 rows) in each CTA
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kAlphaOff = STAGES * kStageBytes;
-  static constexpr uint32_t kBarOff = kAlphaOff + kAlphaRing * kPromoThreads * 4;
+  static constexpr uint32_t kBarOff = STAGES * kStageBytes;
   // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain
   static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 1;
   static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
@@ -210,9 +207,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bars + 8u * (2 * STAGES + NBUF + b); };
   const uint32_t drain_bar = bars + 8u * (L::kNumBars - 1);
-  // per-thread alpha rings: [kAlphaRing][kPromoThreads] floats
-  const float *s_alpha = reinterpret_cast<const float *>(smem + L::kAlphaOff);
-  const uint32_t s_alpha_u32 = base + L::kAlphaOff;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *s_flag = reinterpret_cast<int *>(smem + L::kMiscOff + 8);
@@ -357,15 +351,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
               umma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
             }
           }
+          // publish the buffer first: the promotion is on the critical path,
+          // the producer has STAGES - 1 blocks of slack
           if constexpr (PAIR) {
-            // free the stage and publish the buffer in both CTAs
-            umma_commit_pair(mapa_shared(empty_bar(s), 0));
-            umma_commit_pair(mapa_shared(empty_bar(s), 1));
             umma_commit_pair(mapa_shared(tfull_bar(buf), 0));
             umma_commit_pair(mapa_shared(tfull_bar(buf), 1));
+            umma_commit_pair(mapa_shared(empty_bar(s), 0));
+            umma_commit_pair(mapa_shared(empty_bar(s), 1));
           } else {
-            umma_commit(empty_bar(s));
             umma_commit(tfull_bar(buf));
+            umma_commit(empty_bar(s));
           }
         }
         __syncwarp();
@@ -420,34 +415,31 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
       for (int c = 0; c < W; ++c) acc[c] = 0.0f;
 
-      // This thread's row scale alpha is prefetched kAlphaAhead K blocks
-      // ahead with per-thread 4-byte async copies into its own slots of a
-      // shared-memory ring (one commit group per K block, empty groups past
-      // the end of the unit), so no other thread is involved.  Rows past the
-      // end read the last row's scale (they are never stored).
+      // This thread's row scale alpha is loaded two K blocks ahead into
+      // registers (one coalesced 128-byte load per warp and block); rows past
+      // the end read the last row's scale (they are never stored).  The
+      // column block's beta, the same for the whole warp, is fetched 32 K
+      // blocks at a time, one per lane, a batch ahead, and broadcast with a
+      // shuffle.
       const float *a_src = p.sfa + static_cast<int64_t>(t.slab) * kg_total * p.ld_sfa +
                            min(row, p.rows - 1);
-      const int ptid = threadIdx.x - kControlWarps * 32;
-#pragma unroll
-      for (int d = 0; d < kAlphaAhead; ++d) {
-        if (t.k_begin + d < t.k_end)
-          cp_async4(s_alpha_u32 + 4u * (((it + d) % kAlphaRing) * kPromoThreads + ptid),
-                    a_src + static_cast<int64_t>(t.k_begin + d) * p.ld_sfa);
-        cp_async_commit();
-      }
-      float b_next = __ldg(sfb_ptr + t.k_begin);
+      float a_cur = __ldg(a_src + static_cast<int64_t>(t.k_begin) * p.ld_sfa);
+      float a_next = t.k_begin + 1 < t.k_end
+                         ? __ldg(a_src + static_cast<int64_t>(t.k_begin + 1) * p.ld_sfa)
+                         : 0.0f;
+      float b_batch = t.k_begin + lane < t.k_end ? __ldg(sfb_ptr + t.k_begin + lane) : 0.0f;
+      float b_batch_next =
+          t.k_begin + 32 + lane < t.k_end ? __ldg(sfb_ptr + t.k_begin + 32 + lane) : 0.0f;
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
-        const float b_cur = b_next;
-        if (kb + 1 < t.k_end) b_next = __ldg(sfb_ptr + kb + 1);
+        const int j = (kb - t.k_begin) & 31;
+        const float sc = a_cur * __shfl_sync(0xffffffffu, b_batch, j);
+        if (j == 31) {
+          b_batch = b_batch_next;
+          b_batch_next = kb + 33 + lane < t.k_end ? __ldg(sfb_ptr + kb + 33 + lane) : 0.0f;
+        }
+        a_cur = a_next;
+        if (kb + 2 < t.k_end) a_next = __ldg(a_src + static_cast<int64_t>(kb + 2) * p.ld_sfa);
         const int buf = it % NBUF;
-        cp_async_wait<kAlphaAhead - 1>();  // this block's alpha has landed
-        const float sc = s_alpha[(it % kAlphaRing) * kPromoThreads + ptid] * b_cur;
-        // refill the slot read one block ago (the ring is one slot deeper
-        // than the lead, so the slot just read is not overwritten)
-        if (kb + kAlphaAhead < t.k_end)
-          cp_async4(s_alpha_u32 + 4u * (((it + kAlphaAhead) % kAlphaRing) * kPromoThreads + ptid),
-                    a_src + static_cast<int64_t>(kb + kAlphaAhead) * p.ld_sfa);
-        cp_async_commit();
         if (!mbar_wait(tfull_bar(buf), (it / NBUF) & 1, s_abort, p.status)) {
           alive = false;
           break;
@@ -472,7 +464,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             }
           }
 #pragma unroll
-          for (int c = 0; c < LW; ++c) acc[c0 + c] = fmaf(__uint_as_float(r[c]), sc, acc[c0 + c]);
+          for (int c = 0; c < LW; c += 2)
+            ffma2(acc[c0 + c], acc[c0 + c + 1], __uint_as_float(r[c]), __uint_as_float(r[c + 1]), sc);
         }
       }
       if (!alive) break;

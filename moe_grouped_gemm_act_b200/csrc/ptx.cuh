@@ -147,20 +147,20 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src,
       : "memory");
 }
 
-// Per-thread 4-byte asynchronous copy global -> shared (completion tracked
-// per thread with commit / wait groups).
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// Waits until at most N of this thread's committed groups are pending.
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// ------------------------------------------------------------------ FP32x2
+// a0 = x0 * s + a0 and a1 = x1 * s + a1: two fused multiply-adds with one
+// rounding each (to nearest even, subnormals kept, as fmaf) in one packed
+// f32x2 instruction, which halves the issue slots of the promotion.
+__device__ __forceinline__ void ffma2(float &a0, float &a1, float x0, float x1,
+                                      float s) {
+  asm("{\n\t.reg .b64 d, x, y;\n\t"
+      "mov.b64 d, {%0, %1};\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %4};\n\t"
+      "fma.rn.f32x2 d, x, y, d;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1), "f"(s));
 }
 
 // ------------------------------------------------------------------ tcgen05
