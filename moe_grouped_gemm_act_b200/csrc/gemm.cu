@@ -69,14 +69,20 @@ constexpr int kThreads = 32 * (kControlWarps + kPromoWarps);
 constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 
-template <int BN, int STAGES, int NBUF, bool PAIR>
+template <int BN, int STAGES, int NBUF, bool PAIR, bool STAGED>
 struct Layout {
   // the pair form keeps half of the B tile (BN/2 rows) in each CTA
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kBarOff = STAGES * kStageBytes;
-  // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain
-  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 1;
+  // With STAGED, BF16 staging of the output for coalesced stores: 128 rows
+  // x kOutCols (a 256-wide tile goes out in two column halves), then one
+  // byte per row saying whether it is stored
+  static constexpr uint32_t kOutCols = BN < 128 ? BN : 128;
+  static constexpr uint32_t kOutOff = STAGES * kStageBytes;
+  static constexpr uint32_t kRowOkOff = kOutOff + (STAGED ? BM * kOutCols * 2 : 0);
+  static constexpr uint32_t kBarOff = kRowOkOff + (STAGED ? BM : 0);
+  // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain epi
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
   static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
   static constexpr uint32_t kPrefixOff = kMiscOff + 16;
   static constexpr uint32_t kCols = BN * NBUF;
@@ -185,7 +191,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
                 const GemmParams p) {
-  using L = Layout<BN, STAGES, NBUF, PAIR>;
+  // dense tiles leave through shared memory (coalesced row stores); the
+  // grouped layouts, whose tiles are short and often partly empty, store
+  // each thread's row segment directly (measured faster for them)
+  constexpr bool kStaged = SCHED == kDense;
+  using L = Layout<BN, STAGES, NBUF, PAIR, kStaged>;
   constexpr int TM = PAIR ? 2 * BM : BM;   // rows per tile
   static_assert(!PAIR || SCHED == kDense, "the pair form serves dense GEMMs");
   constexpr int W = BN / 2;                 // columns per promotion thread
@@ -206,7 +216,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
   auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bars + 8u * (2 * STAGES + NBUF + b); };
-  const uint32_t drain_bar = bars + 8u * (L::kNumBars - 1);
+  const uint32_t drain_bar = bars + 8u * (L::kNumBars - 2);
+  // synchronises the promotion threads in the epilogue (bounded, unlike a
+  // named barrier, so that an aborting warp cannot strand the others)
+  const uint32_t epi_bar = bars + 8u * (L::kNumBars - 1);
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *s_flag = reinterpret_cast<int *>(smem + L::kMiscOff + 8);
@@ -232,6 +245,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       mbar_init(tempty_bar(b), PAIR ? 2 * kPromoWarps : kPromoWarps);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(epi_bar, kPromoThreads);
     *s_abort = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -392,6 +406,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const uint32_t tempty_target0 = PAIR ? mapa_shared(tempty_bar(0), 0) : tempty_bar(0);
     int it = 0;
     bool alive = true;
+    // every promotion thread arrives, then waits for the phase (bounded)
+    uint32_t epi_phase = 0;
+    auto epi_sync = [&]() -> bool {
+      mbar_arrive(epi_bar);
+      const bool ok = mbar_wait(epi_bar, epi_phase & 1, s_abort, p.status);
+      ++epi_phase;
+      return ok;
+    };
     for (int u = u_first; u < units && alive; u += u_stride) {
       Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
       const int row = t.m_blk * TM + static_cast<int>(rank) * BM + row_in_tile;
@@ -471,7 +493,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       if (!alive) break;
 
       // ---------------------------------------------------------- epilogue
-      if (p.splits > 1) {
+      // (split K serves dense shapes only; the grouped instances leave it
+      // out, which also keeps their register allocation lean)
+      if (SCHED == kDense && p.splits > 1) {
         if (*s_abort) break;
         // Split K: every CTA of the tile writes its FP32 partial (valid rows
         // only, as float4 slots [column / 4][row] so that a warp's 32 rows
@@ -492,14 +516,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
         }
         __threadfence();
-        asm volatile("bar.sync 1, %0;" ::"n"(kPromoThreads) : "memory");
+        if (!epi_sync()) break;
         const int ptid = threadIdx.x - kControlWarps * 32;
         if (ptid == 0) {
           atomicAdd(p.ws_ticket + tile, 1u);
           if (!wait_counter(p.ws_ticket + tile, static_cast<uint32_t>(p.splits), p.status))
             *s_abort = 1;
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kPromoThreads) : "memory");
+        if (!epi_sync()) break;
         if (*s_abort) break;
         __threadfence();
         const int row0 = t.m_blk * TM + static_cast<int>(rank) * BM;
@@ -507,54 +531,128 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int slots = valid * (BN / 4);
         const int share = (slots + p.splits - 1) / p.splits;
         const int f_end = min(slots, (t.split + 1) * share);
-        for (int f = t.split * share + ptid; f < f_end; f += kPromoThreads) {
-          const int c4 = f / valid, r = f - c4 * valid;
-          const float4 *src = part + c4 * BM + r;
-          float4 sum = __ldcg(src);
-          int s = 1;
-          for (; s + 3 < p.splits; s += 4) {
-            // four independent loads in flight, added in split order
-            const float4 v0 = __ldcg(src + static_cast<int64_t>(s) * kTileSlots);
-            const float4 v1 = __ldcg(src + static_cast<int64_t>(s + 1) * kTileSlots);
-            const float4 v2 = __ldcg(src + static_cast<int64_t>(s + 2) * kTileSlots);
-            const float4 v3 = __ldcg(src + static_cast<int64_t>(s + 3) * kTileSlots);
-            sum.x += v0.x; sum.y += v0.y; sum.z += v0.z; sum.w += v0.w;
-            sum.x += v1.x; sum.y += v1.y; sum.z += v1.z; sum.w += v1.w;
-            sum.x += v2.x; sum.y += v2.y; sum.z += v2.z; sum.w += v2.w;
-            sum.x += v3.x; sum.y += v3.y; sum.z += v3.z; sum.w += v3.w;
+        // Q slots per thread per pass so that their loads overlap; each
+        // slot is summed over splits 0, 1, ... in order (deterministic)
+        constexpr int Q = 4;
+        for (int f0 = t.split * share + ptid; f0 < f_end; f0 += Q * kPromoThreads) {
+          const float4 *src[Q];
+          bool ok[Q];
+          float4 sum[Q];
+#pragma unroll
+          for (int q = 0; q < Q; ++q) {
+            const int f = f0 + q * kPromoThreads;
+            ok[q] = f < f_end;
+            const int c4 = ok[q] ? f / valid : 0;
+            src[q] = part + c4 * BM + (ok[q] ? f - c4 * valid : 0);
+            sum[q] = ok[q] ? __ldcg(src[q]) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
-          for (; s < p.splits; ++s) {
-            const float4 v = __ldcg(src + static_cast<int64_t>(s) * kTileSlots);
-            sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+#pragma unroll 2
+          for (int s = 1; s < p.splits; ++s) {
+            float4 v[Q];
+#pragma unroll
+            for (int q = 0; q < Q; ++q)
+              v[q] = ok[q] ? __ldcg(src[q] + static_cast<int64_t>(s) * kTileSlots)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+              sum[q].x += v[q].x;
+              sum[q].y += v[q].y;
+              sum[q].z += v[q].z;
+              sum[q].w += v[q].w;
+            }
           }
-          const int col = t.n_blk * BN + 4 * c4;
-          if (col < p.n) {
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y);
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z, sum.w);
-            uint2 v;
-            v.x = *reinterpret_cast<const uint32_t *>(&lo);
-            v.y = *reinterpret_cast<const uint32_t *>(&hi);
-            *reinterpret_cast<uint2 *>(p.d + static_cast<int64_t>(row0 + r) * p.n + col) = v;
+#pragma unroll
+          for (int q = 0; q < Q; ++q) {
+            const int f = f0 + q * kPromoThreads;
+            const int c4 = f / valid, r = f - c4 * valid;
+            const int col = t.n_blk * BN + 4 * c4;
+            if (ok[q] && col < p.n) {
+              const __nv_bfloat162 lo = __floats2bfloat162_rn(sum[q].x, sum[q].y);
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(sum[q].z, sum[q].w);
+              uint2 v;
+              v.x = *reinterpret_cast<const uint32_t *>(&lo);
+              v.y = *reinterpret_cast<const uint32_t *>(&hi);
+              *reinterpret_cast<uint2 *>(p.d + static_cast<int64_t>(row0 + r) * p.n + col) = v;
+            }
           }
         }
         continue;  // this split's share of D is written
       }
-      if (row_ok) {
-        uint16_t *drow = p.d + (static_cast<int64_t>(t.slab) * p.rows + row) * p.n;
+      if constexpr (!kStaged) {
+        // each thread stores its row segment (valid rows), 16 bytes at a time
+        if (row_ok) {
+          uint16_t *drow = p.d + (static_cast<int64_t>(t.slab) * p.rows + row) * p.n;
 #pragma unroll
-        for (int c = 0; c < W; c += 8) {
-          if (col0 + c < p.n) {
-            uint4 v;
-            uint32_t *w = reinterpret_cast<uint32_t *>(&v);
+          for (int c = 0; c < W; c += 8) {
+            if (col0 + c < p.n) {
+              uint4 v;
+              uint32_t *w = reinterpret_cast<uint32_t *>(&v);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const __nv_bfloat162 h = __floats2bfloat162_rn(acc[c + 2 * j], acc[c + 2 * j + 1]);
-              w[j] = *reinterpret_cast<const uint32_t *>(&h);
+              for (int j = 0; j < 4; ++j) {
+                const __nv_bfloat162 h =
+                    __floats2bfloat162_rn(acc[c + 2 * j], acc[c + 2 * j + 1]);
+                w[j] = *reinterpret_cast<const uint32_t *>(&h);
+              }
+              *reinterpret_cast<uint4 *>(drow + col0 + c) = v;
             }
-            *reinterpret_cast<uint4 *>(drow + col0 + c) = v;
+          }
+        }
+      } else {
+        // The tile leaves through shared memory so that each warp store
+        // writes whole row segments (16-byte chunks of consecutive columns of
+        // a row in consecutive lanes).  Staging layout: [128 rows][kOutCols]
+        // BF16 with 16-byte chunk c of row r at chunk c ^ (r mod kSw), which
+        // keeps both the row-per-lane writes and the row-major reads free of
+        // bank conflicts.  A 256-wide tile goes out in two column halves,
+        // each written by the warps that own it.
+        constexpr int kChunks = L::kOutCols / 8;        // 16-byte chunks per staged row
+        constexpr int kSw = kChunks < 8 ? kChunks : 8;  // swizzle span, in chunks
+        constexpr int kPhases = BN > 128 ? 2 : 1;
+        constexpr int kRowBytes = L::kOutCols * 2;
+        const uint32_t s_out = base + L::kOutOff;
+        uint8_t *s_rowok = smem + L::kRowOkOff;
+        const int ptid = threadIdx.x - kControlWarps * 32;
+        const int64_t slab_row0 = static_cast<int64_t>(t.slab) * p.rows + t.m_blk * TM +
+                                  static_cast<int>(rank) * BM;
+        if (half == 0) s_rowok[row_in_tile] = row_ok ? 1 : 0;
+#pragma unroll
+        for (int ph = 0; ph < kPhases; ++ph) {
+          if (kPhases == 1 || half == ph) {
+            const int scol0 = kPhases == 1 ? half * W : 0;  // staged column of acc[0]
+#pragma unroll
+            for (int c = 0; c < W; c += 8) {
+              uint32_t w[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(acc[c + 2 * j], acc[c + 2 * j + 1]);
+                w[j] = *reinterpret_cast<const uint32_t *>(&h);
+              }
+              const int chunk = (scol0 + c) / 8;
+              st_shared_v4(s_out + row_in_tile * kRowBytes + ((chunk ^ (row_in_tile % kSw)) * 16),
+                           w[0], w[1], w[2], w[3]);
+            }
+          }
+          if (!epi_sync()) {
+            alive = false;
+            break;
+          }
+          const int col_base = t.n_blk * BN + ph * 128;
+#pragma unroll 1
+          for (int f = ptid; f < BM * kChunks; f += kPromoThreads) {
+            const int r = f / kChunks, ch = f - r * kChunks;
+            const int col = col_base + ch * 8;
+            if (s_rowok[r] && col < p.n) {
+              const uint4 v = ld_shared_v4(s_out + r * kRowBytes + ((ch ^ (r % kSw)) * 16));
+              *reinterpret_cast<uint4 *>(p.d + (slab_row0 + r) * p.n + col) = v;
+            }
+          }
+          if (!epi_sync()) {
+            alive = false;
+            break;
           }
         }
       }
+      if (!alive) break;
     }
   }
 
@@ -585,15 +683,15 @@ constexpr Candidate kCandidates[] = {
 // The pair form: 256 x 256 tiles, half of B per CTA (32 KB stages).
 constexpr Candidate kPairCandidate = {256, 6, 2};
 
-template <int BN, int STAGES, int NBUF, bool PAIR>
+template <int BN, int STAGES, int NBUF, bool PAIR, bool STAGED>
 constexpr int smem_bytes_for(int extra) {
-  return 1024 + Layout<BN, STAGES, NBUF, PAIR>::kPrefixOff + extra;
+  return 1024 + Layout<BN, STAGES, NBUF, PAIR, STAGED>::kPrefixOff + extra;
 }
 
 template <int BN, int STAGES, int NBUF, int SCHED, bool PAIR>
 int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                     int grid, int extra_smem, cudaStream_t stream, bool coop) {
-  const int smem = smem_bytes_for<BN, STAGES, NBUF, PAIR>(extra_smem);
+  const int smem = smem_bytes_for<BN, STAGES, NBUF, PAIR, SCHED == kDense>(extra_smem);
   auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED, PAIR>;
   static int configured_smem[64] = {0};  // per device; grows only
   int dev = 0;
@@ -635,6 +733,36 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
     kern<<<grid, kThreads, smem, stream>>>(ta, tb, p);
   }
   return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
+// Dynamic shared memory of a tile form (extra = the masked prefix tables;
+// `staged` = the dense schedule's output staging).
+int config_smem(int bn, bool pair, int extra, bool staged) {
+  if (pair)
+    return smem_bytes_for<kPairCandidate.bn, kPairCandidate.stages, kPairCandidate.nbuf, true,
+                          true>(extra);
+  switch (bn) {
+    case 256: return staged ? smem_bytes_for<256, 4, 2, false, true>(extra)
+                            : smem_bytes_for<256, 4, 2, false, false>(extra);
+    case 128: return staged ? smem_bytes_for<128, 6, 4, false, true>(extra)
+                            : smem_bytes_for<128, 6, 4, false, false>(extra);
+    case 64: return staged ? smem_bytes_for<64, 8, 8, false, true>(extra)
+                           : smem_bytes_for<64, 8, 8, false, false>(extra);
+    case 32: return staged ? smem_bytes_for<32, 8, 8, false, true>(extra)
+                           : smem_bytes_for<32, 8, 8, false, false>(extra);
+    case 16: return staged ? smem_bytes_for<16, 8, 8, false, true>(extra)
+                           : smem_bytes_for<16, 8, 8, false, false>(extra);
+    default: return 1 << 30;
+  }
+}
+
+// The opt-in shared memory limit per block of the current device.
+int max_smem_per_block() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return 232448;  // B200
+  return v;
 }
 
 template <int SCHED>
@@ -722,17 +850,20 @@ struct Choice {
 // Splitting K is considered for dense shapes of at most two M blocks, only
 // while all units fit in one wave of CTAs, and only when the workspace can
 // hold the split's FP32 partials
-// (`ws_bytes`).  The pair form (2-CTA clusters) is opt-in (DG_PAIR=1): on
-// B200 it halves each SM's B traffic but measured no faster than the single-
-// CTA 256-wide tile, both being bound by the TMEM round trip.
+// (`ws_bytes`).  Tile forms whose shared memory (with `extra` bytes of
+// masked prefix tables) exceeds `max_smem` are skipped.  The pair form
+// (2-CTA clusters) is opt-in (DG_PAIR=1): on B200 it halves each SM's B
+// traffic but measured no faster than the single-CTA 256-wide tile, both
+// being bound by the TMEM round trip.
 Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, int num_sms,
-                     size_t ws_bytes) {
+                     size_t ws_bytes, int extra = 0, int max_smem = 232448) {
   const int64_t m_blocks = (rows + BM - 1) / BM;
   const int64_t k_blocks = k / BK;
   const int64_t m_blocks_eff = sched == kMasked ? m_blocks * groups : m_blocks;
   Choice c{128, 1, false};
   double best = 1e300;
   for (const Candidate &cand : kCandidates) {
+    if (config_smem(cand.bn, false, extra, sched == kDense) > max_smem) continue;
     for (int s = 1; s <= 16; ++s) {
       if (s > 1 && (sched != kDense || m_blocks > 2)) break;
       if (s > k_blocks) break;
@@ -767,7 +898,12 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   if (ws == nullptr) ws_bytes = 0;
 
   // ------------------------------------------------ choose the tile form
-  const Choice choice = choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes);
+  // masked launches keep per-expert row-block counts and prefix sums in
+  // shared memory
+  const int extra = sched == kMasked ? 8 * (p.groups + 1) : 0;
+  const int max_smem = max_smem_per_block();
+  const Choice choice =
+      choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes, extra, max_smem);
   int bn = choice.bn, splits = choice.splits;
   bool pair = choice.pair;
   // Tuning / test overrides: DG_PAIR=0/1 disables / forces the pair form
@@ -801,6 +937,8 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
       splits = v;
     }
   }
+  if (config_smem(bn, pair, extra, sched == kDense) > max_smem)
+    return DG_ERR_INVALID_ARG;  // too many experts
   const int tile_rows = pair ? 2 * BM : BM;
   p.num_m_blocks = static_cast<int>((rows + tile_rows - 1) / tile_rows);
   p.num_n_blocks = static_cast<int>((n + bn - 1) / bn);
@@ -826,11 +964,9 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
 
   // ------------------------------------------------ grid
   int64_t units;
-  int extra = 0;
   if (sched == kMasked) {
     // upper bound; the kernel reads the actual count from masked_m
     units = static_cast<int64_t>(p.num_m_blocks) * p.groups * p.num_n_blocks;
-    extra = 8 * (p.groups + 1);
   } else {
     units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks * splits;
   }

@@ -147,6 +147,23 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src,
       : "memory");
 }
 
+// ------------------------------------------------------------------ shared
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b,
+                                             uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
+               "r"(c), "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 // ------------------------------------------------------------------ FP32x2
 // a0 = x0 * s + a0 and a1 = x1 * s + a1: two fused multiply-adds with one
 // rounding each (to nearest even, subnormals kept, as fmaf) in one packed
