@@ -93,7 +93,9 @@ struct Layout {
 
 // ------------------------------------------------------------------ scheduler
 struct Tile {
-  int m_blk, n_blk, split;
+  int m_blk, n_blk;
+  int tile;           // linear tile index (dense / contiguous)
+  int split, nsplit;  // this unit's K split of the tile's nsplit
   int slab;     // A / D slab (expert for masked, else 0)
   int group;    // B / beta group (expert, 0 for dense)
   int k_begin, k_end;  // K blocks of this unit
@@ -102,15 +104,20 @@ struct Tile {
 __device__ __forceinline__ int num_units(const GemmParams &p, int sched,
                                          const int *s_prefix) {
   if (sched == kMasked) return s_prefix[p.groups];
-  return p.num_m_blocks * p.num_n_blocks * p.splits;
+  return p.full_tiles + (p.num_m_blocks * p.num_n_blocks - p.full_tiles) * p.splits;
 }
 
 // Maps unit u to a tile.  The contiguous expert lookup is done separately.
+// Dense and contiguous: units 0 .. full_tiles-1 are whole tiles; each later
+// tile is `splits` consecutive units (K ranges), so a split tile's units fall
+// on distinct CTAs of the last wave.
 __device__ __forceinline__ Tile unit_to_tile(const GemmParams &p, int sched,
                                              int u, const int *s_prefix,
                                              const int *s_mblocks) {
   Tile t;
+  t.tile = 0;
   t.split = 0;
+  t.nsplit = 1;
   t.slab = 0;
   t.group = 0;
   if (sched == kMasked) {
@@ -129,9 +136,14 @@ __device__ __forceinline__ Tile unit_to_tile(const GemmParams &p, int sched,
     t.n_blk = r / mb;
     t.m_blk = r - t.n_blk * mb;
   } else {
-    const int s = p.splits;
-    const int tile = u / s;
-    t.split = u - tile * s;
+    int tile = u;
+    if (u >= p.full_tiles) {
+      const int v = u - p.full_tiles;
+      tile = p.full_tiles + v / p.splits;
+      t.split = v - (tile - p.full_tiles) * p.splits;
+      t.nsplit = p.splits;
+    }
+    t.tile = tile;
     const int span = kRasterGroupM * p.num_n_blocks;
     const int grp = tile / span;
     const int first_m = grp * kRasterGroupM;
@@ -140,7 +152,7 @@ __device__ __forceinline__ Tile unit_to_tile(const GemmParams &p, int sched,
     t.m_blk = first_m + r % gm;
     t.n_blk = r / gm;
   }
-  const int kb = p.num_k_blocks, s = p.splits;
+  const int kb = p.num_k_blocks, s = t.nsplit;
   t.k_begin = (kb * t.split) / s;
   t.k_end = (kb * (t.split + 1)) / s;
   return t;
@@ -495,7 +507,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       // ---------------------------------------------------------- epilogue
       // (split K serves dense shapes only; the grouped instances leave it
       // out, which also keeps their register allocation lean)
-      if (SCHED == kDense && p.splits > 1) {
+      if (SCHED == kDense && t.nsplit > 1) {
         if (*s_abort) break;
         // Split K: every CTA of the tile writes its FP32 partial (valid rows
         // only, as float4 slots [column / 4][row] so that a warp's 32 rows
@@ -504,7 +516,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         // cooperative, so they are all resident); then each split reduces its
         // own 1/S share of the tile's slots, summing splits 0, 1, ... in
         // order (deterministic), and stores that share as BF16.
-        const int tile = u / p.splits;
+        const int tile = t.tile - p.full_tiles;  // index among the split tiles
         constexpr int kTileSlots = BM * BN / 4;
         float4 *part = reinterpret_cast<float4 *>(p.ws) +
                        static_cast<int64_t>(tile) * p.splits * kTileSlots;
@@ -844,12 +856,22 @@ size_t split_ws_bytes(int64_t tiles, int splits, int bn) {
 struct Choice {
   int bn, splits;
   bool pair;
+  int64_t full_tiles;  // dense: tiles computed whole; the rest are split
 };
 
+// Estimated time of the dense "tail split": the whole waves of tiles, then
+// the tiles of the last, partial wave split `s` ways along K over the CTAs.
+double estimate_tail(int64_t waves, int64_t k, int bn, int s) {
+  const int64_t kb = k / BK;
+  const double whole = waves * (kb * kb_cycles(bn) + 2500.0);
+  return whole + ((kb + s - 1) / s) * kb_cycles(bn) + 2500.0 + 1500.0 + 300.0 * s;
+}
+
 // Tile form for a launch: a tile width and K split from the cost model.
-// Splitting K is considered for dense shapes of at most two M blocks, only
-// while all units fit in one wave of CTAs, and only when the workspace can
-// hold the split's FP32 partials
+// Splitting every tile's K is considered for dense shapes of at most two M
+// blocks, only while all units fit in one wave of CTAs; larger dense shapes
+// may split only the tiles of a last, partial wave (spreading them over all
+// CTAs).  Either needs a workspace that holds the split tiles' FP32 partials
 // (`ws_bytes`).  Tile forms whose shared memory (with `extra` bytes of
 // masked prefix tables) exceeds `max_smem` are skipped.  The pair form
 // (2-CTA clusters) is opt-in (DG_PAIR=1): on B200 it halves each SM's B
@@ -860,20 +882,32 @@ Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, 
   const int64_t m_blocks = (rows + BM - 1) / BM;
   const int64_t k_blocks = k / BK;
   const int64_t m_blocks_eff = sched == kMasked ? m_blocks * groups : m_blocks;
-  Choice c{128, 1, false};
+  Choice c{128, 1, false, 0};
   double best = 1e300;
   for (const Candidate &cand : kCandidates) {
     if (config_smem(cand.bn, false, extra, sched == kDense) > max_smem) continue;
+    const int64_t tiles = m_blocks * ((n + cand.bn - 1) / cand.bn);
     for (int s = 1; s <= 16; ++s) {
       if (s > 1 && (sched != kDense || m_blocks > 2)) break;
       if (s > k_blocks) break;
-      const int64_t tiles = m_blocks * ((n + cand.bn - 1) / cand.bn);
       if (s > 1 && tiles * s > num_sms) break;
       if (s > 1 && split_ws_bytes(tiles, s, cand.bn) > ws_bytes) break;
       const double e = estimate(m_blocks_eff, n, k, cand.bn, s, num_sms);
       if (e < best * 0.97) {
         best = e;
-        c = {cand.bn, s, false};
+        c = {cand.bn, s, false, 0};
+      }
+    }
+    if (sched == kDense && m_blocks > 2) {
+      const int64_t waves = tiles / num_sms, tail = tiles % num_sms;
+      const int s = tail > 0 ? static_cast<int>(std::min<int64_t>(num_sms / tail, 16)) : 1;
+      if (waves > 0 && s >= 2 && s <= k_blocks && split_ws_bytes(tail, s, cand.bn) <= ws_bytes) {
+        const double bytes = static_cast<double>(n) * k + m_blocks * 128.0 * k;
+        const double e = std::max(estimate_tail(waves, k, cand.bn, s), bytes / (23.0 * num_sms));
+        if (e < best * 0.97) {
+          best = e;
+          c = {cand.bn, s, false, waves * num_sms};
+        }
       }
     }
   }
@@ -887,7 +921,7 @@ size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int num_sms) {
   // the split the heuristic picks when the workspace is not a constraint
   const Choice c = choose_config(kDense, M, N, K, 1, num_sms, ~static_cast<size_t>(0));
   if (c.splits <= 1) return 0;
-  const int64_t tiles = ((M + BM - 1) / BM) * ((N + c.bn - 1) / c.bn);
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + c.bn - 1) / c.bn) - c.full_tiles;
   return (split_ws_bytes(tiles, c.splits, c.bn) + 255) & ~static_cast<size_t>(255);
 }
 
@@ -906,9 +940,11 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
       choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes, extra, max_smem);
   int bn = choice.bn, splits = choice.splits;
   bool pair = choice.pair;
+  int64_t full_tiles = choice.full_tiles;
   // Tuning / test overrides: DG_PAIR=0/1 disables / forces the pair form
   // (dense only), DG_BLOCK_N forces the N tile of the single-CTA form,
-  // DG_SPLITS the K split (dense, single-CTA; needs enough workspace).
+  // DG_SPLITS splits every tile's K, DG_TAIL_SPLITS only the last partial
+  // wave's tiles (dense, single-CTA; both need enough workspace).
   if (const char *e = getenv("DG_PAIR")) {
     if (*e == '0') {
       if (pair) {
@@ -919,14 +955,20 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
       pair = true;
       bn = kPairCandidate.bn;
       splits = 1;
+      full_tiles = 0;
     }
   }
   if (const char *e = getenv("DG_BLOCK_N")) {
     const int v = atoi(e);
     for (const Candidate &c : kCandidates)
-      if (c.bn == v && !pair) bn = v;
+      if (c.bn == v && !pair && v != bn) {
+        bn = v;
+        splits = 1;  // the split chosen for another width does not carry over
+        full_tiles = 0;
+      }
   }
   if (const char *e = getenv("DG_SPLITS")) {
+    // every tile split v ways (v = 1: no split)
     const int v = atoi(e);
     if (v >= 1 && !pair) {
       const int64_t tiles = ((rows + BM - 1) / BM) * ((n + bn - 1) / bn);
@@ -935,6 +977,20 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
         return DG_ERR_WORKSPACE;
       if (v > 1 && tiles * v > num_sms) return DG_ERR_INVALID_ARG;  // one unit per CTA
       splits = v;
+      full_tiles = 0;
+    }
+  }
+  if (const char *e = getenv("DG_TAIL_SPLITS")) {
+    // the tiles of a partial last wave split v ways, after whole waves
+    const int v = atoi(e);
+    if (v >= 2 && !pair && sched == kDense) {
+      const int64_t tiles = ((rows + BM - 1) / BM) * ((n + bn - 1) / bn);
+      const int64_t waves = tiles / num_sms, tail = tiles % num_sms;
+      if (waves == 0 || tail == 0 || tail * v > num_sms || v > p.num_k_blocks)
+        return DG_ERR_INVALID_ARG;
+      if (ws == nullptr || split_ws_bytes(tail, v, bn) > ws_bytes) return DG_ERR_WORKSPACE;
+      splits = v;
+      full_tiles = waves * num_sms;
     }
   }
   if (config_smem(bn, pair, extra, sched == kDense) > max_smem)
@@ -943,12 +999,17 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   p.num_m_blocks = static_cast<int>((rows + tile_rows - 1) / tile_rows);
   p.num_n_blocks = static_cast<int>((n + bn - 1) / bn);
   p.splits = splits;
+  p.full_tiles = splits > 1 ? static_cast<int>(full_tiles) : 0;
+  const int64_t all_tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
   if (splits > 1) {
-    const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-    const size_t part = static_cast<size_t>(tiles) * splits * BM * bn * 4;
+    const int64_t split_tiles = all_tiles - p.full_tiles;
+    if (ws == nullptr || split_ws_bytes(split_tiles, splits, bn) > ws_bytes)
+      return DG_ERR_WORKSPACE;
+    const size_t part = static_cast<size_t>(split_tiles) * splits * BM * bn * 4;
     p.ws = static_cast<float *>(ws);
     p.ws_ticket = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + part);
-    if (cudaMemsetAsync(p.ws_ticket, 0, tiles * 4, stream) != cudaSuccess) return DG_ERR_CUDA;
+    if (cudaMemsetAsync(p.ws_ticket, 0, split_tiles * 4, stream) != cudaSuccess)
+      return DG_ERR_CUDA;
   } else {
     p.ws = nullptr;
     p.ws_ticket = nullptr;
@@ -968,7 +1029,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
     // upper bound; the kernel reads the actual count from masked_m
     units = static_cast<int64_t>(p.num_m_blocks) * p.groups * p.num_n_blocks;
   } else {
-    units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks * splits;
+    units = p.full_tiles + (all_tiles - p.full_tiles) * splits;
   }
   int grid;
   if (pair) {
@@ -978,11 +1039,11 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   }
   if (print_configs()) {
     fprintf(stderr,
-            "[dg] gemm sched=%d rows=%lld n=%lld k=%lld groups=%d: %s BN=%d splits=%d grid=%d "
-            "units=%lld\n",
+            "[dg] gemm sched=%d rows=%lld n=%lld k=%lld groups=%d: %s BN=%d splits=%d "
+            "whole=%d grid=%d units=%lld\n",
             sched, static_cast<long long>(rows), static_cast<long long>(n),
-            static_cast<long long>(k), p.groups, pair ? "pair" : "single", bn, splits, grid,
-            static_cast<long long>(units));
+            static_cast<long long>(k), p.groups, pair ? "pair" : "single", bn, splits,
+            p.full_tiles, grid, static_cast<long long>(units));
   }
   switch (sched) {
     case kDense: return dispatch<kDense>(bn, pair, ta, tb, p, grid, extra, stream);

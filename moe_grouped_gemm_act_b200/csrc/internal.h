@@ -42,7 +42,9 @@ struct GemmParams {
   int num_m_blocks;      // ceil(rows / 128)
   int num_n_blocks;      // ceil(n / BN)
   int num_k_blocks;      // k / 128
-  int splits;            // K splits (1 = none)
+  int splits;            // K splits of the split tiles (1 = none)
+  int full_tiles;        // dense: tiles (in raster order) computed whole before
+                         // the remaining ones, each split `splits` ways
   int a_box_rows;        // rows of A per TMA load: 128, or 64 when M <= 64
 };
 

@@ -52,7 +52,12 @@ def test_host_helpers(lib):
     assert "timed out" in dg.status_string(-6)
     assert dg.status_string(12345) == "unknown status"
     assert lib.dg_fp8_gemm_nt_workspace_size(0, 128, 128) == 0
-    assert lib.dg_fp8_gemm_nt_workspace_size(4096, 7168, 7168) == 0   # never splits
+    # 32 x 96 tiles of 128 x 256 fill whole waves closely enough: no split
+    assert lib.dg_fp8_gemm_nt_workspace_size(4096, 24576, 1536) == 0
+    # 32 x 28 = 896 tiles = 6 waves of 148 + 8: the last 8 tiles split 16 ways
+    # (8 x 16 FP32 partial tiles of 128 x 256, then 8 counters, 256-aligned)
+    assert lib.dg_fp8_gemm_nt_workspace_size(4096, 7168, 7168) == \
+        (8 * 16 * 128 * 256 * 4 + 8 * 4 + 255) // 256 * 256
     assert lib.dg_fp8_gemm_nt_workspace_size(64, 7168, 16384) % 256 == 0
 
 

@@ -117,6 +117,23 @@ def test_dense_split_k(splits, bn):
     assert np.array_equal(a, b), "split-K result not deterministic"
 
 
+@pytest.mark.parametrize("splits", [2, 3])
+def test_dense_tail_split(splits):
+    # 8 x 5 = 40 tiles of 128 x 256 (ragged M and N) on 12 CTAs: three whole
+    # waves, then the last 4 tiles split along K over the CTAs
+    qa, alpha, qb, beta = dense_case(1000, 1032, 1024, seed=20 + splits)
+    want = gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta)
+    dg.dg_set_num_sms(12)
+    try:
+        with env(DG_BLOCK_N=256, DG_TAIL_SPLITS=splits):
+            a = run_dense(qa, alpha, qb, beta, workspace=True)
+            b = run_dense(qa, alpha, qb, beta, workspace=True)
+    finally:
+        dg.dg_set_num_sms(0)
+    check_gemm(a, want, f"tail split {splits}")
+    assert np.array_equal(a, b), "tail-split result not deterministic"
+
+
 def test_dense_exact_integers_bit_exact():
     # integer codes in [-4, 4] with unit scales: every 128-K partial and the
     # FP32 running sum are exact, so D must equal BF16(exact) bit for bit
@@ -159,7 +176,10 @@ def test_dense_prefill_full_size_sampled_rows(n, k):
     qa_d, sfa_d = dg.dg_quantize_1x128(torch.from_numpy(x).cuda())
     qb_d, sfb_d = dg.dg_quantize_128x128(torch.from_numpy(w).cuda())
     d = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
-    dg.dg_fp8_gemm_nt(qa_d, sfa_d, qb_d, sfb_d, d)
+    # with the workspace the library asks for, as the bench runs it
+    nbytes = dg.dg_fp8_gemm_nt_workspace_size(m, n, k)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
+    dg.dg_fp8_gemm_nt(qa_d, sfa_d, qb_d, sfb_d, d, workspace=ws)
     torch.cuda.synchronize()
     assert dg.dg_get_device_status() == 0
     g = np.random.default_rng(n + k)
