@@ -60,11 +60,11 @@ FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 # SHA-256 of csrc/gemm.cu + csrc/ptx.cuh + csrc/internal.h; on a mismatch the
 # bench reports null.
 GEMM_TRAFFIC = {
-    "source": "dd79907dc2e955a3",
-    "prefill": 201.7e6,
+    "source": "18b121e5ced4ee13",
+    "prefill": 211.3e6,
     "decode64": 51.8e6,
-    "masked": 540.1e6,
-    "contiguous": 987.9e6,
+    "masked": 533.9e6,
+    "contiguous": 976.5e6,
 }
 
 
