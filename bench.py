@@ -459,6 +459,23 @@ def run_reference(args, rank: int) -> None:
     print(json.dumps(line))
 
 
+def max_over_ranks(values, world: int, device) -> list:
+    """Element-wise maximum of per-rank timings over all ranks (every rank
+    gets the result).  With one rank, the values themselves."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(work_per_step: float, steps: int, world: int, ms: float) -> float:
+    """Whole-job rate: the work all ranks did (each rank runs the same steps
+    on its own replica) over the slowest rank's time, per second."""
+    return work_per_step * steps * world / (ms * 1e-3)
+
+
 def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     import torch
     import torch.distributed as dist
@@ -528,16 +545,14 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     e2e_ms = e0.elapsed_time(e1) * args.steps / e2e_steps
 
     # ------------------------------------------------ max over ranks
-    t = torch.tensor([total_ms, e2e_ms, sum(gemm_ms)], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms, gemm_total_ms = t.tolist()
+    total_ms, e2e_ms, gemm_total_ms = max_over_ranks([total_ms, e2e_ms, sum(gemm_ms)], world,
+                                                     device)
     if rank != 0:
         return
 
     flops_step = data.flops()
-    value = flops_step * args.steps * world / (total_ms * 1e-3) / 1e12
-    e2e = flops_step * args.steps * world / (e2e_ms * 1e-3) / 1e12
+    value = job_throughput(flops_step, args.steps, world, total_ms) / 1e12
+    e2e = job_throughput(flops_step, args.steps, world, e2e_ms) / 1e12
     pk = peaks()
     # dominant kernel: the GEMM
     if spec["bound"] == "tensor":
