@@ -245,6 +245,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   const int u_stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   // ---------------------------------------------------------------- setup
+  // the next kernel of the stream may begin its own set-up as our CTAs leave
+  grid_launch_dependents();
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
@@ -271,6 +273,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       tmem_relinquish();
     }
   }
+  // nothing above touched global memory; from here on the previous kernel's
+  // results (A, the scales, the index arrays) are visible
+  grid_dependency_wait();
   if constexpr (SCHED == kMasked) {
     if (warp == 2) {
       // prefix[e] = sum_{e' < e} ceil(clamp(masked_m[e']) / 128) * n_blocks
@@ -727,22 +732,26 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return DG_ERR_CUDA;
-  } else if constexpr (PAIR) {
+  } else {
+    // programmatic dependent launch: the kernel's set-up overlaps the tail of
+    // the previous kernel (it waits for that grid before touching memory)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0] = pdl_attribute();
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if constexpr (PAIR) {
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = 2;
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = 1;
+      cfg.numAttrs = 2;
+    }
     if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return DG_ERR_CUDA;
-  } else {
-    kern<<<grid, kThreads, smem, stream>>>(ta, tb, p);
   }
   return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }

@@ -20,6 +20,15 @@ int launch_quantize_128x128(const float *w, int64_t G, int64_t N, int64_t K,
                             uint8_t *q, float *sf, int flags,
                             cudaStream_t stream);
 
+// Launch attribute for programmatic dependent launch (the kernel waits for
+// the previous grid on the device, after its own set-up).
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a = {};
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
 // ---------------------------------------------------------------- GEMM
 enum Sched : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 

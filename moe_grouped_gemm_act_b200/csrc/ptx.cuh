@@ -147,6 +147,22 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src,
       : "memory");
 }
 
+// ------------------------------------------------------------------ PDL
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel of the stream is still
+// running.  It does its set-up (barrier initialisation, TMEM allocation,
+// descriptor prefetch) first and calls grid_dependency_wait() before touching
+// global memory: that returns once the previous grid has completed and its
+// memory operations are visible, so stream order holds as before.
+// grid_launch_dependents() lets the next such kernel start early.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ shared
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b,
                                              uint32_t c, uint32_t d) {

@@ -29,6 +29,7 @@
 
 #include "dg.h"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace dg {
 
@@ -116,6 +117,8 @@ __global__ void __launch_bounds__(256)
 quantize_1x128_kernel(const T *__restrict__ x, int64_t batch, int64_t M, int64_t Kg,
                       int64_t ld_x, uint8_t *__restrict__ q, int64_t ld_q,
                       float *__restrict__ sf, int64_t ld_sf, int flags) {
+  grid_launch_dependents();
+  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int sub = lane >> 3, j = lane & 7;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -221,14 +224,24 @@ int launch_quantize_1x128(const void *x, int x_dtype, int64_t batch, int64_t M, 
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;  // 8 x 256 threads per SM
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
+  // one wave of CTAs (all resident), launched as a programmatic dependent
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(threads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   if (x_dtype == DG_DTYPE_F32) {
-    quantize_1x128_kernel<float><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        static_cast<const float *>(x), batch, M, Kg, ld_x, q, ld_q, sf, ld_sf, flags);
+    e = cudaLaunchKernelEx(&cfg, quantize_1x128_kernel<float>, static_cast<const float *>(x),
+                           batch, M, Kg, ld_x, q, ld_q, sf, ld_sf, flags);
   } else {
-    quantize_1x128_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(x), batch, M, Kg, ld_x, q, ld_q, sf, ld_sf, flags);
+    e = cudaLaunchKernelEx(&cfg, quantize_1x128_kernel<__nv_bfloat16>,
+                           static_cast<const __nv_bfloat16 *>(x), batch, M, Kg, ld_x, q, ld_q, sf,
+                           ld_sf, flags);
   }
-  return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
 int launch_quantize_128x128(const float *w, int64_t G, int64_t N, int64_t K, uint8_t *q,
