@@ -68,6 +68,7 @@ constexpr int kPromoThreads = 32 * kPromoWarps;
 constexpr int kThreads = 32 * (kControlWarps + kPromoWarps);
 constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
+constexpr int kClusterNoFit = 1;        // launch_instance: clusters do not fit one wave
 
 template <int BN, int STAGES, int NBUF, bool PAIR, bool STAGED>
 struct Layout {
@@ -595,6 +596,23 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
         continue;  // this split's share of D is written
       }
+      if constexpr (SCHED == kDenseCluster) {
+        // Leave this split's FP32 partial in this CTA's shared memory (the
+        // stage ring, drained: every block's MMAs have completed) for the
+        // cluster reduction after the role loops.  Layout [128 rows][BN/4]
+        // 16-byte chunks, chunk c of row r at c ^ (r mod kSwF): the
+        // row-per-lane writes and the row-major reads are both conflict-free.
+        constexpr int kChunksF = BN / 4;
+        constexpr int kSwF = kChunksF < 8 ? kChunksF : 8;
+        float4 *s_part = reinterpret_cast<float4 *>(smem);
+#pragma unroll
+        for (int c = 0; c < W; c += 4) {
+          const int chunk = (half * W + c) / 4;
+          s_part[row_in_tile * kChunksF + (chunk ^ (row_in_tile % kSwF))] =
+              make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+        }
+        continue;  // one unit per CTA in this schedule
+      }
       if constexpr (!kStaged) {
         // each thread stores its row segment (valid rows), 16 bytes at a time
         if (row_ok) {
@@ -673,6 +691,49 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
   }
 
+  // ------------------------------------------------ cluster split reduction
+  // The splits of a tile are the CTAs of one cluster (rank = split).  Every
+  // thread of every CTA passes both cluster barriers, whatever happened in
+  // its role loop, so none can strand the others.
+  if constexpr (SCHED == kDenseCluster) {
+    __syncwarp();
+    cluster_sync();  // all partials written
+    if (warp >= kControlWarps && !*s_abort) {
+      const Tile t = unit_to_tile(p, SCHED, static_cast<int>(blockIdx.x), s_prefix, s_mblocks);
+      constexpr int kChunksF = BN / 4;
+      constexpr int kSwF = kChunksF < 8 ? kChunksF : 8;
+      const int split = static_cast<int>(cluster_ctarank());
+      const int row0 = t.m_blk * BM;
+      const int valid = min(BM, p.rows - row0);
+      const int total = valid * kChunksF;  // row-major chunks of the valid rows
+      const int share = (total + p.splits - 1) / p.splits;
+      const int f_end = min(total, (split + 1) * share);
+      const int ptid = threadIdx.x - kControlWarps * 32;
+      for (int f = split * share + ptid; f < f_end; f += kPromoThreads) {
+        const int r = f / kChunksF, c = f - r * kChunksF;
+        const uint32_t off = base + 16u * (r * kChunksF + (c ^ (r % kSwF)));
+        float4 sum = ld_shared_cluster_v4(mapa_shared(off, 0));
+        for (int q = 1; q < p.splits; ++q) {  // split order: deterministic
+          const float4 v = ld_shared_cluster_v4(mapa_shared(off, static_cast<uint32_t>(q)));
+          sum.x += v.x;
+          sum.y += v.y;
+          sum.z += v.z;
+          sum.w += v.w;
+        }
+        const int col = t.n_blk * BN + 4 * c;
+        if (col < p.n) {
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y);
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z, sum.w);
+          uint2 v;
+          v.x = *reinterpret_cast<const uint32_t *>(&lo);
+          v.y = *reinterpret_cast<const uint32_t *>(&hi);
+          *reinterpret_cast<uint2 *>(p.d + static_cast<int64_t>(row0 + r) * p.n + col) = v;
+        }
+      }
+    }
+    cluster_sync();  // no CTA leaves while its partial is being read
+  }
+
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
@@ -705,6 +766,11 @@ constexpr int smem_bytes_for(int extra) {
   return 1024 + Layout<BN, STAGES, NBUF, PAIR, STAGED>::kPrefixOff + extra;
 }
 
+bool print_configs() {
+  const char *e = getenv("DG_PRINT_CONFIGS");
+  return e && *e && *e != '0';
+}
+
 template <int BN, int STAGES, int NBUF, int SCHED, bool PAIR>
 int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                     int grid, int extra_smem, cudaStream_t stream, bool coop) {
@@ -718,6 +784,38 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
         cudaSuccess)
       return DG_ERR_CUDA;
     configured_smem[dev] = smem;
+  }
+  // clusters: the CTA pair, or the `splits` CTAs of a tile
+  const int cluster = PAIR ? 2 : SCHED == kDenseCluster ? p.splits : 1;
+  if constexpr (SCHED == kDenseCluster) {
+    // every cluster must be resident at once (one wave): ask the occupancy
+    // calculator how many clusters of this size fit (cached per device)
+    static int fit[64][9] = {};  // max active clusters + 1; 0 = not asked yet
+    if (cluster < 2 || cluster > 8) return kClusterNoFit;
+    if (fit[dev][cluster] == 0) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(grid);
+      q.blockDim = dim3(kThreads);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = cluster;
+      a[0].val.clusterDim.y = 1;
+      a[0].val.clusterDim.z = 1;
+      q.attrs = a;
+      q.numAttrs = 1;
+      int n = 0;
+      const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &q);
+      if (e != cudaSuccess) {
+        cudaGetLastError();  // clear: the caller falls back to the other path
+        n = 0;
+      }
+      if (print_configs())
+        fprintf(stderr, "[dg] BN=%d clusters of %d: at most %d resident (%s)\n", BN, cluster, n,
+                cudaGetErrorString(e));
+      fit[dev][cluster] = n + 1;
+    }
+    if (grid / cluster > fit[dev][cluster] - 1) return kClusterNoFit;
   }
   if (coop) {
     // the splits of a tile wait for each other: all CTAs must be resident
@@ -744,9 +842,9 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
     attr[0] = pdl_attribute();
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if constexpr (PAIR) {
+    if (cluster > 1) {
       attr[1].id = cudaLaunchAttributeClusterDimension;
-      attr[1].val.clusterDim.x = 2;
+      attr[1].val.clusterDim.x = cluster;
       attr[1].val.clusterDim.y = 1;
       attr[1].val.clusterDim.z = 1;
       cfg.numAttrs = 2;
@@ -789,7 +887,9 @@ int max_smem_per_block() {
 template <int SCHED>
 int dispatch(int bn, bool pair, const CUtensorMap &ta, const CUtensorMap &tb,
              const GemmParams &p, int grid, int extra, cudaStream_t st) {
-  const bool coop = p.splits > 1;
+  // splits that wait for each other through global memory need all CTAs
+  // resident; a cluster's splits are co-scheduled by construction
+  const bool coop = p.splits > 1 && SCHED != kDenseCluster;
   if (pair) {
     if constexpr (SCHED == kDense) {
       return launch_instance<kPairCandidate.bn, kPairCandidate.stages, kPairCandidate.nbuf,
@@ -825,10 +925,6 @@ int make_tmap(CUtensorMap *m, const void *ptr, int64_t k, int64_t rows, int64_t 
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
-bool print_configs() {
-  const char *e = getenv("DG_PRINT_CONFIGS");
-  return e && *e && *e != '0';
-}
 
 // Cycles one CTA spends per 128-K block of a unit, measured on B200.  The
 // tensor cores take ~540 cycles per block for any N up to 256 (one
@@ -950,6 +1046,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   int bn = choice.bn, splits = choice.splits;
   bool pair = choice.pair;
   int64_t full_tiles = choice.full_tiles;
+  bool splits_forced = false;  // DG_SPLITS: exactly this many, or none
   // Tuning / test overrides: DG_PAIR=0/1 disables / forces the pair form
   // (dense only), DG_BLOCK_N forces the N tile of the single-CTA form,
   // DG_SPLITS splits every tile's K, DG_TAIL_SPLITS only the last partial
@@ -987,6 +1084,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
       if (v > 1 && tiles * v > num_sms) return DG_ERR_INVALID_ARG;  // one unit per CTA
       splits = v;
       full_tiles = 0;
+      splits_forced = true;
     }
   }
   if (const char *e = getenv("DG_TAIL_SPLITS")) {
@@ -1010,7 +1108,18 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   p.splits = splits;
   p.full_tiles = splits > 1 ? static_cast<int>(full_tiles) : 0;
   const int64_t all_tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-  if (splits > 1) {
+  p.ws = nullptr;
+  p.ws_ticket = nullptr;
+  // Every tile split (decode-sized shapes, one wave): the splits of a tile
+  // form a cluster and reduce through distributed shared memory, needing no
+  // workspace or arrival counters, when all clusters fit in one wave
+  // (DG_CLUSTER_SPLIT=0 forces the workspace path).
+  bool try_cluster = sched == kDense && !pair && splits > 1 && splits <= 8 &&
+                     p.full_tiles == 0 && all_tiles * splits <= num_sms;
+  if (const char *e = getenv("DG_CLUSTER_SPLIT"))
+    if (*e == '0') try_cluster = false;
+  // the workspace path: FP32 partials and one arrival counter per split tile
+  auto setup_workspace = [&]() -> int {
     const int64_t split_tiles = all_tiles - p.full_tiles;
     if (ws == nullptr || split_ws_bytes(split_tiles, splits, bn) > ws_bytes)
       return DG_ERR_WORKSPACE;
@@ -1019,9 +1128,11 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
     p.ws_ticket = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + part);
     if (cudaMemsetAsync(p.ws_ticket, 0, split_tiles * 4, stream) != cudaSuccess)
       return DG_ERR_CUDA;
-  } else {
-    p.ws = nullptr;
-    p.ws_ticket = nullptr;
+    return DG_OK;
+  };
+  if (splits > 1 && !try_cluster) {
+    const int rc = setup_workspace();
+    if (rc) return rc;
   }
 
   // ------------------------------------------------ tensor maps
@@ -1045,6 +1156,34 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
     grid = 2 * static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms / 2)));
   } else {
     grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
+  }
+  if (try_cluster) {
+    // the chosen split, else (unless forced) fewer splits while the grid
+    // still keeps 3/5 of the SMs busy
+    int rc = kClusterNoFit;
+    const int chosen = p.splits;
+    const int lowest = splits_forced ? chosen : 2;
+    for (int sc = chosen; sc >= lowest && rc == kClusterNoFit; --sc) {
+      if (sc < chosen && all_tiles * sc * 5 < static_cast<int64_t>(num_sms) * 3) break;
+      p.splits = sc;
+      grid = static_cast<int>(all_tiles * sc);
+      rc = dispatch<kDenseCluster>(bn, false, ta, tb, p, grid, extra, stream);
+    }
+    if (rc == kClusterNoFit) {
+      p.splits = chosen;
+      grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
+    }
+    if (rc != kClusterNoFit) {
+      if (print_configs())
+        fprintf(stderr,
+                "[dg] gemm sched=dense rows=%lld n=%lld k=%lld: single BN=%d splits=%d "
+                "(cluster reduction) grid=%d\n",
+                static_cast<long long>(rows), static_cast<long long>(n),
+                static_cast<long long>(k), bn, p.splits, grid);
+      return rc;
+    }
+    const int wrc = setup_workspace();  // the clusters do not fit one wave
+    if (wrc) return wrc;
   }
   if (print_configs()) {
     fprintf(stderr,

@@ -30,7 +30,10 @@ inline cudaLaunchAttribute pdl_attribute() {
 }
 
 // ---------------------------------------------------------------- GEMM
-enum Sched : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+// kDenseCluster: dense tiles every one split `splits` ways along K, the splits
+// of a tile forming one thread-block cluster that reduces through
+// distributed shared memory (decode-sized shapes; no workspace).
+enum Sched : int { kDense = 0, kContiguous = 1, kMasked = 2, kDenseCluster = 3 };
 
 // Kernel parameters besides the two tensor maps.  Row coordinates are inside
 // one "slab": the whole of A for dense and contiguous, one expert's M_max rows

@@ -323,7 +323,8 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
-// All threads of both CTAs of the cluster.
+// All threads of every CTA of the cluster (release / acquire: shared-memory
+// writes before it are visible to the cluster's reads after it).
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
                "barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -335,6 +336,16 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
+}
+
+// 16 bytes from the cluster shared window (this or a peer CTA's memory).
+__device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
 // Arrive on an mbarrier given by its cluster-window address (possibly in the

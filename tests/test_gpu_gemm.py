@@ -106,15 +106,30 @@ def test_dense_pair_exact_integers_bit_exact():
 
 
 @pytest.mark.parametrize("splits", [2, 3, 8])
-@pytest.mark.parametrize("bn", [32, 128])
+@pytest.mark.parametrize("bn", [32, 128, 256])
 def test_dense_split_k(splits, bn):
+    # both reductions: the splits of a tile as one cluster (distributed shared
+    # memory) and through the workspace; both sum the splits in order, so
+    # they must agree bit for bit
     qa, alpha, qb, beta = dense_case(64, 528, 2048, seed=splits)
     want = gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta)
-    with env(DG_BLOCK_N=bn, DG_SPLITS=splits):
+    with env(DG_BLOCK_N=bn, DG_SPLITS=splits, DG_CLUSTER_SPLIT=1):
         a = run_dense(qa, alpha, qb, beta, workspace=True)
         b = run_dense(qa, alpha, qb, beta, workspace=True)
+    with env(DG_BLOCK_N=bn, DG_SPLITS=splits, DG_CLUSTER_SPLIT=0):
+        c = run_dense(qa, alpha, qb, beta, workspace=True)
     check_gemm(a, want, f"split {splits}")
     assert np.array_equal(a, b), "split-K result not deterministic"
+    assert np.array_equal(a, c), "cluster and workspace reductions differ"
+
+
+def test_dense_split_k_cluster_ragged_rows():
+    # M = 200: two M blocks, the second with 72 valid rows; N ragged
+    qa, alpha, qb, beta = dense_case(200, 776, 3072, seed=31)
+    want = gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta)
+    with env(DG_BLOCK_N=128, DG_SPLITS=4, DG_CLUSTER_SPLIT=1):
+        got = run_dense(qa, alpha, qb, beta, workspace=True)
+    check_gemm(got, want, "cluster split, ragged")
 
 
 @pytest.mark.parametrize("splits", [2, 3])
