@@ -74,7 +74,9 @@ constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 constexpr int kClusterNoFit = 1;        // launch_instance: clusters do not fit one wave
 
 // Schedules whose epilogue stages the BF16 tile in shared memory.
-constexpr bool staged_epilogue(int sched) { return sched == kDense || sched == kMasked; }
+__host__ __device__ constexpr bool staged_epilogue(int sched) {
+  return sched == kDense || sched == kMasked;
+}
 
 template <int BN, int STAGES, int NBUF, bool PAIR, bool STAGED>
 struct Layout {
