@@ -60,11 +60,12 @@ FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 # SHA-256 of csrc/gemm.cu + csrc/ptx.cuh + csrc/internal.h; on a mismatch the
 # bench reports null.
 GEMM_TRAFFIC = {
-    "source": "18b121e5ced4ee13",
-    "prefill": 211.3e6,
-    "decode64": 51.8e6,
-    "masked": 533.9e6,
-    "contiguous": 976.5e6,
+    "source": "aab113a73d8421b0",
+    "prefill": 210.6e6,
+    "decode64": 51.3e6,
+    "decode128": 51.9e6,
+    "masked": 533.8e6,
+    "contiguous": 956.7e6,
 }
 
 
