@@ -324,6 +324,9 @@ class GroupedData(DenseData):
         w = inputs.weights((G, n, k), seed=spec["seed"] + 2)
         a32 = torch.from_numpy(x).to(device)
         qb, sfb = dg.dg_quantize_128x128(torch.from_numpy(w).to(device))
+        # host inputs for the oracle's timed sample (a few experts' rows and
+        # the first columns of their weights)
+        self.sample_src = GroupedOracleSample.source(spec, x, w, index.cpu().numpy())
         del w
         qa, sfa = dg.dg_quantize_1x128(a32)
         d = torch.empty(d_shape, dtype=torch.bfloat16, device=device)
@@ -414,6 +417,86 @@ class OracleSample:
         return time.perf_counter() - t0, flops
 
 
+class GroupedOracleSample:
+    """The CPU oracle on a bounded sample of a grouped workload: the first
+    ``experts`` experts holding rows, up to ``rows`` of each expert's rows and
+    the first ``cols`` columns of D over the full K.  One run = quantize the
+    sampled A rows (1x128) and run the oracle's masked or contiguous GEMM on
+    that sub-problem (weights quantized once beforehand, as on the GPU)."""
+
+    EXPERTS = 2
+
+    @staticmethod
+    def source(spec, x, w, index):
+        """The slices the sample needs, from the workload's host inputs."""
+        cols = 1024
+        picked = []
+        for e in range(spec["groups"]):
+            if spec["kind"] == "masked":
+                rows = x[e, :int(index[e])]
+            else:
+                rows = x[index == e]
+            if len(rows):
+                picked.append((rows[:64].copy(), w[e, :cols].copy()))
+            if len(picked) == GroupedOracleSample.EXPERTS:
+                break
+        return picked
+
+    def __init__(self, spec, rows: int, cols: int, src=None):
+        from oracle import quant as oq
+        self.kind = spec["kind"]
+        self.k = spec["k"]
+        if src is None:
+            src = self.source(spec, *self._generate(spec))
+        self.prepared = []
+        for xr, wc in src:
+            xr, wc = xr[:rows], wc[:cols]
+            qb, beta = oq.quantize_128x128(wc)
+            self.prepared.append((xr, qb, beta))
+        c = min(cols, spec["n"])
+        self.desc = (f"{rows} rows of each of the first {len(self.prepared)} experts with rows "
+                     f"x first {c} columns of D, full K ({self.kind} oracle)")
+
+    @staticmethod
+    def _generate(spec):
+        G, k = spec["groups"], spec["k"]
+        w = inputs.weights((G, spec["n"], k), seed=spec["seed"] + 2)
+        if spec["kind"] == "masked":
+            counts = inputs.masked_counts(G, spec["m_max"], seed=spec["seed"])
+            x = inputs.activations(G * spec["m_max"], k, seed=spec["seed"] + 1,
+                                   outliers=True).reshape(G, spec["m_max"], k)
+            return x, w, counts
+        lay = inputs.contiguous_layout(spec["tokens"], G, seed=spec["seed"])
+        x = inputs.activations(lay.m_total, k, seed=spec["seed"] + 1, outliers=True)
+        return x, w, lay.m_indices
+
+    def run(self) -> tuple[float, float]:
+        """Returns (seconds, FLOPs) of one pass."""
+        from oracle import gemm as og, quant as oq
+        t0 = time.perf_counter()
+        qas = [oq.quantize_1x128(xr) for xr, _, _ in self.prepared]
+        qb = np.stack([q for _, q, _ in self.prepared])
+        beta = np.stack([b for _, _, b in self.prepared])
+        n_rows = [len(xr) for xr, _, _ in self.prepared]
+        c = qb.shape[1]
+        if self.kind == "masked":
+            m = max(n_rows)
+            qa = np.zeros((len(qas), m, self.k), np.uint8)
+            alpha = np.zeros((len(qas), m, self.k // 128), np.float32)
+            for e, (q, a) in enumerate(qas):
+                qa[e, :len(q)], alpha[e, :len(a)] = q, a
+            og.m_grouped_masked(qa, alpha, qb, beta, np.array(n_rows, np.int32),
+                                np.zeros((len(qas), m, c), np.uint16))
+        else:
+            qa = np.concatenate([q for q, _ in qas])
+            alpha = np.concatenate([a for _, a in qas])
+            idx = np.concatenate([np.full(r, e, np.int32) for e, r in enumerate(n_rows)])
+            og.m_grouped_contiguous(qa, alpha, qb, beta, idx,
+                                    np.zeros((len(idx), c), np.uint16))
+        flops = 2.0 * sum(n_rows) * c * self.k
+        return time.perf_counter() - t0, flops
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -431,11 +514,10 @@ def run_reference(args, rank: int) -> None:
     if rank != 0:
         return
     spec = workload_spec(args.workload)
-    if spec["kind"] != "dense":
-        print(json.dumps({"impl": "reference", "unavailable":
-                          "reference arm implemented for the dense workloads only"}))
-        return
-    sampler = OracleSample(spec, args.ref_rows, args.ref_cols)
+    if spec["kind"] == "dense":
+        sampler = OracleSample(spec, args.ref_rows, args.ref_cols)
+    else:
+        sampler = GroupedOracleSample(spec, args.ref_rows, args.ref_cols)
     for _ in range(args.warmup):
         sampler.run()
     secs, flops = 0.0, 0.0
@@ -574,8 +656,12 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                  for s, ms in zip(data.shapes, per_shape_ms)]
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline and spec["kind"] == "dense":
-        sampler = OracleSample(spec, args.ref_rows, args.ref_cols)
+    if world == 1 and not args.no_cpu_baseline:
+        if spec["kind"] == "dense":
+            sampler = OracleSample(spec, args.ref_rows, args.ref_cols)
+        else:
+            sampler = GroupedOracleSample(spec, args.ref_rows, args.ref_cols,
+                                          src=data.sample_src)
         sampler.run()
         secs, fl = 0.0, 0.0
         while secs < 10.0:          # about 10 s of CPU work

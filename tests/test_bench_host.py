@@ -1,0 +1,51 @@
+"""Host-side pieces of bench.py that run without a GPU: the oracle samples
+behind `cpu_baseline` and the reference arm, on tiny versions of the grouped
+workloads."""
+
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from moe_grouped_gemm_act_b200 import inputs  # noqa: E402
+
+
+@pytest.mark.parametrize("kind", ["masked", "contiguous"])
+def test_grouped_oracle_sample_counts_valid_rows(kind):
+    spec = dict(kind=kind, groups=4, n=256, k=256, seed=3, m_max=64, tokens=300)
+    s = bench.GroupedOracleSample(spec, rows=8, cols=128)
+    secs, flops = s.run()
+    assert secs > 0
+    n_rows = sum(len(xr) for xr, _, _ in s.prepared)
+    assert 0 < n_rows <= 8 * bench.GroupedOracleSample.EXPERTS
+    assert flops == 2.0 * n_rows * 128 * 256
+
+
+def test_grouped_oracle_sample_takes_experts_with_rows():
+    # masked: experts with zero valid rows are skipped
+    spec = dict(kind="masked", groups=6, n=128, k=128, seed=0, m_max=32)
+    counts = inputs.masked_counts(6, 32, seed=0)
+    s = bench.GroupedOracleSample(spec, rows=64, cols=128)
+    want = [int(c) for c in counts if c > 0][:bench.GroupedOracleSample.EXPERTS]
+    assert [len(xr) for xr, _, _ in s.prepared] == [min(c, 64) for c in want]
+
+
+def test_workload_specs_name_their_bound():
+    for name, bound in [("prefill", "tensor"), ("decode64", "hbm"), ("decode128", "hbm"),
+                        ("contiguous", "tensor"), ("masked", "hbm")]:
+        assert bench.workload_spec(name)["bound"] == bound
+    with pytest.raises(SystemExit):
+        bench.workload_spec("nope")
+
+
+def test_measured_traffic_follows_the_source_hash(monkeypatch):
+    monkeypatch.setitem(bench.GEMM_TRAFFIC, "source", bench.gemm_source_hash())
+    assert bench.measured_traffic("prefill") == bench.GEMM_TRAFFIC["prefill"]
+    monkeypatch.setitem(bench.GEMM_TRAFFIC, "source", "0" * 16)
+    assert bench.measured_traffic("prefill") is None
+    assert np.isfinite(bench.job_throughput(1.0, 1, 1, 1.0))
