@@ -143,11 +143,15 @@ int dg_quantize_128x128(const float *w, int64_t G, int64_t N, int64_t K,
  *   D      device BF16 [M][N] row-major, written for all i < M, j < N.
  *   workspace, workspace_bytes
  *          optional device scratch (may be NULL / 0).  When at least
- *          dg_fp8_gemm_nt_workspace_size(M, N, K) bytes are given, small-M
- *          (decode) shapes may split K across CTAs: FP32 partial results go
- *          to the workspace and the last CTA of each tile sums them in a fixed
- *          order.  The workspace must not be used by another call that runs
- *          at the same time; its contents between calls do not matter.
+ *          dg_fp8_gemm_nt_workspace_size(M, N, K) bytes are given, the GEMM
+ *          may split K across CTAs: small-M (decode) shapes split every tile,
+ *          large shapes only the tiles of a last, partial wave of CTAs.  A
+ *          decode tile's splits usually form one thread-block cluster and
+ *          sum their partials in on-chip shared memory, leaving the workspace
+ *          unused; otherwise FP32 partials go to the workspace and the splits
+ *          of a tile sum them there.  Either way the splits are added in a
+ *          fixed order.  The workspace must not be used by another call that
+ *          runs at the same time; its contents between calls do not matter.
  *   M >= 0 (0 is a no-op), N > 0 with N % 8 == 0, K > 0 with K % 128 == 0.
  * Deterministic: repeated calls give identical bits (also with split K).
  */
