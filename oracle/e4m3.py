@@ -5,7 +5,7 @@ Lesson 13, Fig. 13-1 and the answer to Q1: E4M3 has 8 bits -- 1 sign bit,
 maximum of 448 fixes the FN variant: exponent field 15 is an ordinary binade
 and only the all-ones pattern (0x7F / 0xFF) is NaN.  The exponent bias is 7.
 
-Readings taken where the pages are silent (each listed in the design doc):
+Readings taken where the pages are silent:
 
 * rounding is round-to-nearest, ties to the even code (mantissa LSB 0);
 * magnitudes above 448 saturate to 448 ("satfinite");

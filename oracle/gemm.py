@@ -26,8 +26,8 @@ section 3, the grouped GEMM table):
   valid; only those rows are computed.
 
 Rows that are not computed (padding, rows >= masked_m[g]) are left exactly as
-they were in the output (reading stated in the design doc); the oracle copies the
-caller's initial output for them.
+they were in the output (the pages do not say; this is the reading taken);
+the oracle copies the caller's initial output for them.
 """
 
 from __future__ import annotations

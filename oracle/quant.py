@@ -8,7 +8,7 @@ blocks") and the answer to Q1:
 * weight B [N, K]: one FP32 scale beta per 128 x 128 block, quantized offline;
 * scales are FP32; newer versions also allow UE8M0 (power-of-two) scales.
 
-Readings taken where the pages are silent (listed in the design doc):
+Readings taken where the pages are silent:
 
 * the code of an element is E4M3_RNE(fl32(x / alpha)): the float32 quotient,
   correctly rounded, then rounded to E4M3 (ties to even, satfinite);
