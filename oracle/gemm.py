@@ -72,6 +72,22 @@ def fp8_gemm_nt(qa, alpha, qb, beta) -> np.ndarray:
     return bf16.to_bits(fp8_gemm_nt_f64(qa, alpha, qb, beta))
 
 
+def fp8_gemm_nt_accumulate_f64(qa, alpha, qb, beta, c) -> np.ndarray:
+    """float64 C + A B^T (Deep dive, section 3: the NT GEMM's D = C + A @ B.T
+    form), with C float32 [M, N] taken exactly and added to the float64
+    result of the Fig. 13-1 formula."""
+    d = fp8_gemm_nt_f64(qa, alpha, qb, beta)
+    c64 = np.asarray(c, np.float64)
+    if c64.shape != d.shape:
+        raise ValueError("C must be [M, N]")
+    return c64 + d
+
+
+def fp8_gemm_nt_accumulate(qa, alpha, qb, beta, c) -> np.ndarray:
+    """BF16 bit patterns of D = C + A B^T, rounded once."""
+    return bf16.to_bits(fp8_gemm_nt_accumulate_f64(qa, alpha, qb, beta, c))
+
+
 def m_grouped_contiguous_f64(qa, alpha, qb, beta, m_indices, d_init):
     """Contiguous m-grouped GEMM in float64.
 

@@ -215,3 +215,52 @@ def test_masked_clamps_out_of_range_counts():
                                 np.zeros((G, m_max, N), np.uint16))
     assert np.all(out[0] == 0)
     assert np.all(bf16.from_bits(out[1]) == 128.0)
+
+
+# ------------------------------------------------------------- D = C + A B^T
+def test_accumulate_with_zero_c_is_the_plain_gemm():
+    qa, alpha, qb, beta = small_case(m=24, n=200, k=384, seed=41)
+    c = np.zeros((24, 200), np.float32)
+    assert np.array_equal(gemm.fp8_gemm_nt_accumulate(qa, alpha, qb, beta, c),
+                          gemm.fp8_gemm_nt(qa, alpha, qb, beta))
+
+
+def test_accumulate_with_zero_product_rounds_c_like_torch():
+    import torch
+    g = np.random.default_rng(42)
+    c = (g.standard_normal((16, 136)) * 7).astype(np.float32)
+    qa = np.zeros((16, 256), np.uint8)                      # all +0.0
+    qb = e4m3.encode_rne(g.standard_normal((136, 256)).astype(np.float32))
+    got = gemm.fp8_gemm_nt_accumulate(qa, np.ones((16, 2), np.float32), qb,
+                                      np.ones((2, 2), np.float32), c)
+    want = torch.from_numpy(c).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_accumulate_integer_exact():
+    g = np.random.default_rng(43)
+    M, N, K = 8, 64, 512
+    a = g.integers(-4, 5, size=(M, K)).astype(np.float32)
+    b = g.integers(-4, 5, size=(N, K)).astype(np.float32)
+    c = g.integers(-100, 101, size=(M, N)).astype(np.float32)
+    d = gemm.fp8_gemm_nt_accumulate_f64(e4m3.encode_rne(a), np.ones((M, 4), np.float32),
+                                        e4m3.encode_rne(b), np.ones((1, 4), np.float32), c)
+    assert np.array_equal(d, a.astype(np.int64) @ b.astype(np.int64).T + c.astype(np.int64))
+
+
+def test_accumulate_rounds_once_after_adding_c():
+    # A.B = 1 + 2^-8 (a tie between two BF16 values, rounding to 1.0) and
+    # C = 2^-8: rounding once gives BF16(1 + 2^-7) = 0x3F81; rounding the
+    # product first and then adding C would give 0x3F80
+    qa = np.zeros((1, 128), np.uint8)
+    qb = np.zeros((1, 128), np.uint8)
+    a = np.zeros((1, 128), np.float32)
+    a[0, 0], a[0, 1] = 1.0, 2.0 ** -8
+    qa[:] = e4m3.encode_rne(a)
+    qb[0, 0], qb[0, 1] = e4m3.encode_rne(np.array([1.0, 1.0], np.float32))
+    one = np.ones((1, 1), np.float32)
+    assert gemm.fp8_gemm_nt_f64(qa, one, qb, one)[0, 0] == 1.0 + 2.0 ** -8
+    c = np.array([[2.0 ** -8]], np.float32)
+    assert gemm.fp8_gemm_nt_accumulate(qa, one, qb, one, c)[0, 0] == 0x3F81
+    twice = bf16.to_bits(bf16.round_f64(gemm.fp8_gemm_nt_f64(qa, one, qb, one)) + c)
+    assert twice[0, 0] == 0x3F80
