@@ -96,6 +96,12 @@ def workload_spec(name: str) -> dict:
                          "{(7168,16384),(4096,7168),(24576,1536),(2112,7168)}; "
                          "A~N(0,1) with 0.1% x50 outliers, B~N(0,0.02); "
                          "1x128 / 128x128 FP32 scales, BF16 out")
+    if name == "prefill_acc":
+        return dict(name=name, kind="dense", m=inputs.PREFILL_M, nk=inputs.PREFILL_NK,
+                    seeds=inputs.PREFILL_SEEDS, bound="tensor", acc=True,
+                    desc="dense NT prefill with D = C + A*B^T, C FP32 ~ N(0,16) [M,N], "
+                         "M=4096, (N,K) in {(7168,16384),(4096,7168),(24576,1536),"
+                         "(2112,7168)}; A, B and scales as prefill")
     if name in ("decode64", "decode128"):
         m = 64 if name == "decode64" else 128
         return dict(name=name, kind="dense", m=m, nk=inputs.PREFILL_NK,
@@ -202,7 +208,9 @@ class DenseData:
         self.dg = dg
         m = spec["m"]
         self.m = m
+        self.acc = bool(spec.get("acc"))
         self.shapes = []
+        gen = torch.Generator(device=device)
         for n, k in spec["nk"]:
             x = inputs.activations(m, k, seed=spec["seeds"]["seed_a"] + k, outliers=True)
             w = inputs.weights((n, k), seed=spec["seeds"]["seed_b"] + n + k)
@@ -214,8 +222,12 @@ class DenseData:
             d = torch.empty((m, n), dtype=torch.bfloat16, device=device)
             wsb = dg.dg_fp8_gemm_nt_workspace_size(m, n, k)
             ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=device) if wsb else None
+            c = None
+            if self.acc:  # D = C + A B^T: a seeded FP32 C per shape
+                gen.manual_seed(spec["seeds"]["seed_a"] + 7 * k + n)
+                c = torch.randn((m, n), generator=gen, device=device, dtype=torch.float32) * 4
             self.shapes.append(dict(n=n, k=k, a32=a32, qb=qb, sfb=sfb, qa=qa, sfa=sfa, d=d,
-                                    ws=ws, x_host=x, w_host=w))
+                                    ws=ws, x_host=x, w_host=w, c=c))
         torch.cuda.synchronize()
 
     def flops(self) -> float:
@@ -228,10 +240,17 @@ class DenseData:
             n, k = s["n"], s["k"]
             tot += self.m * k + 4 * self.m * (k // 128) + n * k + \
                 4 * (-(-n // 128)) * (k // 128) + 2 * self.m * n
+            if self.acc:
+                tot += 4 * self.m * n  # C
         return tot
 
     def gemm(self, s):
-        self.dg.dg_fp8_gemm_nt(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"], workspace=s["ws"])
+        if self.acc:
+            self.dg.dg_fp8_gemm_nt_accumulate(s["qa"], s["sfa"], s["qb"], s["sfb"], s["c"], s["d"],
+                                              workspace=s["ws"])
+        else:
+            self.dg.dg_fp8_gemm_nt(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"],
+                                   workspace=s["ws"])
 
     def step(self):
         """One pass of the hot path: for every shape, quantize A, then GEMM."""
@@ -275,9 +294,10 @@ class DenseData:
             self.host.append(dict(
                 a=torch.from_numpy(s["x_host"]).pin_memory(),
                 qb=s["qb"].cpu().pin_memory(), sfb=s["sfb"].cpu().pin_memory(),
+                c=None if s["c"] is None else s["c"].cpu().pin_memory(),
                 d=torch.empty(s["d"].shape, dtype=torch.bfloat16).pin_memory()))
-        self.h2d = sum(h["a"].numel() * 4 + h["qb"].numel() + h["sfb"].numel() * 4
-                       for h in self.host)
+        self.h2d = sum(h["a"].numel() * 4 + h["qb"].numel() + h["sfb"].numel() * 4 +
+                       (0 if h["c"] is None else h["c"].numel() * 4) for h in self.host)
         self.d2h = sum(h["d"].numel() * 2 for h in self.host)
 
     def e2e_step(self, device):
@@ -287,7 +307,11 @@ class DenseData:
             qb = h["qb"].to(device, non_blocking=True)
             sfb = h["sfb"].to(device, non_blocking=True)
             qa, sfa = dg.dg_quantize_1x128(a)
-            dg.dg_fp8_gemm_nt(qa, sfa, qb, sfb, s["d"], workspace=s["ws"])
+            if h["c"] is not None:
+                c = h["c"].to(device, non_blocking=True)
+                dg.dg_fp8_gemm_nt_accumulate(qa, sfa, qb, sfb, c, s["d"], workspace=s["ws"])
+            else:
+                dg.dg_fp8_gemm_nt(qa, sfa, qb, sfb, s["d"], workspace=s["ws"])
             h["d"].copy_(s["d"], non_blocking=True)
 
 
@@ -395,24 +419,30 @@ class OracleSample:
     def __init__(self, spec, rows: int, cols: int):
         from oracle import quant as oq
         self.prepared = []
+        self.acc = bool(spec.get("acc"))
+        g = np.random.default_rng(spec["seeds"]["seed_a"])
         for n, k in spec["nk"]:
             x = inputs.activations(spec["m"], k, seed=spec["seeds"]["seed_a"] + k,
                                    outliers=True)
             w = inputs.weights((n, k), seed=spec["seeds"]["seed_b"] + n + k)
             c = min(n, cols)
             qb, beta = oq.quantize_128x128(w[:c])
-            self.prepared.append((x[:rows].copy(), qb, beta, c, k))
+            cs = (g.standard_normal((rows, c)) * 4).astype(np.float32) if self.acc else None
+            self.prepared.append((x[:rows].copy(), qb, beta, c, k, cs))
         self.desc = (f"{rows} rows of A x first {cols} columns of D per (N,K) pair, "
-                     f"full K")
+                     f"full K" + (", D = C + A B^T" if self.acc else ""))
 
     def run(self) -> tuple[float, float]:
         """Returns (seconds, FLOPs) of one pass."""
         from oracle import gemm as og, quant as oq
         t0 = time.perf_counter()
         flops = 0.0
-        for xs, qb, beta, c, k in self.prepared:
+        for xs, qb, beta, c, k, cs in self.prepared:
             qa, alpha = oq.quantize_1x128(xs)
-            og.fp8_gemm_nt(qa, alpha, qb, beta)
+            if cs is None:
+                og.fp8_gemm_nt(qa, alpha, qb, beta)
+            else:
+                og.fp8_gemm_nt_accumulate(qa, alpha, qb, beta, cs)
             flops += 2.0 * xs.shape[0] * c * k
         return time.perf_counter() - t0, flops
 
@@ -698,7 +728,8 @@ def main():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="prefill",
-                    choices=["prefill", "decode64", "decode128", "contiguous", "masked"])
+                    choices=["prefill", "prefill_acc", "decode64", "decode128", "contiguous",
+                             "masked"])
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--ref-rows", type=int, default=16,
                     help="rows of A per shape in the oracle's timed sample")

@@ -196,6 +196,24 @@ int dg_fp8_gemm_nt_noalloc(const uint8_t *A, const float *sfa, int64_t ld_sfa,
                            int64_t N, int64_t K, dg_stream_t stream);
 
 /*
+ * dg_fp8_gemm_nt_accumulate -- D = C + A * B^T (Deep dive, section 3: the NT
+ * GEMM's accumulating form): the block-scaled product of dg_fp8_gemm_nt plus
+ * an FP32 matrix C, added to the FP32 accumulator before the single rounding
+ * of D to BF16.
+ *
+ * Same arguments, layouts, workspace use and errors as dg_fp8_gemm_nt, plus
+ *   C      device float [M][N] row-major, 16-byte aligned, read only; must
+ *          not overlap D.  NULL is DG_ERR_INVALID_ARG (unless M == 0).
+ * Decode-sized splits of K go through the workspace (not through clusters);
+ * the 2-CTA pair form is not used.  Deterministic.
+ */
+int dg_fp8_gemm_nt_accumulate(const uint8_t *A, const float *sfa,
+                              int64_t ld_sfa, const uint8_t *B,
+                              const float *sfb, const float *C, void *D,
+                              int64_t M, int64_t N, int64_t K, void *workspace,
+                              size_t workspace_bytes, dg_stream_t stream);
+
+/*
  * dg_m_grouped_fp8_gemm_nt_contiguous -- MoE m-grouped GEMM, contiguous
  * layout (Lesson 13, Fig. 13-3 "contiguous"; Deep dive, section 3).
  *

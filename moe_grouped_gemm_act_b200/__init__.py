@@ -11,6 +11,8 @@ Entry points (same names as the C ABI):
 * ``dg_quantize_1x128(x, pow2=False)`` -> (q, sf)    1 x 128 E4M3 activations
 * ``dg_quantize_128x128(w, pow2=False)`` -> (q, sf)  128 x 128 E4M3 weights
 * ``dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace=None)``
+* ``dg_fp8_gemm_nt_accumulate(a, sfa, b, sfb, c, d, workspace=None)``  D = C + A B^T
+* ``dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, d)``
 * ``dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices)``
 * ``dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m)``
 * ``dg_get_device_status()``, helpers ``dg_get_tma_aligned_size``,
@@ -35,13 +37,15 @@ LIB_PATH = os.path.join(_HERE, "libdg.so")
 DG_OK = 0
 DG_DTYPE_F32, DG_DTYPE_BF16 = 0, 1
 DG_SCALE_FP32, DG_SCALE_POW2 = 0, 1
+DG_ERR_INVALID_ARG, DG_ERR_ALIGNMENT, DG_ERR_UNSUPPORTED_ARCH = -1, -2, -3
+DG_ERR_CUDA, DG_ERR_WORKSPACE = -4, -5
 DG_ERR_TIMEOUT, DG_ERR_DEVICE_DATA = -6, -7
 
 EXPORTS = [
     "dg_status_string", "dg_get_mk_alignment_for_contiguous_layout",
     "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms",
     "dg_quantize_1x128", "dg_quantize_128x128", "dg_fp8_gemm_nt",
-    "dg_fp8_gemm_nt_workspace_size", "dg_fp8_gemm_nt_noalloc",
+    "dg_fp8_gemm_nt_workspace_size", "dg_fp8_gemm_nt_noalloc", "dg_fp8_gemm_nt_accumulate",
     "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_get_device_status",
 ]
@@ -76,6 +80,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_fp8_gemm_nt": (I, [P, P, I64, P, P, P, I64, I64, I64, P, SZ, P]),
         "dg_fp8_gemm_nt_workspace_size": (SZ, [I64, I64, I64]),
         "dg_fp8_gemm_nt_noalloc": (I, [P, P, I64, P, P, P, I64, I64, I64, P]),
+        "dg_fp8_gemm_nt_accumulate": (I, [P, P, I64, P, P, P, P, I64, I64, I64, P, SZ, P]),
         "dg_m_grouped_fp8_gemm_nt_contiguous":
             (I, [P, P, I64, P, P, P, P, I64, I64, I64, I, P]),
         "dg_m_grouped_fp8_gemm_nt_masked":
@@ -210,6 +215,21 @@ def dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace: torch.Tensor | None = None,
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d), m, n, k,
         _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "dg_fp8_gemm_nt")
+    return d
+
+
+def dg_fp8_gemm_nt_accumulate(a, sfa, b, sfb, c, d, workspace: torch.Tensor | None = None,
+                              stream=None) -> torch.Tensor:
+    """D = C + A * B^T: as dg_fp8_gemm_nt, with c a float32 [M, N] tensor added
+    before the BF16 rounding of d; d is returned."""
+    _need_cuda(a, sfa, b, sfb, c, d)
+    m, k = a.shape
+    n = b.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load_library().dg_fp8_gemm_nt_accumulate(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(c), _ptr(d), m, n, k,
+        _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dg_fp8_gemm_nt_accumulate")
     return d
 
 

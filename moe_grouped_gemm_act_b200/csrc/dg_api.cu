@@ -191,6 +191,34 @@ int dg_fp8_gemm_nt(const uint8_t *A, const float *sfa, int64_t ld_sfa, const uin
                          effective_num_sms(), workspace_bytes, workspace);
 }
 
+int dg_fp8_gemm_nt_accumulate(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                              const uint8_t *B, const float *sfb, const float *C, void *D,
+                              int64_t M, int64_t N, int64_t K, void *workspace,
+                              size_t workspace_bytes, dg_stream_t stream) {
+  int rc = check_gemm_common(A, sfa, ld_sfa, B, sfb, D, M, N, K);
+  if (rc) return rc;
+  if (M > 0 && !C) return DG_ERR_INVALID_ARG;
+  if (C && !aligned16(C)) return DG_ERR_ALIGNMENT;
+  if (workspace && !aligned16(workspace)) return DG_ERR_ALIGNMENT;
+  if (!workspace) workspace_bytes = 0;
+  rc = check_device();
+  if (rc) return rc;
+  if (M == 0) return DG_OK;
+  GemmParams p{};
+  p.status = device_info()->status;
+  p.sfa = sfa;
+  p.ld_sfa = ld_sfa;
+  p.sfb = sfb;
+  p.d = static_cast<uint16_t *>(D);
+  p.c = C;
+  p.rows = static_cast<int>(M);
+  p.n = static_cast<int>(N);
+  p.k = static_cast<int>(K);
+  p.groups = 1;
+  return launch_fp8_gemm(kDense, A, B, p, reinterpret_cast<cudaStream_t>(stream),
+                         effective_num_sms(), workspace_bytes, workspace);
+}
+
 int dg_m_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sfa, int64_t ld_sfa,
                                         const uint8_t *B, const float *sfb, void *D,
                                         const int32_t *m_indices, int64_t M_total,

@@ -73,22 +73,27 @@ constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 constexpr int kClusterNoFit = 1;        // launch_instance: clusters do not fit one wave
 
-// Schedules whose epilogue stages the BF16 tile in shared memory.
-__host__ __device__ constexpr bool staged_epilogue(int sched) {
-  return sched == kDense || sched == kMasked;
+// How a schedule's epilogue stages the output tile in shared memory: 0 not
+// at all, 1 the BF16 tile, 2 the FP32 tile (D = C + A B^T adds C as it
+// leaves).
+__host__ __device__ constexpr int staged_epilogue(int sched) {
+  return sched == kDenseAcc ? 2 : (sched == kDense || sched == kMasked) ? 1 : 0;
 }
 
-template <int BN, int STAGES, int NBUF, bool PAIR, bool STAGED>
+template <int BN, int STAGES, int NBUF, bool PAIR, int STAGED>
 struct Layout {
   // the pair form keeps half of the B tile (BN/2 rows) in each CTA
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  // With STAGED, BF16 staging of the output for coalesced stores: 128 rows
-  // x kOutCols (a 256-wide tile goes out in two column halves), then one
-  // byte per row saying whether it is stored
-  static constexpr uint32_t kOutCols = BN < 128 ? BN : 128;
+  // With STAGED, staging of the output for coalesced stores: 128 rows x
+  // kOutCols BF16 (kind 1: a 256-wide tile goes out in two column halves) or
+  // FP32 (kind 2: 64-column phases), then one byte per row saying whether it
+  // is stored
+  static constexpr uint32_t kOutCols =
+      STAGED == 2 ? (BN < 64 ? BN : 64) : (BN < 128 ? BN : 128);
+  static constexpr uint32_t kOutElem = STAGED == 2 ? 4 : 2;
   static constexpr uint32_t kOutOff = STAGES * kStageBytes;
-  static constexpr uint32_t kRowOkOff = kOutOff + (STAGED ? BM * kOutCols * 2 : 0);
+  static constexpr uint32_t kRowOkOff = kOutOff + (STAGED ? BM * kOutCols * kOutElem : 0);
   static constexpr uint32_t kBarOff = kRowOkOff + (STAGED ? BM : 0);
   // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain epi
   static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
@@ -215,7 +220,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // dense and masked tiles leave through shared memory (coalesced row
   // stores); contiguous tiles store each thread's row segment directly
   // (measured 1 % faster for them)
-  constexpr bool kStaged = staged_epilogue(SCHED);
+  constexpr int kStaged = staged_epilogue(SCHED);
+  constexpr bool kDenseLike = SCHED == kDense || SCHED == kDenseAcc;
   using L = Layout<BN, STAGES, NBUF, PAIR, kStaged>;
   constexpr int TM = PAIR ? 2 * BM : BM;   // rows per tile
   static_assert(!PAIR || SCHED == kDense, "the pair form serves dense GEMMs");
@@ -521,7 +527,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       // ---------------------------------------------------------- epilogue
       // (split K serves dense shapes only; the grouped instances leave it
       // out, which also keeps their register allocation lean)
-      if (SCHED == kDense && t.nsplit > 1) {
+      if (kDenseLike && t.nsplit > 1) {
         if (*s_abort) break;
         // Split K: every CTA of the tile writes its FP32 partial (valid rows
         // only, as float4 slots [column / 4][row] so that a warp's 32 rows
@@ -593,6 +599,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             const int c4 = f / valid, r = f - c4 * valid;
             const int col = t.n_blk * BN + 4 * c4;
             if (ok[q] && col < p.n) {
+              if constexpr (SCHED == kDenseAcc) {
+                const float4 cv = __ldg(reinterpret_cast<const float4 *>(
+                    p.c + static_cast<int64_t>(row0 + r) * p.n + col));
+                sum[q].x += cv.x;
+                sum[q].y += cv.y;
+                sum[q].z += cv.z;
+                sum[q].w += cv.w;
+              }
               const __nv_bfloat162 lo = __floats2bfloat162_rn(sum[q].x, sum[q].y);
               const __nv_bfloat162 hi = __floats2bfloat162_rn(sum[q].z, sum[q].w);
               uint2 v;
@@ -638,6 +652,61 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
               }
               *reinterpret_cast<uint4 *>(drow + col0 + c) = v;
             }
+          }
+        }
+      } else if constexpr (kStaged == 2) {
+        // D = C + A B^T: the FP32 tile goes through shared memory in 64-column
+        // phases ([128 rows][kOutCols] FP32, 16-byte chunk c of row r at
+        // c ^ (r mod kSw)); on the way out each lane adds the matching 16
+        // bytes of C (consecutive lanes read consecutive columns of a row),
+        // rounds the sum to BF16 and stores 8 bytes.
+        constexpr int kChunks = L::kOutCols / 4;        // 16-byte chunks per staged row
+        constexpr int kSw = kChunks < 8 ? kChunks : 8;
+        constexpr int kPhases = BN / L::kOutCols;
+        constexpr int kRowBytes = L::kOutCols * 4;
+        const uint32_t s_out = base + L::kOutOff;
+        uint8_t *s_rowok = smem + L::kRowOkOff;
+        const int ptid = threadIdx.x - kControlWarps * 32;
+        const int64_t row0 = static_cast<int64_t>(t.m_blk) * TM;
+        if (half == 0) s_rowok[row_in_tile] = row_ok ? 1 : 0;
+#pragma unroll
+        for (int ph = 0; ph < kPhases; ++ph) {
+#pragma unroll
+          for (int c = 0; c < W; c += 4) {
+            const int tcol = half * W + c;  // tile column of acc[c]
+            if (tcol / L::kOutCols == ph) {
+              const int chunk = (tcol % L::kOutCols) / 4;
+              st_shared_v4(s_out + row_in_tile * kRowBytes + ((chunk ^ (row_in_tile % kSw)) * 16),
+                           __float_as_uint(acc[c]), __float_as_uint(acc[c + 1]),
+                           __float_as_uint(acc[c + 2]), __float_as_uint(acc[c + 3]));
+            }
+          }
+          if (!epi_sync()) {
+            alive = false;
+            break;
+          }
+          const int col_base = t.n_blk * BN + ph * L::kOutCols;
+#pragma unroll 1
+          for (int f = ptid; f < BM * kChunks; f += kPromoThreads) {
+            const int r = f / kChunks, ch = f - r * kChunks;
+            const int col = col_base + ch * 4;
+            if (s_rowok[r] && col < p.n) {
+              const uint4 a = ld_shared_v4(s_out + r * kRowBytes + ((ch ^ (r % kSw)) * 16));
+              const int64_t off = (row0 + r) * p.n + col;
+              const float4 cv = __ldg(reinterpret_cast<const float4 *>(p.c + off));
+              const __nv_bfloat162 lo =
+                  __floats2bfloat162_rn(__uint_as_float(a.x) + cv.x, __uint_as_float(a.y) + cv.y);
+              const __nv_bfloat162 hi =
+                  __floats2bfloat162_rn(__uint_as_float(a.z) + cv.z, __uint_as_float(a.w) + cv.w);
+              uint2 v;
+              v.x = *reinterpret_cast<const uint32_t *>(&lo);
+              v.y = *reinterpret_cast<const uint32_t *>(&hi);
+              *reinterpret_cast<uint2 *>(p.d + off) = v;
+            }
+          }
+          if (!epi_sync()) {
+            alive = false;
+            break;
           }
         }
       } else {
@@ -769,7 +838,7 @@ constexpr Candidate kCandidates[] = {
 // The pair form: 256 x 256 tiles, half of B per CTA (32 KB stages).
 constexpr Candidate kPairCandidate = {256, 6, 2};
 
-template <int BN, int STAGES, int NBUF, bool PAIR, bool STAGED>
+template <int BN, int STAGES, int NBUF, bool PAIR, int STAGED>
 constexpr int smem_bytes_for(int extra) {
   return 1024 + Layout<BN, STAGES, NBUF, PAIR, STAGED>::kPrefixOff + extra;
 }
@@ -1055,6 +1124,10 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   bool pair = choice.pair;
   int64_t full_tiles = choice.full_tiles;
   bool splits_forced = false;  // DG_SPLITS: exactly this many, or none
+  // D = C + A B^T (dense only): single-CTA tiles, splits through the
+  // workspace (the FP32 tile is staged in the 32 KB the BF16 tile uses, so
+  // every tile form still fits)
+  const bool acc = p.c != nullptr;
   // Tuning / test overrides: DG_PAIR=0/1 disables / forces the pair form
   // (dense only), DG_BLOCK_N forces the N tile of the single-CTA form,
   // DG_SPLITS splits every tile's K, DG_TAIL_SPLITS only the last partial
@@ -1065,7 +1138,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
         pair = false;
         bn = 256;
       }
-    } else if (*e == '1' && sched == kDense && num_sms >= 2) {
+    } else if (*e == '1' && sched == kDense && !acc && num_sms >= 2) {
       pair = true;
       bn = kPairCandidate.bn;
       splits = 1;
@@ -1122,7 +1195,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   // form a cluster and reduce through distributed shared memory, needing no
   // workspace or arrival counters, when all clusters fit in one wave
   // (DG_CLUSTER_SPLIT=0 forces the workspace path).
-  bool try_cluster = sched == kDense && !pair && splits > 1 && splits <= 8 &&
+  bool try_cluster = sched == kDense && !acc && !pair && splits > 1 && splits <= 8 &&
                      p.full_tiles == 0 && all_tiles * splits <= num_sms;
   if (const char *e = getenv("DG_CLUSTER_SPLIT"))
     if (*e == '0') try_cluster = false;
@@ -1202,7 +1275,9 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
             p.full_tiles, grid, static_cast<long long>(units));
   }
   switch (sched) {
-    case kDense: return dispatch<kDense>(bn, pair, ta, tb, p, grid, extra, stream);
+    case kDense:
+      return acc ? dispatch<kDenseAcc>(bn, false, ta, tb, p, grid, extra, stream)
+                 : dispatch<kDense>(bn, pair, ta, tb, p, grid, extra, stream);
     case kContiguous: return dispatch<kContiguous>(bn, false, ta, tb, p, grid, extra, stream);
     case kMasked: return dispatch<kMasked>(bn, false, ta, tb, p, grid, extra, stream);
     default: return DG_ERR_INVALID_ARG;

@@ -33,7 +33,9 @@ inline cudaLaunchAttribute pdl_attribute() {
 // kDenseCluster: dense tiles every one split `splits` ways along K, the splits
 // of a tile forming one thread-block cluster that reduces through
 // distributed shared memory (decode-sized shapes; no workspace).
-enum Sched : int { kDense = 0, kContiguous = 1, kMasked = 2, kDenseCluster = 3 };
+// kDenseAcc: dense tiles with D = C + A B^T (an FP32 C added before the BF16
+// rounding); the host picks it for a dense launch that has a C.
+enum Sched : int { kDense = 0, kContiguous = 1, kMasked = 2, kDenseCluster = 3, kDenseAcc = 4 };
 
 // Kernel parameters besides the two tensor maps.  Row coordinates are inside
 // one "slab": the whole of A for dense and contiguous, one expert's M_max rows
@@ -43,6 +45,7 @@ struct GemmParams {
   int64_t ld_sfa;
   const float *sfb;      // beta: [group][ceil(N/128)][K/128]
   uint16_t *d;           // BF16 output [slab][rows][N]
+  const float *c;        // dense D = C + A B^T: FP32 C [rows][N] (nullptr: none)
   const int32_t *m_indices;  // contiguous: expert per row (-1 = padding)
   const int32_t *masked_m;   // masked: valid rows per expert
   int *status;           // device status word (first error wins)

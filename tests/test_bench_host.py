@@ -36,7 +36,8 @@ def test_grouped_oracle_sample_takes_experts_with_rows():
 
 
 def test_workload_specs_name_their_bound():
-    for name, bound in [("prefill", "tensor"), ("decode64", "hbm"), ("decode128", "hbm"),
+    for name, bound in [("prefill", "tensor"), ("prefill_acc", "tensor"), ("decode64", "hbm"),
+                        ("decode128", "hbm"),
                         ("contiguous", "tensor"), ("masked", "hbm")]:
         assert bench.workload_spec(name)["bound"] == bound
     with pytest.raises(SystemExit):

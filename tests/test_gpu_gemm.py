@@ -227,6 +227,89 @@ def test_dense_decode_full_size(m, n, k):
     check_gemm(bits_of(d), gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"decode {m}x{n}x{k}")
 
 
+# ------------------------------------------------------------ D = C + A B^T
+def run_dense_acc(qa, alpha, qb, beta, c, workspace=False):
+    m, n = qa.shape[0], qb.shape[0]
+    d = torch.full((m, n), 0, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    ws = None
+    if workspace:
+        nbytes = max(dg.dg_fp8_gemm_nt_workspace_size(m, n, qa.shape[1]),
+                     -(-m // 128) * (n + 256) * 8 * 128 * 4 + (1 << 16))
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    dg.dg_fp8_gemm_nt_accumulate(dev(qa), sfa_to_device(alpha), dev(qb), dev(beta),
+                                 torch.from_numpy(c).cuda(), d, workspace=ws)
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    return bits_of(d)
+
+
+def acc_c(m, n, seed):
+    return (np.random.default_rng(seed).standard_normal((m, n)) * 4).astype(np.float32)
+
+
+@pytest.mark.parametrize("bn", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("m,n,k", [(300, 520, 1024), (1, 136, 256), (129, 2112, 384)])
+def test_dense_accumulate_ragged_every_block_n(bn, m, n, k):
+    qa, alpha, qb, beta = dense_case(m, n, k, seed=3 * m + n + k)
+    c = acc_c(m, n, seed=m + n)
+    with env(DG_BLOCK_N=bn):
+        got = run_dense_acc(qa, alpha, qb, beta, c)
+    want = gemm.fp8_gemm_nt_accumulate_f64(qa, alpha, qb, beta, c)
+    check_gemm(got, want, f"C + AB^T {m}x{n}x{k} BN={bn}")
+
+
+@pytest.mark.parametrize("mode", ["split", "tail"])
+def test_dense_accumulate_split_paths(mode):
+    # C is added once, by the split that stores the reduced tile
+    if mode == "split":
+        m, n, k, knobs = 64, 528, 2048, dict(DG_BLOCK_N=128, DG_SPLITS=4)
+    else:
+        m, n, k, knobs = 1000, 1032, 1024, dict(DG_BLOCK_N=256, DG_TAIL_SPLITS=3)
+    qa, alpha, qb, beta = dense_case(m, n, k, seed=77)
+    c = acc_c(m, n, seed=78)
+    if mode == "tail":
+        dg.dg_set_num_sms(12)
+    try:
+        with env(**knobs):
+            a = run_dense_acc(qa, alpha, qb, beta, c, workspace=True)
+            b = run_dense_acc(qa, alpha, qb, beta, c, workspace=True)
+    finally:
+        dg.dg_set_num_sms(0)
+    check_gemm(a, gemm.fp8_gemm_nt_accumulate_f64(qa, alpha, qb, beta, c), f"C + AB^T {mode}")
+    assert np.array_equal(a, b), "not deterministic"
+
+
+def test_dense_accumulate_integers_bit_exact():
+    # integer codes in [-4, 4], unit scales, integer C: D = BF16(exact)
+    g = np.random.default_rng(5)
+    m, n, k = 256, 384, 2048
+    a = g.integers(-4, 5, size=(m, k)).astype(np.float32)
+    b = g.integers(-4, 5, size=(n, k)).astype(np.float32)
+    c = g.integers(-300, 301, size=(m, n)).astype(np.float32)
+    got = run_dense_acc(e4m3.encode_rne(a), np.ones((m, k // 128), np.float32),
+                        e4m3.encode_rne(b), np.ones((3, k // 128), np.float32), c)
+    exact = a.astype(np.int64) @ b.astype(np.int64).T + c.astype(np.int64)
+    assert np.array_equal(got, bf16.to_bits(exact.astype(np.float64)))
+
+
+def test_dense_accumulate_zero_c_matches_plain_gemm():
+    qa, alpha, qb, beta = dense_case(384, 1024, 1536, seed=9)
+    plain = run_dense(qa, alpha, qb, beta)
+    acc = run_dense_acc(qa, alpha, qb, beta, np.zeros((384, 1024), np.float32))
+    assert np.array_equal(plain, acc)
+
+
+def test_dense_accumulate_requires_c():
+    qa, alpha, qb, beta = dense_case(128, 128, 128, seed=1)
+    lib = dg.load_library()
+    d = torch.empty((128, 128), dtype=torch.bfloat16, device="cuda")
+    a_d, s_d, b_d, t_d = dev(qa), sfa_to_device(alpha), dev(qb), dev(beta)
+    rc = lib.dg_fp8_gemm_nt_accumulate(a_d.data_ptr(), s_d.data_ptr(), s_d.shape[-1],
+                                       b_d.data_ptr(), t_d.data_ptr(), None, d.data_ptr(),
+                                       128, 128, 128, None, 0, None)
+    assert rc == dg.DG_ERR_INVALID_ARG
+
+
 def test_dense_m_zero_is_noop():
     d = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
     a = torch.empty((0, 128), dtype=torch.uint8, device="cuda")
