@@ -686,7 +686,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             break;
           }
           const int col_base = t.n_blk * BN + ph * L::kOutCols;
-#pragma unroll 1
+          // unrolled so that the read-only loads of C of several iterations
+          // are in flight together
+#pragma unroll 4
           for (int f = ptid; f < BM * kChunks; f += kPromoThreads) {
             const int r = f / kChunks, ch = f - r * kChunks;
             const int col = col_base + ch * 4;
