@@ -60,13 +60,13 @@ FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 # SHA-256 of csrc/gemm.cu + csrc/ptx.cuh + csrc/internal.h; on a mismatch the
 # bench reports null.
 GEMM_TRAFFIC = {
-    "source": "7980b2dd003a5dd7",
-    "prefill": 210.4e6,
-    "prefill_acc": 388.0e6,
+    "source": "3444ff888e1a7ea1",
+    "prefill": 211.2e6,
+    "prefill_acc": 405.3e6,
     "decode64": 51.3e6,
-    "decode128": 51.8e6,
-    "masked": 533.7e6,
-    "contiguous": 948.9e6,
+    "decode128": 52.0e6,
+    "masked": 533.6e6,
+    "contiguous": 978.3e6,
 }
 
 

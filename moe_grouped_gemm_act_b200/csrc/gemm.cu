@@ -70,6 +70,7 @@ constexpr int kPromoWarps = 8;          // two column halves x four lane quarter
 constexpr int kPromoThreads = 32 * kPromoWarps;
 constexpr int kThreads = 32 * (kControlWarps + kPromoWarps);
 constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
+constexpr int kCAhead = 8;              // K blocks between the C prefetch and the tile's end
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 constexpr int kClusterNoFit = 1;        // launch_instance: clusters do not fit one wave
 
@@ -341,7 +342,22 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       }
       const int a_row = t.m_blk * TM + static_cast<int>(rank) * BM;
       const int b_row = t.n_blk * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
+      // D = C + A B^T: the epilogue's C rows are asked into L2 kCAhead K
+      // blocks before the tile's last one -- late enough that the operand
+      // stream of a long K does not evict them first, early enough to cover
+      // the DRAM latency the epilogue would otherwise wait on
+      const int c_kb = (SCHED == kDenseAcc && t.split == 0) ? max(t.k_begin, t.k_end - kCAhead)
+                                                            : -1;
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
+        if constexpr (SCHED == kDenseAcc) {
+          if (kb == c_kb) {
+            const int col0 = t.n_blk * BN;
+            const uint32_t bytes = static_cast<uint32_t>(min(BN, p.n - col0)) * 4u;
+            const int valid = min(BM, p.rows - a_row);
+            for (int r = lane; r < valid; r += 32)
+              prefetch_l2_bulk(p.c + static_cast<int64_t>(a_row + r) * p.n + col0, bytes);
+          }
+        }
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!mbar_wait(empty_bar(s), ph ^ 1, s_abort, p.status)) { alive = false; break; }

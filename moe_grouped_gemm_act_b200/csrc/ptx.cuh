@@ -163,6 +163,13 @@ __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Asks for `bytes` of global memory at `src` to be brought into L2 (no
+// destination, no completion to wait for).  src 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------------------ shared
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b,
                                              uint32_t c, uint32_t d) {
