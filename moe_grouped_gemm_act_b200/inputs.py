@@ -15,6 +15,9 @@ public dataset stands in for):
   each expert segment padded up to a multiple of 128 rows, a per-row int32
   expert index with -1 on padding rows;
 * masked MoE layout: masked_m[g] ~ Uniform{0, ..., M_max}.
+* k-grouped MoE layout (weight gradient): token counts ~ Multinomial(T,
+  uniform over G experts) along K, each segment padded up to a multiple of
+  128 tokens.
 
 All generators are numpy PCG64 streams with explicit seeds.
 """
@@ -71,6 +74,26 @@ def contiguous_layout(num_tokens: int, num_groups: int, seed: int,
         row += p
     return ContiguousLayout(counts=np.asarray(counts), m_indices=m_indices,
                             m_total=m_total)
+
+
+@dataclass
+class KGroupedLayout:
+    counts: np.ndarray      # int64 [G]: tokens per expert
+    k_sizes: np.ndarray     # int32 [G]: K segment per expert, counts padded to 128
+    k_total: int
+
+
+def k_grouped_layout(num_tokens: int, num_groups: int, seed: int,
+                     align: int = ALIGN_M) -> KGroupedLayout:
+    """Multinomial split of ``num_tokens`` over ``num_groups`` experts along
+    the K axis, each segment padded up to a multiple of ``align`` tokens (an
+    expert with no tokens gets an empty segment).  The padding tokens are
+    for the caller to fill with zeros."""
+    g = rng(seed)
+    counts = g.multinomial(num_tokens, np.full(num_groups, 1.0 / num_groups))
+    k_sizes = np.array([(-(-int(c) // align)) * align for c in counts], dtype=np.int32)
+    return KGroupedLayout(counts=np.asarray(counts), k_sizes=k_sizes,
+                          k_total=int(k_sizes.sum()))
 
 
 def masked_counts(num_groups: int, m_max: int, seed: int) -> np.ndarray:

@@ -26,7 +26,8 @@ Modules
 ``bf16``   round-to-nearest-even of float64 values to bfloat16.
 ``quant``  1x128 activation and 128x128 weight quantization (FP32 or
            power-of-two scales).
-``gemm``   the block-scaled NT GEMM, its m-grouped contiguous and masked forms.
+``gemm``   the block-scaled NT GEMM, its accumulating form, its m-grouped
+           contiguous and masked forms and the k-grouped contiguous form.
 
 Every function is pinned by ``tests/test_oracle_*.py`` against something other
 than itself (closed forms, brute force, library conversions, the page's worked

@@ -24,6 +24,9 @@ section 3, the grouped GEMM table):
   the expert, -1 on padding rows; N and K are shared by all experts.
 * m-grouped masked: A is [G, M_max, K]; masked_m[g] rows of expert g are
   valid; only those rows are computed.
+* k-grouped contiguous (the MoE weight gradient): the groups split the K
+  axis (tokens) instead of M; M and N are shared by all groups and every
+  group has its own [M, N] output.
 
 Rows that are not computed (padding, rows >= masked_m[g]) are left exactly as
 they were in the output (the pages do not say; this is the reading taken);
@@ -140,3 +143,53 @@ def m_grouped_masked(qa, alpha, qb, beta, masked_m, d_init_bits):
         if m:
             out[e, :m] = fp8_gemm_nt(qa[e, :m], alpha[e, :m], qb[e], beta[e])
     return out
+
+
+def k_grouped_contiguous_f64(qa, alpha, qb, beta, k_sizes, c=None):
+    """K-grouped contiguous GEMM in float64: for every group g,
+    D[g] = C[g] + A_g B_g^T, where A_g and B_g are group g's segment of the
+    shared K axis (Deep dive, section 3, the grouped GEMM table: the group
+    axis is K, M and N are fixed, used for the MoE weight gradient; NT form).
+
+    qa uint8 [M, K_total], alpha float32 [M, K_total/128]; qb uint8
+    [N, K_total], beta float32 [N, K_total/128]: both operands are
+    token-indexed activations here, so both carry the 1x128 scaling of
+    Fig. 13-1's A (one scale per row per 128 K elements).  k_sizes int [G]:
+    group g owns the K segment starting at sum(k_sizes[:g]); every size is a
+    multiple of 128, so a scale group never spans two experts (zero is
+    allowed: that group's D is its C).  c float [G, M, N] or None (zeros).
+
+    Within a segment the Fig. 13-1 order is kept: per 128-wide K block, the
+    block's partial product of the decoded codes, times the outer product of
+    the block's row scales of A and of B, added in float64.
+    """
+    M, K = qa.shape
+    N, Kb = qb.shape
+    k_sizes = np.asarray(k_sizes, dtype=np.int64)
+    if K != Kb or K % GROUP:
+        raise ValueError("K mismatch or K not a multiple of 128")
+    if np.any(k_sizes < 0) or np.any(k_sizes % GROUP) or int(k_sizes.sum()) != K:
+        raise ValueError("group sizes must be multiples of 128 that sum to K")
+    kg = K // GROUP
+    if alpha.shape != (M, kg) or beta.shape != (N, kg):
+        raise ValueError("scale shapes do not match the 1x128 grids of A and B")
+    G = len(k_sizes)
+    d = np.zeros((G, M, N), dtype=np.float64)
+    if c is not None:
+        c64 = np.asarray(c, np.float64)
+        if c64.shape != d.shape:
+            raise ValueError("C must be [G, M, N]")
+        d += c64
+    a_vals = e4m3.decode(qa)
+    b_vals = e4m3.decode(qb)
+    alpha64 = np.asarray(alpha, np.float64)
+    beta64 = np.asarray(beta, np.float64)
+    first_block = 0
+    for g in range(G):
+        blocks = int(k_sizes[g]) // GROUP
+        for b in range(first_block, first_block + blocks):
+            ks = slice(b * GROUP, (b + 1) * GROUP)
+            partial = a_vals[:, ks] @ b_vals[:, ks].T
+            d[g] += partial * (alpha64[:, b][:, None] * beta64[:, b][None, :])
+        first_block += blocks
+    return d
