@@ -28,10 +28,12 @@ Modules
            power-of-two scales).
 ``gemm``   the block-scaled NT GEMM, its accumulating form, its m-grouped
            contiguous and masked forms and the k-grouped contiguous form.
+``ue8m0``  UE8M0 (power-of-two) scale codes and the packed 4-per-int32,
+           MN-major scale layout.
 
 Every function is pinned by ``tests/test_oracle_*.py`` against something other
 than itself (closed forms, brute force, library conversions, the page's worked
 exercise).  No function here is "parity unpinned".
 """
 
-from . import bf16, e4m3, gemm, quant  # noqa: F401
+from . import bf16, e4m3, gemm, quant, ue8m0  # noqa: F401
