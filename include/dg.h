@@ -132,6 +132,32 @@ int dg_quantize_128x128(const float *w, int64_t G, int64_t N, int64_t K,
                         uint8_t *q, float *sf, int flags, dg_stream_t stream);
 
 /*
+ * dg_pack_ue8m0 -- the packed UE8M0 scale layout ("DeepGEMM architecture deep
+ * dive", section 3: on sm_100 the LHS scales are four UE8M0 values per 32-bit
+ * integer, transposed and TMA-aligned; UE8M0 itself: Lesson 13, Fig. 13-1
+ * text).  UE8M0 code e stands for 2^(e - 127); for a power-of-two FP32 scale
+ * it is the FP32 exponent field, and +0 is coded 0.
+ *
+ *   sf      device float [batch][Kg][ld_sf], MN-major: the scale of row i,
+ *           K group g at sf[(b * Kg + g) * ld_sf + i] -- the layout
+ *           dg_quantize_1x128 writes; with DG_SCALE_POW2 every scale is +0
+ *           or a normal power of two.
+ *   packed  device int32 [batch][ceil(Kg/4)][ld_packed], MN-major: word
+ *           (b, p, i) holds groups 4p .. 4p+3 of row i, group 4p+t in bits
+ *           8t .. 8t+7; groups past Kg are zero bytes.  Entries i >= M are
+ *           not written.
+ *   batch >= 1, M >= 0 (M == 0 is a no-op), Kg >= 1; ld_sf >= M and
+ *   ld_packed >= M, both multiples of 4; both pointers 16-byte aligned.
+ * A scale that is not +0 or a positive normal power of two (a signed value,
+ * a non-power of two, a subnormal, inf or NaN) is recorded in the device
+ * status word as DG_ERR_DEVICE_DATA (see dg_get_device_status); its byte is
+ * then its exponent field.  Output is bit-exact.  Memory is caller-owned.
+ */
+int dg_pack_ue8m0(const float *sf, int64_t batch, int64_t M, int64_t Kg,
+                  int64_t ld_sf, int32_t *packed, int64_t ld_packed,
+                  dg_stream_t stream);
+
+/*
  * dg_fp8_gemm_nt -- dense NT GEMM, D = A * B^T with 1x128 / 128x128 scales
  * (Lesson 13, Fig. 13-1; DeepGEMM launch article: gemm_fp8_fp8_bf16_nt).
  *

@@ -10,6 +10,7 @@ Entry points (same names as the C ABI):
 
 * ``dg_quantize_1x128(x, pow2=False)`` -> (q, sf)    1 x 128 E4M3 activations
 * ``dg_quantize_128x128(w, pow2=False)`` -> (q, sf)  128 x 128 E4M3 weights
+* ``dg_pack_ue8m0(sf, m)`` -> packed int32 UE8M0 scales (4 K groups per word)
 * ``dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace=None)``
 * ``dg_fp8_gemm_nt_accumulate(a, sfa, b, sfb, c, d, workspace=None)``  D = C + A B^T
 * ``dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, d)``
@@ -44,7 +45,7 @@ DG_ERR_TIMEOUT, DG_ERR_DEVICE_DATA = -6, -7
 EXPORTS = [
     "dg_status_string", "dg_get_mk_alignment_for_contiguous_layout",
     "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms",
-    "dg_quantize_1x128", "dg_quantize_128x128", "dg_fp8_gemm_nt",
+    "dg_quantize_1x128", "dg_quantize_128x128", "dg_pack_ue8m0", "dg_fp8_gemm_nt",
     "dg_fp8_gemm_nt_workspace_size", "dg_fp8_gemm_nt_noalloc", "dg_fp8_gemm_nt_accumulate",
     "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_get_device_status",
@@ -77,6 +78,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_get_num_sms": (I, []),
         "dg_quantize_1x128": (I, [P, I, I64, I64, I64, I64, P, I64, P, I64, I, P]),
         "dg_quantize_128x128": (I, [P, I64, I64, I64, P, P, I, P]),
+        "dg_pack_ue8m0": (I, [P, I64, I64, I64, I64, P, I64, P]),
         "dg_fp8_gemm_nt": (I, [P, P, I64, P, P, P, I64, I64, I64, P, SZ, P]),
         "dg_fp8_gemm_nt_workspace_size": (SZ, [I64, I64, I64]),
         "dg_fp8_gemm_nt_noalloc": (I, [P, P, I64, P, P, P, I64, I64, I64, P]),
@@ -200,6 +202,30 @@ def dg_quantize_128x128(w: torch.Tensor, pow2: bool = False, stream=None):
     if not grouped:
         return q[0], sf[0]
     return q, sf
+
+
+def dg_pack_ue8m0(sf: torch.Tensor, m: int, packed=None, stream=None) -> torch.Tensor:
+    """Packs power-of-two scales sf (float32 [Kg, ld] or [B, Kg, ld], the
+    MN-major layout dg_quantize_1x128 returns) of m rows into UE8M0 words:
+    int32 [ceil(Kg/4), ld'] (or [B, ceil(Kg/4), ld']), ld' =
+    dg_get_tma_aligned_size(m, 4); word (p, i) holds groups 4p .. 4p+3 of row
+    i, one byte each, lowest group in the lowest byte.  Scales that are not +0
+    or a normal power of two are reported through dg_get_device_status()."""
+    _need_cuda(sf)
+    if sf.dtype != torch.float32:
+        raise ValueError("sf must be float32")
+    batched = sf.dim() == 3
+    sb = sf if batched else sf.unsqueeze(0)
+    b, kg, ld = sb.shape
+    words = -(-kg // 4)
+    if packed is None:
+        packed = torch.empty((b, words, dg_get_tma_aligned_size(m, 4)), dtype=torch.int32,
+                             device=sf.device)
+    _need_cuda(packed)
+    rc = load_library().dg_pack_ue8m0(_ptr(sb), b, m, kg, ld, _ptr(packed), packed.shape[-1],
+                                      _stream(stream))
+    _check(rc, "dg_pack_ue8m0")
+    return packed if batched else packed.view(words, packed.shape[-1])
 
 
 # ------------------------------------------------------------------ GEMMs

@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libdg.so")
 
-SOURCES = ["dg_api.cu", "quantize.cu", "gemm.cu", "gemm_noalloc.cu"]
+SOURCES = ["dg_api.cu", "quantize.cu", "gemm.cu", "gemm_noalloc.cu", "ue8m0.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
