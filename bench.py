@@ -55,37 +55,68 @@ FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per GEMM launch,
 # averaged over the workload's launches, from ncu captures of this bench
-# (profiles/fp8_gemm_*.md give the commands).  Valid only for the GEMM
-# sources they were taken on: `source` is the first 16 hex digits of the
-# SHA-256 of csrc/gemm.cu + csrc/ptx.cuh + csrc/internal.h; on a mismatch the
-# bench reports null.
+# (profiles/fp8_gemm_*.md give the commands).  Each figure is valid only for
+# the GEMM code it was taken on (gemm_source_hash, stored beside it); on a
+# mismatch the bench reports null.
 GEMM_TRAFFIC = {
-    "source": "3444ff888e1a7ea1",
-    "prefill": 211.2e6,
-    "prefill_acc": 405.3e6,
-    "decode64": 51.3e6,
-    "decode128": 52.0e6,
-    "masked": 533.6e6,
-    "contiguous": 978.3e6,
+    "prefill": ("3e97d80689d725cc", 210.8e6),
+    "prefill_acc": ("05d65bb9d3528fd6", 405.3e6),
+    "decode64": ("05d65bb9d3528fd6", 51.3e6),
+    "decode128": ("05d65bb9d3528fd6", 52.0e6),
+    "masked": ("05d65bb9d3528fd6", 533.6e6),
+    "contiguous": ("05d65bb9d3528fd6", 978.3e6),
 }
 
 
-def gemm_source_hash() -> str:
+def strip_comments(src: str) -> str:
+    """C/C++ source without comments and with whitespace runs collapsed, so
+    that the traffic key follows the code, not its comments.  String and
+    character literals are kept verbatim."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        ch = src[i]
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif ch in "\"'":
+            j = i + 1
+            while j < n and src[j] != ch:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(ch)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def gemm_source_hash(texts=None) -> str:
+    """Key of the GEMM's code: SHA-256 (first 16 hex digits) of csrc/gemm.cu,
+    csrc/ptx.cuh and csrc/internal.h without comments."""
     import hashlib
     h = hashlib.sha256()
-    for f in ("gemm.cu", "ptx.cuh", "internal.h"):
-        with open(os.path.join(ROOT, "moe_grouped_gemm_act_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    if texts is None:
+        texts = []
+        for f in ("gemm.cu", "ptx.cuh", "internal.h"):
+            with open(os.path.join(ROOT, "moe_grouped_gemm_act_b200", "csrc", f)) as fh:
+                texts.append(fh.read())
+    for t in texts:
+        h.update(strip_comments(t).encode())
     return h.hexdigest()[:16]
 
 
 def measured_traffic(workload: str):
+    entry = GEMM_TRAFFIC.get(workload)
+    if entry is None:
+        return None
     try:
-        if gemm_source_hash() != GEMM_TRAFFIC["source"]:
-            return None
+        return entry[1] if gemm_source_hash() == entry[0] else None
     except OSError:
         return None
-    return GEMM_TRAFFIC.get(workload)
 
 
 # ---------------------------------------------------------------- workloads

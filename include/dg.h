@@ -293,6 +293,43 @@ int dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *A, const float *sfa,
                                     dg_stream_t stream);
 
 /*
+ * dg_k_grouped_fp8_gemm_nt_contiguous -- the K-grouped contiguous GEMM of
+ * the MoE weight gradient ("DeepGEMM architecture deep dive", section 3, the
+ * grouped GEMM table: the group axis is K, M and N are shared).  The K axis
+ * (tokens) is cut into G consecutive segments; for every group g,
+ *
+ *   D[g][i][j] = C[g][i][j] + sum over the 128-K blocks b of segment g of
+ *                alpha[i][b] * beta[j][b] * sum_{k < 128} A[i][128b+k] B[j][128b+k]
+ *
+ * in FP32: both operands carry 1x128 scales along K (Lesson 13, Fig. 13-1's
+ * activation scaling; here A and B are both token-indexed).
+ *
+ *   A        device E4M3 [M][K] row-major (K-major); B device E4M3 [N][K].
+ *   sfa      device float [K/128][ld_sfa], MN-major (dg_quantize_1x128 of A);
+ *            ld_sfa >= M, ld_sfa % 4 == 0.
+ *   sfb      device float [K/128][ld_sfb], MN-major (dg_quantize_1x128 of B);
+ *            ld_sfb >= N, ld_sfb % 4 == 0.
+ *   C        device float [G][M][N] added to the product, or NULL (zero).
+ *   D        device float [G][M][N], written whole (an empty group gets C,
+ *            or zeros).
+ *   k_sizes  device int32 [G]: K of each segment, each a multiple of 128,
+ *            summing to K (0 allowed).  Sizes off the 128 grid or not adding
+ *            up to K are recorded in the device status word as
+ *            DG_ERR_DEVICE_DATA; the kernel then clamps every segment into
+ *            [0, K) and reads nothing outside the operands.
+ *   1 <= G <= 1024, M >= 0 (M == 0 is a no-op), N > 0, N % 8 == 0,
+ *   K > 0, K % 128 == 0.  All pointers 16-byte aligned.
+ * Memory is caller-owned; nothing is allocated.  Results are deterministic.
+ */
+int dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sfa,
+                                        int64_t ld_sfa, const uint8_t *B,
+                                        const float *sfb, int64_t ld_sfb,
+                                        const float *C, float *D,
+                                        const int32_t *k_sizes, int G,
+                                        int64_t M, int64_t N, int64_t K,
+                                        dg_stream_t stream);
+
+/*
  * dg_get_device_status -- synchronizes `stream`, then reads and clears the
  * current device's status word.  *status receives DG_OK or the first device
  * error recorded since the last read (DG_ERR_TIMEOUT, DG_ERR_DEVICE_DATA).

@@ -16,6 +16,7 @@ Entry points (same names as the C ABI):
 * ``dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, d)``
 * ``dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices)``
 * ``dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m)``
+* ``dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, k_sizes, c=None)``
 * ``dg_get_device_status()``, helpers ``dg_get_tma_aligned_size``,
   ``dg_get_mk_alignment_for_contiguous_layout``, ``dg_set_num_sms``,
   ``dg_get_num_sms``, ``dg_fp8_gemm_nt_workspace_size``.
@@ -48,7 +49,8 @@ EXPORTS = [
     "dg_quantize_1x128", "dg_quantize_128x128", "dg_pack_ue8m0", "dg_fp8_gemm_nt",
     "dg_fp8_gemm_nt_workspace_size", "dg_fp8_gemm_nt_noalloc", "dg_fp8_gemm_nt_accumulate",
     "dg_m_grouped_fp8_gemm_nt_contiguous",
-    "dg_m_grouped_fp8_gemm_nt_masked", "dg_get_device_status",
+    "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_nt_contiguous",
+    "dg_get_device_status",
 ]
 
 _lib = None
@@ -87,6 +89,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             (I, [P, P, I64, P, P, P, P, I64, I64, I64, I, P]),
         "dg_m_grouped_fp8_gemm_nt_masked":
             (I, [P, P, I64, P, P, P, P, I, I64, I64, I64, P]),
+        "dg_k_grouped_fp8_gemm_nt_contiguous":
+            (I, [P, P, I64, P, P, I64, P, P, P, I, I64, I64, I64, P]),
         "dg_get_device_status": (I, [P, ctypes.POINTER(ctypes.c_int)]),
     }
     for name, (res, args) in sig.items():
@@ -300,4 +304,24 @@ def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m,
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d),
         _ptr(masked_m), g, m_max, n, k, _stream(stream))
     _check(rc, "dg_m_grouped_fp8_gemm_nt_masked")
+    return d
+
+
+def dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, k_sizes, c=None,
+                                        stream=None) -> torch.Tensor:
+    """K-grouped GEMM (MoE weight gradient): a [M, K] and b [N, K] uint8 with
+    1x128 scales sfa [K/128, ld_a] and sfb [K/128, ld_b] (both from
+    dg_quantize_1x128), k_sizes int32 [G] on the device (multiples of 128
+    summing to K), d float32 [G, M, N]; d[g] = c[g] + a_g b_g^T over group
+    g's K segment (c float32 [G, M, N] or None).  d is returned."""
+    _need_cuda(a, sfa, b, sfb, d, k_sizes)
+    if c is not None:
+        _need_cuda(c)
+    m, k = a.shape
+    n = b.shape[0]
+    g = k_sizes.numel()
+    rc = load_library().dg_k_grouped_fp8_gemm_nt_contiguous(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), sfb.shape[-1], _ptr(c),
+        _ptr(d), _ptr(k_sizes), g, m, n, k, _stream(stream))
+    _check(rc, "dg_k_grouped_fp8_gemm_nt_contiguous")
     return d

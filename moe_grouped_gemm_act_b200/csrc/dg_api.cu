@@ -270,6 +270,37 @@ int dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *A, const float *sfa, int64_t 
                          effective_num_sms(), 0, nullptr);
 }
 
+int dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                                        const uint8_t *B, const float *sfb, int64_t ld_sfb,
+                                        const float *C, float *D, const int32_t *k_sizes,
+                                        int G, int64_t M, int64_t N, int64_t K,
+                                        dg_stream_t stream) {
+  int rc = check_gemm_common(A, sfa, ld_sfa, B, sfb, D, M, N, K);
+  if (rc) return rc;
+  if (G < 1 || G > 1024) return DG_ERR_INVALID_ARG;
+  if (M == 0) return DG_OK;
+  if (!k_sizes || ld_sfb < N) return DG_ERR_INVALID_ARG;
+  if (ld_sfb % 4 != 0) return DG_ERR_ALIGNMENT;
+  if (!aligned16(k_sizes) || (C && !aligned16(C))) return DG_ERR_ALIGNMENT;
+  rc = check_device();
+  if (rc) return rc;
+  GemmParams p{};
+  p.status = device_info()->status;
+  p.sfa = sfa;
+  p.ld_sfa = ld_sfa;
+  p.sfb = sfb;
+  p.ld_sfb = ld_sfb;
+  p.d_f32 = D;
+  p.c = C;
+  p.k_sizes = k_sizes;
+  p.rows = static_cast<int>(M);
+  p.n = static_cast<int>(N);
+  p.k = static_cast<int>(K);
+  p.groups = G;
+  return launch_fp8_gemm(kKGrouped, A, B, p, reinterpret_cast<cudaStream_t>(stream),
+                         effective_num_sms(), 0, nullptr);
+}
+
 int dg_get_device_status(dg_stream_t stream, int *status) {
   if (!status) return DG_ERR_INVALID_ARG;
   if (!device_info()) return DG_ERR_CUDA;

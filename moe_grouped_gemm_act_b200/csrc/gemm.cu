@@ -20,7 +20,8 @@
 //               sum per block), then tcgen05.commit frees the smem stage and
 //               publishes the buffer.  NBUF buffers let the tensor cores run
 //               up to NBUF blocks ahead of the promotion.
-//   warps 2-3   idle after set-up (warp 2 builds the masked prefix table);
+//   warps 2-3   idle after set-up (warp 2 builds the masked or k-grouped
+//               prefix table);
 //               warps 0-3 form the control warpgroup, whose registers the
 //               promotion warpgroups take over for BN = 256.
 //   warps 4-11  promotion: warp w reads TMEM lanes 32 (w mod 4) .. +31; warps
@@ -33,12 +34,18 @@
 //               and stores its row segment (valid rows).
 //
 // The kernel is persistent (one CTA per SM).  All roles walk the same tile
-// sequence produced by a scheduler that knows the three layouts:
+// sequence produced by a scheduler that knows the layouts:
 //   dense       tiles of D in an M-grouped raster (L2 reuse of B);
 //   contiguous  as dense over M_total, the expert of each 128-row block read
 //               from the per-row index; blocks holding only padding skipped;
 //   masked      per expert g, ceil(masked_m[g] / 128) row blocks x N blocks,
-//               counts read on the device (launch shape independent of them).
+//               counts read on the device (launch shape independent of them);
+//   k-grouped   the weight gradient ("DeepGEMM architecture deep dive",
+//               section 3, the grouped GEMM table): per group, a dense raster
+//               over its own K segment (sizes read on the device); B's scales
+//               are per column, so the producer also copies each block's
+//               slice of them into a shared-memory ring and the promotion
+//               scales per element; the output is FP32 D[g] = C[g] + ....
 // Dense small-M shapes split K (units = tile x split, one unit per CTA): the
 // splits of a tile form one thread-block cluster, leave their FP32 partials
 // in shared memory and each reduces a share over the cluster's distributed
@@ -81,7 +88,7 @@ __host__ __device__ constexpr int staged_epilogue(int sched) {
   return sched == kDenseAcc ? 2 : (sched == kDense || sched == kMasked) ? 1 : 0;
 }
 
-template <int BN, int STAGES, int NBUF, bool PAIR, int STAGED>
+template <int BN, int STAGES, int NBUF, bool PAIR, int STAGED, bool KG = false>
 struct Layout {
   // the pair form keeps half of the B tile (BN/2 rows) in each CTA
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK;
@@ -100,6 +107,14 @@ struct Layout {
   static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
   static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
   static constexpr uint32_t kPrefixOff = kMiscOff + 16;
+  // k-grouped: a ring of per-column B scale slices, one per K block in
+  // flight (STAGES in the shared-memory stages plus NBUF in the TMEM
+  // buffers), so the producer never refills a slot the promotion may still
+  // read; then the per-schedule tables (masked / k-grouped prefix sums)
+  static constexpr int kBetaSlots = KG ? STAGES + NBUF : 0;
+  static constexpr uint32_t kBetaOff = (kPrefixOff + 15u) & ~15u;
+  static constexpr uint32_t kBetaBytes = static_cast<uint32_t>(kBetaSlots) * BN * 4u;
+  static constexpr uint32_t kTableOff = kBetaOff + kBetaBytes;
   static constexpr uint32_t kCols = BN * NBUF;
   static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64
                                       : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
@@ -119,6 +134,7 @@ struct Tile {
 __device__ __forceinline__ int num_units(const GemmParams &p, int sched,
                                          const int *s_prefix) {
   if (sched == kMasked) return s_prefix[p.groups];
+  if (sched == kKGrouped) return p.groups * p.num_m_blocks * p.num_n_blocks;
   return p.full_tiles + (p.num_m_blocks * p.num_n_blocks - p.full_tiles) * p.splits;
 }
 
@@ -152,7 +168,12 @@ __device__ __forceinline__ Tile unit_to_tile(const GemmParams &p, int sched,
     t.m_blk = r - t.n_blk * mb;
   } else {
     int tile = u;
-    if (u >= p.full_tiles) {
+    if (sched == kKGrouped) {
+      // groups one after the other, each rastered like a dense GEMM
+      const int per_group = p.num_m_blocks * p.num_n_blocks;
+      t.group = u / per_group;
+      tile = u - t.group * per_group;
+    } else if (u >= p.full_tiles) {
       const int v = u - p.full_tiles;
       tile = p.full_tiles + v / p.splits;
       t.split = v - (tile - p.full_tiles) * p.splits;
@@ -166,6 +187,12 @@ __device__ __forceinline__ Tile unit_to_tile(const GemmParams &p, int sched,
     const int r = tile - grp * span;
     t.m_blk = first_m + r % gm;
     t.n_blk = r / gm;
+  }
+  if (sched == kKGrouped) {
+    // the group's K blocks (prefix sums of the group sizes, in K blocks)
+    t.k_begin = s_prefix[t.group];
+    t.k_end = s_prefix[t.group + 1];
+    return t;
   }
   const int kb = p.num_k_blocks, s = t.nsplit;
   t.k_begin = (kb * t.split) / s;
@@ -223,7 +250,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // (measured 1 % faster for them)
   constexpr int kStaged = staged_epilogue(SCHED);
   constexpr bool kDenseLike = SCHED == kDense || SCHED == kDenseAcc;
-  using L = Layout<BN, STAGES, NBUF, PAIR, kStaged>;
+  constexpr bool kKG = SCHED == kKGrouped;
+  using L = Layout<BN, STAGES, NBUF, PAIR, kStaged, kKG>;
   constexpr int TM = PAIR ? 2 * BM : BM;   // rows per tile
   static_assert(!PAIR || SCHED == kDense, "the pair form serves dense GEMMs");
   constexpr int W = BN / 2;                 // columns per promotion thread
@@ -251,7 +279,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *s_flag = reinterpret_cast<int *>(smem + L::kMiscOff + 8);
-  int *s_prefix = reinterpret_cast<int *>(smem + L::kPrefixOff);        // [groups + 1]
+  int *s_prefix = reinterpret_cast<int *>(smem + L::kTableOff);         // [groups + 1]
   int *s_mblocks = s_prefix + (SCHED == kMasked ? p.groups + 1 : 0);   // [groups]
 
   const int warp = threadIdx.x >> 5;
@@ -318,6 +346,41 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       if (lane == 0) s_prefix[p.groups] = running;
     }
   }
+  if constexpr (kKG) {
+    if (warp == 2) {
+      // prefix[g] = K blocks of groups 0 .. g-1.  A size that is negative or
+      // off the 128 grid, or sizes that do not add up to K, are recorded as
+      // DG_ERR_DEVICE_DATA; every prefix is clamped to [0, K/128] (each lane
+      // adds at most K/128, the running sum stops at K/128 + 1), so no group
+      // reads past the operands or their scales.
+      const int kb_all = p.num_k_blocks;
+      int running = 0;
+      for (int g0 = 0; g0 < p.groups; g0 += 32) {
+        const int g = g0 + lane;
+        int nb = 0;
+        if (g < p.groups) {
+          const int ks = __ldg(p.k_sizes + g);
+          if (ks < 0 || ks % BK != 0) {
+            record_status(p.status, DG_ERR_DEVICE_DATA);
+          } else {
+            nb = min(ks / BK, kb_all);
+          }
+        }
+        int incl = nb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        if (g < p.groups) s_prefix[g] = min(running + incl - nb, kb_all);
+        running = min(running + __shfl_sync(0xffffffffu, incl, 31), kb_all + 1);
+      }
+      if (lane == 0) {
+        if (running != kb_all) record_status(p.status, DG_ERR_DEVICE_DATA);
+        s_prefix[p.groups] = min(running, kb_all);
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before any remote use
@@ -348,6 +411,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       // the DRAM latency the epilogue would otherwise wait on
       const int c_kb = (SCHED == kDenseAcc && t.split == 0) ? max(t.k_begin, t.k_end - kCAhead)
                                                             : -1;
+      // k-grouped: the tile's slice of B's column scales for each K block
+      // (N % 8 == 0, so a multiple of 32 bytes; 16-byte aligned because the
+      // scale rows are and the tile starts on a 16-column boundary)
+      const int b_col0 = t.n_blk * BN;
+      const uint32_t beta_bytes = kKG ? static_cast<uint32_t>(min(BN, p.n - b_col0)) * 4u : 0u;
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
         if constexpr (SCHED == kDenseAcc) {
           if (kb == c_kb) {
@@ -370,6 +438,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2 * stage_tx);
             tma_load_3d_pair(sa, &tmap_a, fb, kb * BK, a_row, t.slab);
             tma_load_3d_pair(sa + kABytes, &tmap_b, fb, kb * BK, b_row, t.group);
+          } else if constexpr (kKG) {
+            // B is one [N][K] tensor for all groups
+            mbar_arrive_expect_tx(full_bar(s), stage_tx + beta_bytes);
+            tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, 0);
+            tma_load_3d(sa + kABytes, &tmap_b, full_bar(s), kb * BK, b_row, 0);
+            bulk_load(base + L::kBetaOff + static_cast<uint32_t>(it % L::kBetaSlots) * (BN * 4u),
+                      p.sfb + static_cast<int64_t>(kb) * p.ld_sfb + b_col0, beta_bytes,
+                      full_bar(s));
           } else {
             mbar_arrive_expect_tx(full_bar(s), stage_tx);
             tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, t.slab);
@@ -493,19 +569,27 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       // shuffle.
       const float *a_src = p.sfa + static_cast<int64_t>(t.slab) * kg_total * p.ld_sfa +
                            min(row, p.rows - 1);
-      float a_cur = __ldg(a_src + static_cast<int64_t>(t.k_begin) * p.ld_sfa);
+      // (a k-grouped tile may have no K blocks: its D is its C)
+      float a_cur = !kKG || t.k_begin < t.k_end
+                        ? __ldg(a_src + static_cast<int64_t>(t.k_begin) * p.ld_sfa)
+                        : 0.0f;
       float a_next = t.k_begin + 1 < t.k_end
                          ? __ldg(a_src + static_cast<int64_t>(t.k_begin + 1) * p.ld_sfa)
                          : 0.0f;
-      float b_batch = t.k_begin + lane < t.k_end ? __ldg(sfb_ptr + t.k_begin + lane) : 0.0f;
+      float b_batch =
+          !kKG && t.k_begin + lane < t.k_end ? __ldg(sfb_ptr + t.k_begin + lane) : 0.0f;
       float b_batch_next =
-          t.k_begin + 32 + lane < t.k_end ? __ldg(sfb_ptr + t.k_begin + 32 + lane) : 0.0f;
+          !kKG && t.k_begin + 32 + lane < t.k_end ? __ldg(sfb_ptr + t.k_begin + 32 + lane)
+                                                   : 0.0f;
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
-        const int j = (kb - t.k_begin) & 31;
-        const float sc = a_cur * __shfl_sync(0xffffffffu, b_batch, j);
-        if (j == 31) {
-          b_batch = b_batch_next;
-          b_batch_next = kb + 33 + lane < t.k_end ? __ldg(sfb_ptr + kb + 33 + lane) : 0.0f;
+        float sc = a_cur;
+        if constexpr (!kKG) {
+          const int j = (kb - t.k_begin) & 31;
+          sc = a_cur * __shfl_sync(0xffffffffu, b_batch, j);
+          if (j == 31) {
+            b_batch = b_batch_next;
+            b_batch_next = kb + 33 + lane < t.k_end ? __ldg(sfb_ptr + kb + 33 + lane) : 0.0f;
+          }
         }
         a_cur = a_next;
         if (kb + 2 < t.k_end) a_next = __ldg(a_src + static_cast<int64_t>(kb + 2) * p.ld_sfa);
@@ -515,27 +599,57 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           break;
         }
         tc_fence_after();
+        // k-grouped: this block's column scales (landed with the stage that
+        // fed the MMA, which completed before tmem_full); this thread's W
+        // columns, the same addresses for the whole warp (a broadcast)
+        const uint32_t beta_s = kKG ? base + L::kBetaOff +
+                                          static_cast<uint32_t>(it % L::kBetaSlots) * (BN * 4u) +
+                                          static_cast<uint32_t>(half * W) * 4u
+                                    : 0u;
 #pragma unroll
         for (int c0 = 0; c0 < W; c0 += LW) {
           uint32_t r[LW];
           tmem_ld<LW>(tmem_base + t_lane + buf * BN + half * W + c0, r);
           tmem_wait_ld();
           reg_barrier<LW>(r);
-          if (c0 + LW == W) {
-            // all of this buffer has been read: hand it back to the MMA warp
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-              if constexpr (PAIR) {
-                mbar_arrive_cluster(tempty_target0 + 8u * buf);
-              } else {
-                mbar_arrive(tempty_bar(buf));
+          if constexpr (kKG) {
+            // acc += alpha_i * (P_ij * beta_j).  The buffer goes back only
+            // after the last scale read: its release lets the MMA warp free
+            // the stage whose refill reuses this block's ring slot.
+#pragma unroll
+            for (int c = 0; c < LW; c += 4) {
+              const uint4 bq = ld_shared_v4(beta_s + static_cast<uint32_t>(c0 + c) * 4u);
+              float y0 = 0.0f, y1 = 0.0f, y2 = 0.0f, y3 = 0.0f;
+              ffma2v(y0, y1, __uint_as_float(r[c]), __uint_as_float(r[c + 1]),
+                     __uint_as_float(bq.x), __uint_as_float(bq.y));
+              ffma2v(y2, y3, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]),
+                     __uint_as_float(bq.z), __uint_as_float(bq.w));
+              ffma2(acc[c0 + c], acc[c0 + c + 1], y0, y1, sc);
+              ffma2(acc[c0 + c + 2], acc[c0 + c + 3], y2, y3, sc);
+            }
+            if (c0 + LW == W) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tempty_bar(buf));
+            }
+          } else {
+            if (c0 + LW == W) {
+              // all of this buffer has been read: hand it back to the MMA warp
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                if constexpr (PAIR) {
+                  mbar_arrive_cluster(tempty_target0 + 8u * buf);
+                } else {
+                  mbar_arrive(tempty_bar(buf));
+                }
               }
             }
-          }
 #pragma unroll
-          for (int c = 0; c < LW; c += 2)
-            ffma2(acc[c0 + c], acc[c0 + c + 1], __uint_as_float(r[c]), __uint_as_float(r[c + 1]), sc);
+            for (int c = 0; c < LW; c += 2)
+              ffma2(acc[c0 + c], acc[c0 + c + 1], __uint_as_float(r[c]), __uint_as_float(r[c + 1]),
+                    sc);
+          }
         }
       }
       if (!alive) break;
@@ -633,6 +747,29 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           }
         }
         continue;  // this split's share of D is written
+      }
+      if constexpr (kKG) {
+        // D[g] = C[g] + A_g B_g^T in FP32: each thread stores its row
+        // segment, 16 bytes at a time, adding the matching 16 bytes of C
+        if (row_ok) {
+          const int64_t off = (static_cast<int64_t>(t.group) * p.rows + row) * p.n;
+          float *drow = p.d_f32 + off;
+#pragma unroll
+          for (int c = 0; c < W; c += 4) {
+            if (col0 + c < p.n) {
+              float4 v = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+              if (p.c != nullptr) {
+                const float4 cv = __ldg(reinterpret_cast<const float4 *>(p.c + off + col0 + c));
+                v.x += cv.x;
+                v.y += cv.y;
+                v.z += cv.z;
+                v.w += cv.w;
+              }
+              *reinterpret_cast<float4 *>(drow + col0 + c) = v;
+            }
+          }
+        }
+        continue;
       }
       if constexpr (SCHED == kDenseCluster) {
         // Leave this split's FP32 partial in this CTA's shared memory (the
@@ -856,9 +993,9 @@ constexpr Candidate kCandidates[] = {
 // The pair form: 256 x 256 tiles, half of B per CTA (32 KB stages).
 constexpr Candidate kPairCandidate = {256, 6, 2};
 
-template <int BN, int STAGES, int NBUF, bool PAIR, int STAGED>
+template <int BN, int STAGES, int NBUF, bool PAIR, int STAGED, bool KG = false>
 constexpr int smem_bytes_for(int extra) {
-  return 1024 + Layout<BN, STAGES, NBUF, PAIR, STAGED>::kPrefixOff + extra;
+  return 1024 + Layout<BN, STAGES, NBUF, PAIR, STAGED, KG>::kTableOff + extra;
 }
 
 bool print_configs() {
@@ -869,7 +1006,8 @@ bool print_configs() {
 template <int BN, int STAGES, int NBUF, int SCHED, bool PAIR>
 int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                     int grid, int extra_smem, cudaStream_t stream, bool coop) {
-  const int smem = smem_bytes_for<BN, STAGES, NBUF, PAIR, staged_epilogue(SCHED)>(extra_smem);
+  const int smem = smem_bytes_for<BN, STAGES, NBUF, PAIR, staged_epilogue(SCHED),
+                                  SCHED == kKGrouped>(extra_smem);
   auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED, PAIR>;
   static int configured_smem[64] = {0};  // per device; grows only
   int dev = 0;
@@ -949,23 +1087,29 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
   return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
-// Dynamic shared memory of a tile form (extra = the masked prefix tables;
-// `staged` = the output staging tile, see staged_epilogue).
-int config_smem(int bn, bool pair, int extra, bool staged) {
+// Dynamic shared memory of a single-CTA tile form for a schedule (extra =
+// its prefix tables).
+template <int BN, int STAGES, int NBUF>
+int single_smem(int sched, int extra) {
+  switch (staged_epilogue(sched)) {
+    case 1: return smem_bytes_for<BN, STAGES, NBUF, false, 1>(extra);
+    case 2: return smem_bytes_for<BN, STAGES, NBUF, false, 2>(extra);
+    default:
+      return sched == kKGrouped ? smem_bytes_for<BN, STAGES, NBUF, false, 0, true>(extra)
+                                : smem_bytes_for<BN, STAGES, NBUF, false, 0>(extra);
+  }
+}
+
+int config_smem(int bn, bool pair, int extra, int sched) {
   if (pair)
     return smem_bytes_for<kPairCandidate.bn, kPairCandidate.stages, kPairCandidate.nbuf, true,
-                          true>(extra);
+                          staged_epilogue(kDense)>(extra);
   switch (bn) {
-    case 256: return staged ? smem_bytes_for<256, 4, 2, false, true>(extra)
-                            : smem_bytes_for<256, 4, 2, false, false>(extra);
-    case 128: return staged ? smem_bytes_for<128, 6, 4, false, true>(extra)
-                            : smem_bytes_for<128, 6, 4, false, false>(extra);
-    case 64: return staged ? smem_bytes_for<64, 8, 8, false, true>(extra)
-                           : smem_bytes_for<64, 8, 8, false, false>(extra);
-    case 32: return staged ? smem_bytes_for<32, 8, 8, false, true>(extra)
-                           : smem_bytes_for<32, 8, 8, false, false>(extra);
-    case 16: return staged ? smem_bytes_for<16, 8, 8, false, true>(extra)
-                           : smem_bytes_for<16, 8, 8, false, false>(extra);
+    case 256: return single_smem<256, 4, 2>(sched, extra);
+    case 128: return single_smem<128, 6, 4>(sched, extra);
+    case 64: return single_smem<64, 8, 8>(sched, extra);
+    case 32: return single_smem<32, 8, 8>(sched, extra);
+    case 16: return single_smem<16, 8, 8>(sched, extra);
     default: return 1 << 30;
   }
 }
@@ -1081,11 +1225,12 @@ Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, 
                      size_t ws_bytes, int extra = 0, int max_smem = 232448) {
   const int64_t m_blocks = (rows + BM - 1) / BM;
   const int64_t k_blocks = k / BK;
-  const int64_t m_blocks_eff = sched == kMasked ? m_blocks * groups : m_blocks;
+  const int64_t m_blocks_eff =
+      (sched == kMasked || sched == kKGrouped) ? m_blocks * groups : m_blocks;
   Choice c{128, 1, false, 0};
   double best = 1e300;
   for (const Candidate &cand : kCandidates) {
-    if (config_smem(cand.bn, false, extra, staged_epilogue(sched)) > max_smem) continue;
+    if (config_smem(cand.bn, false, extra, sched) > max_smem) continue;
     const int64_t tiles = m_blocks * ((n + cand.bn - 1) / cand.bn);
     for (int s = 1; s <= 16; ++s) {
       if (s > 1 && (sched != kDense || m_blocks > 2)) break;
@@ -1134,7 +1279,8 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   // ------------------------------------------------ choose the tile form
   // masked launches keep per-expert row-block counts and prefix sums in
   // shared memory
-  const int extra = sched == kMasked ? 8 * (p.groups + 1) : 0;
+  const int extra = sched == kMasked ? 8 * (p.groups + 1)
+                    : sched == kKGrouped ? 4 * (p.groups + 1) : 0;
   const int max_smem = max_smem_per_block();
   const Choice choice =
       choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes, extra, max_smem);
@@ -1199,7 +1345,8 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
       full_tiles = waves * num_sms;
     }
   }
-  if (config_smem(bn, pair, extra, staged_epilogue(sched)) > max_smem)
+  if (config_smem(bn, pair, extra, pair ? kDense : (sched == kDense && acc ? kDenseAcc : sched)) >
+      max_smem)
     return DG_ERR_INVALID_ARG;  // too many experts
   const int tile_rows = pair ? 2 * BM : BM;
   p.num_m_blocks = static_cast<int>((rows + tile_rows - 1) / tile_rows);
@@ -1208,7 +1355,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   p.full_tiles = splits > 1 ? static_cast<int>(full_tiles) : 0;
   const int64_t all_tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
   p.ws = nullptr;
-  p.ws_ticket = nullptr;
+  if (sched != kKGrouped) p.ws_ticket = nullptr;  // (k-grouped: ld_sfb shares it)
   // Every tile split (decode-sized shapes, one wave): the splits of a tile
   // form a cluster and reduce through distributed shared memory, needing no
   // workspace or arrival counters, when all clusters fit in one wave
@@ -1239,7 +1386,8 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   p.a_box_rows = (sched == kDense && !pair && rows <= BM / 2) ? BM / 2 : BM;
   int rc = make_tmap(&ta, A, k, rows, sched == kMasked ? p.groups : 1, p.a_box_rows);
   if (rc) return rc;
-  rc = make_tmap(&tb, B, k, n, sched == kDense ? 1 : p.groups, pair ? bn / 2 : bn);
+  rc = make_tmap(&tb, B, k, n, (sched == kDense || sched == kKGrouped) ? 1 : p.groups,
+                 pair ? bn / 2 : bn);
   if (rc) return rc;
 
   // ------------------------------------------------ grid
@@ -1247,6 +1395,9 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   if (sched == kMasked) {
     // upper bound; the kernel reads the actual count from masked_m
     units = static_cast<int64_t>(p.num_m_blocks) * p.groups * p.num_n_blocks;
+  } else if (sched == kKGrouped) {
+    units = static_cast<int64_t>(p.groups) * all_tiles;
+    if (units > 0x7FFFFFFF) return DG_ERR_INVALID_ARG;
   } else {
     units = p.full_tiles + (all_tiles - p.full_tiles) * splits;
   }
@@ -1298,6 +1449,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
                  : dispatch<kDense>(bn, pair, ta, tb, p, grid, extra, stream);
     case kContiguous: return dispatch<kContiguous>(bn, false, ta, tb, p, grid, extra, stream);
     case kMasked: return dispatch<kMasked>(bn, false, ta, tb, p, grid, extra, stream);
+    case kKGrouped: return dispatch<kKGrouped>(bn, false, ta, tb, p, grid, extra, stream);
     default: return DG_ERR_INVALID_ARG;
   }
 }

@@ -35,22 +35,40 @@ inline cudaLaunchAttribute pdl_attribute() {
 // distributed shared memory (decode-sized shapes; no workspace).
 // kDenseAcc: dense tiles with D = C + A B^T (an FP32 C added before the BF16
 // rounding); the host picks it for a dense launch that has a C.
-enum Sched : int { kDense = 0, kContiguous = 1, kMasked = 2, kDenseCluster = 3, kDenseAcc = 4 };
+// kKGrouped: the groups split K; group g computes its own FP32
+// D[g] = C[g] + A_g B_g^T over its K segment, with 1x128 scales on both
+// operands (one B scale per column and K block).
+enum Sched : int {
+  kDense = 0, kContiguous = 1, kMasked = 2, kDenseCluster = 3, kDenseAcc = 4, kKGrouped = 5
+};
 
 // Kernel parameters besides the two tensor maps.  Row coordinates are inside
 // one "slab": the whole of A for dense and contiguous, one expert's M_max rows
-// for masked.
+// for masked.  The k-grouped schedule's own fields share storage with fields
+// it does not use (so the struct, and every other schedule's code, stays as
+// it was).
 struct GemmParams {
   const float *sfa;      // MN-major alpha: [slab][K/128][ld_sfa]
   int64_t ld_sfa;
-  const float *sfb;      // beta: [group][ceil(N/128)][K/128]
-  uint16_t *d;           // BF16 output [slab][rows][N]
-  const float *c;        // dense D = C + A B^T: FP32 C [rows][N] (nullptr: none)
+  const float *sfb;      // beta: [group][ceil(N/128)][K/128]; k-grouped:
+                         // MN-major [K/128][ld_sfb], one scale per column
+  union {
+    uint16_t *d;         // BF16 output [slab][rows][N]
+    float *d_f32;        // k-grouped: FP32 output [group][rows][N]
+  };
+  const float *c;        // dense D = C + A B^T: FP32 C [rows][N]; k-grouped:
+                         // [group][rows][N] (nullptr: none)
   const int32_t *m_indices;  // contiguous: expert per row (-1 = padding)
-  const int32_t *masked_m;   // masked: valid rows per expert
+  union {
+    const int32_t *masked_m;  // masked: valid rows per expert
+    const int32_t *k_sizes;   // k-grouped: K of each group, multiples of 128
+  };
   int *status;           // device status word (first error wins)
   float *ws;             // split-K partials (nullptr: no split)
-  uint32_t *ws_ticket;   // split-K arrival counters, one per output tile
+  union {
+    uint32_t *ws_ticket;  // split-K arrival counters, one per output tile
+    int64_t ld_sfb;       // k-grouped: row stride of the B scales
+  };
   int rows;              // dense: M; contiguous: M_total; masked: M_max
   int n, k;
   int groups;            // experts (1 for dense)

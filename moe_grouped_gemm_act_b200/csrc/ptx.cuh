@@ -203,6 +203,19 @@ __device__ __forceinline__ void ffma2(float &a0, float &a1, float x0, float x1,
       : "f"(x0), "f"(x1), "f"(s));
 }
 
+// a0 = x0 * s0 + a0 and a1 = x1 * s1 + a1: as ffma2 with a scale per lane.
+__device__ __forceinline__ void ffma2v(float &a0, float &a1, float x0, float x1,
+                                       float s0, float s1) {
+  asm("{\n\t.reg .b64 d, x, y;\n\t"
+      "mov.b64 d, {%0, %1};\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %5};\n\t"
+      "fma.rn.f32x2 d, x, y, d;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1), "f"(s0), "f"(s1));
+}
+
 // ------------------------------------------------------------------ tcgen05
 // Allocates `ncols` TMEM columns (power of two >= 32); the base address is
 // written to shared memory at `dst`.  Whole warp.

@@ -57,3 +57,17 @@ def check_gemm(got_bits: np.ndarray, want_f64: np.ndarray, what: str = "") -> No
     worst = np.max(np.abs(diff) - bound)
     assert fro <= REL_FRO, f"{what}: relative Frobenius error {fro:.3e}"
     assert worst <= 0, f"{what}: element bound exceeded by {worst:.3e}"
+
+
+def check_f32(got: np.ndarray, want_f64: np.ndarray, what: str = "") -> None:
+    """The same acceptance bound for an FP32 result."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want_f64, np.float64)
+    assert got.shape == want.shape
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    diff = got - want
+    fro = np.linalg.norm(diff) / max(np.linalg.norm(want), 1e-300)
+    rms = np.sqrt(np.mean(want ** 2))
+    worst = np.max(np.abs(diff) - (REL_ELEM * np.abs(want) + ABS_RMS * rms))
+    assert fro <= REL_FRO, f"{what}: relative Frobenius error {fro:.3e}"
+    assert worst <= 0, f"{what}: element bound exceeded by {worst:.3e}"

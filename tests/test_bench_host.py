@@ -45,8 +45,26 @@ def test_workload_specs_name_their_bound():
 
 
 def test_measured_traffic_follows_the_source_hash(monkeypatch):
-    monkeypatch.setitem(bench.GEMM_TRAFFIC, "source", bench.gemm_source_hash())
-    assert bench.measured_traffic("prefill") == bench.GEMM_TRAFFIC["prefill"]
-    monkeypatch.setitem(bench.GEMM_TRAFFIC, "source", "0" * 16)
+    monkeypatch.setitem(bench.GEMM_TRAFFIC, "prefill", (bench.gemm_source_hash(), 1.5e8))
+    assert bench.measured_traffic("prefill") == 1.5e8
+    monkeypatch.setitem(bench.GEMM_TRAFFIC, "prefill", ("0" * 16, 1.5e8))
     assert bench.measured_traffic("prefill") is None
+    assert bench.measured_traffic("no such workload") is None
     assert np.isfinite(bench.job_throughput(1.0, 1, 1, 1.0))
+
+
+def test_default_workload_traffic_matches_the_current_sources():
+    # the bench's default line must carry the traffic of the sources it runs
+    assert bench.measured_traffic("prefill") is not None
+
+
+def test_code_key_ignores_comments_but_not_code():
+    src = 'int f(int x) {  // doubles\n  /* the "// value" */ return 2 * x; }\nconst char *s = "a // b";\n'
+    same = 'int f(int x) {\n  return 2 * x;  // changed comment\n}\nconst char *s = "a // b";'
+    other = 'int f(int x) { return 3 * x; }\nconst char *s = "a // b";'
+    lit = 'int f(int x) { return 2 * x; }\nconst char *s = "a // c";'
+    key = bench.gemm_source_hash([src])
+    assert bench.gemm_source_hash([same]) == key
+    assert bench.gemm_source_hash([other]) != key
+    assert bench.gemm_source_hash([lit]) != key       # text inside a literal is code
+    assert bench.strip_comments("a/*x*/b") == "a b"

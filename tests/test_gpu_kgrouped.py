@@ -1,0 +1,184 @@
+"""GPU parity of the k-grouped contiguous GEMM (MoE weight gradient) against
+the oracle, through the C ABI: every N-tile instance on ragged M and N with
+empty groups (also the first and the last), with and without C, exact
+integers, a weight-gradient-shaped layout, determinism, and segment sizes
+that break the layout's rules reported through the device status word."""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import moe_grouped_gemm_act_b200 as dg
+from moe_grouped_gemm_act_b200 import inputs
+from oracle import e4m3, gemm, quant
+
+from _helpers import check_f32, dev, sfa_to_device
+
+pytestmark = pytest.mark.gpu
+
+
+class env:
+    def __init__(self, **kv):
+        self.kv = {k: str(v) for k, v in kv.items()}
+
+    def __enter__(self):
+        self.old = {k: os.environ.get(k) for k in self.kv}
+        os.environ.update(self.kv)
+
+    def __exit__(self, *a):
+        for k, v in self.old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
+def make_case(m, n, k_sizes, seed, with_c=True):
+    k_total = int(sum(k_sizes))
+    a = inputs.activations(m, k_total, seed=seed, outliers=True)
+    b = inputs.activations(n, k_total, seed=seed + 1)
+    qa, alpha = quant.quantize_1x128(a)
+    qb, beta = quant.quantize_1x128(b)
+    c = (inputs.rng(seed + 2).standard_normal((len(k_sizes), m, n)) * 4).astype(np.float32) \
+        if with_c else None
+    return qa, alpha, qb, beta, np.asarray(k_sizes, np.int32), c
+
+
+def run(qa, alpha, qb, beta, k_sizes, c):
+    g = len(k_sizes)
+    m, n = qa.shape[0], qb.shape[0]
+    d = torch.full((g, m, n), float("nan"), dtype=torch.float32, device="cuda")
+    dg.dg_k_grouped_fp8_gemm_nt_contiguous(
+        dev(qa), sfa_to_device(alpha), dev(qb), sfa_to_device(beta), d, dev(k_sizes),
+        c=None if c is None else dev(c))
+    torch.cuda.synchronize()
+    return d.cpu().numpy()
+
+
+@pytest.mark.parametrize("bn", [256, 128, 64, 32, 16])
+def test_ragged_every_block_n_with_empty_groups(cuda_device, bn):
+    k_sizes = [0, 384, 0, 128, 640, 0]
+    qa, alpha, qb, beta, ks, c = make_case(200, 264, k_sizes, seed=100 + bn)
+    dg.dg_get_device_status()
+    with env(DG_BLOCK_N=bn):
+        got = run(qa, alpha, qb, beta, ks, c)
+    assert dg.dg_get_device_status() == dg.DG_OK
+    want = gemm.k_grouped_contiguous_f64(qa, alpha, qb, beta, ks, c)
+    for g, size in enumerate(k_sizes):
+        if size == 0:
+            assert np.array_equal(got[g], c[g]), f"empty group {g} is not C"
+        else:
+            check_f32(got[g], want[g], f"BN={bn} group {g}")
+
+
+def test_without_c_empty_groups_are_zero(cuda_device):
+    k_sizes = [256, 0, 512]
+    qa, alpha, qb, beta, ks, _ = make_case(130, 136, k_sizes, seed=110, with_c=False)
+    got = run(qa, alpha, qb, beta, ks, None)
+    want = gemm.k_grouped_contiguous_f64(qa, alpha, qb, beta, ks)
+    assert not got[1].any()
+    check_f32(got[0], want[0], "group 0")
+    check_f32(got[2], want[2], "group 2")
+
+
+def test_integer_codes_are_exact(cuda_device):
+    rng = np.random.default_rng(111)
+    k_sizes = [1024, 128, 0, 2048]
+    m, n, k = 136, 144, sum(k_sizes)
+    a = rng.integers(-4, 5, size=(m, k)).astype(np.float32)
+    b = rng.integers(-4, 5, size=(n, k)).astype(np.float32)
+    qa, qb = e4m3.encode_rne(a), e4m3.encode_rne(b)
+    ones_a = np.ones((m, k // 128), np.float32)
+    ones_b = np.ones((n, k // 128), np.float32)
+    ks = np.asarray(k_sizes, np.int32)
+    got = run(qa, ones_a, qb, ones_b, ks, None)
+    want = gemm.k_grouped_contiguous_f64(qa, ones_a, qb, ones_b, ks)
+    assert np.array_equal(got.astype(np.float64), want)
+
+
+def test_weight_gradient_layout_and_determinism(cuda_device):
+    lay = inputs.k_grouped_layout(8192, 8, seed=112)
+    m, n = 512, 1024
+    k_total = lay.k_total
+    a = inputs.activations(m, k_total, seed=113, outliers=True)
+    b = inputs.activations(n, k_total, seed=114)
+    # the padding tokens of every segment are zeros
+    valid = np.zeros(k_total, bool)
+    start = 0
+    for cnt, size in zip(lay.counts, lay.k_sizes):
+        valid[start:start + int(cnt)] = True
+        start += int(size)
+    a[:, ~valid] = 0.0
+    b[:, ~valid] = 0.0
+    qa, alpha = quant.quantize_1x128(a)
+    qb, beta = quant.quantize_1x128(b)
+    c = (inputs.rng(115).standard_normal((8, m, n))).astype(np.float32)
+    got = run(qa, alpha, qb, beta, lay.k_sizes, c)
+    again = run(qa, alpha, qb, beta, lay.k_sizes, c)
+    assert np.array_equal(got.view(np.uint32), again.view(np.uint32))
+    want = gemm.k_grouped_contiguous_f64(qa, alpha, qb, beta, lay.k_sizes, c)
+    for g in range(8):
+        check_f32(got[g], want[g], f"group {g}")
+
+
+def test_device_quantized_operands(cuda_device):
+    # A and B quantized on the device: the layout the entry point documents
+    k_sizes = [256, 384]
+    m, n = 96, 200
+    a = inputs.activations(m, sum(k_sizes), seed=116, outliers=True)
+    b = inputs.activations(n, sum(k_sizes), seed=117)
+    qa_d, sfa_d = dg.dg_quantize_1x128(torch.from_numpy(a).cuda())
+    qb_d, sfb_d = dg.dg_quantize_1x128(torch.from_numpy(b).cuda())
+    d = torch.empty((2, m, n), dtype=torch.float32, device="cuda")
+    dg.dg_k_grouped_fp8_gemm_nt_contiguous(qa_d, sfa_d, qb_d, sfb_d, d,
+                                           dev(np.asarray(k_sizes, np.int32)))
+    torch.cuda.synchronize()
+    qa, alpha = quant.quantize_1x128(a)
+    qb, beta = quant.quantize_1x128(b)
+    want = gemm.k_grouped_contiguous_f64(qa, alpha, qb, beta, k_sizes)
+    got = d.cpu().numpy()
+    for g in range(2):
+        check_f32(got[g], want[g], f"group {g}")
+
+
+@pytest.mark.parametrize("k_sizes", [[128, 100, 28], [128, 128], [512, 256], [-128, 512]])
+def test_sizes_off_the_rules_are_reported(cuda_device, k_sizes):
+    # K is 384 here: sizes off the 128 grid, short or long of K, negative
+    qa, alpha, qb, beta, _, _ = make_case(64, 64, [384], seed=118, with_c=False)
+    ks = np.asarray(k_sizes, np.int32)
+    dg.dg_get_device_status()
+    d = torch.zeros((len(k_sizes), 64, 64), dtype=torch.float32, device="cuda")
+    dg.dg_k_grouped_fp8_gemm_nt_contiguous(dev(qa), sfa_to_device(alpha), dev(qb),
+                                           sfa_to_device(beta), d, dev(ks))
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == dg.DG_ERR_DEVICE_DATA
+    assert torch.isfinite(d).all()
+
+
+def test_host_argument_checks(cuda_device):
+    qa, alpha, qb, beta, ks, _ = make_case(8, 16, [128], seed=119, with_c=False)
+    lib = dg.load_library()
+    a_d, b_d = dev(qa), dev(qb)
+    sfa_d, sfb_d = sfa_to_device(alpha), sfa_to_device(beta)
+    d = torch.zeros((1, 8, 16), dtype=torch.float32, device="cuda")
+    ks_d = dev(ks)
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def call(G=1, M=8, N=16, K=128, ld_sfa=8, ld_sfb=16, k_sizes=ks_d.data_ptr()):
+        return lib.dg_k_grouped_fp8_gemm_nt_contiguous(
+            a_d.data_ptr(), sfa_d.data_ptr(), ld_sfa, b_d.data_ptr(), sfb_d.data_ptr(), ld_sfb,
+            None, d.data_ptr(), k_sizes, G, M, N, K, stream)
+
+    assert call() == dg.DG_OK
+    assert call(G=0) == dg.DG_ERR_INVALID_ARG
+    assert call(G=1025) == dg.DG_ERR_INVALID_ARG
+    assert call(K=100) == dg.DG_ERR_INVALID_ARG
+    assert call(N=12) == dg.DG_ERR_INVALID_ARG
+    assert call(ld_sfb=8) == dg.DG_ERR_INVALID_ARG
+    assert call(ld_sfb=18) == dg.DG_ERR_ALIGNMENT
+    assert call(k_sizes=None) == dg.DG_ERR_INVALID_ARG
+    assert call(M=0) == dg.DG_OK
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == dg.DG_OK
