@@ -147,6 +147,12 @@ def workload_spec(name: str) -> dict:
         return dict(name=name, kind="masked", bound="hbm", **inputs.MASKED,
                     desc="m-grouped masked, G=32, M_max=256, N=7168 K=2048, "
                          "masked_m ~ U{0..256}")
+    if name == "kgrouped":
+        return dict(name=name, kind="kgrouped", bound="tensor", **inputs.K_GROUPED,
+                    desc="k-grouped contiguous (MoE weight gradient), G=8, M=4096 N=7168, "
+                         "32768 tokens multinomial over experts along K, segments padded "
+                         "to 128; A~N(0,1) with 0.1% x50 outliers, B~N(0,1); 1x128 FP32 "
+                         "scales on both, FP32 D[g] out")
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -318,6 +324,10 @@ class DenseData:
         # shape (a split-K call also enqueues a runtime memset, not counted)
         return 2 * len(self.shapes)
 
+    def input_bytes(self) -> float:
+        """Bytes of inputs a step streams (FP32 activations and FP8 B)."""
+        return sum(s["a32"].numel() * 4 + s["qb"].numel() for s in self.shapes)
+
     # end-to-end through the public API from pinned host buffers
     def make_host(self):
         import torch
@@ -428,6 +438,79 @@ class GroupedData(DenseData):
             self.dg.dg_m_grouped_fp8_gemm_nt_masked(qa, sfa, qb, sfb, s["d"], index)
         else:
             self.dg.dg_m_grouped_fp8_gemm_nt_contiguous(qa, sfa, qb, sfb, s["d"], index)
+        h["d"].copy_(s["d"], non_blocking=True)
+
+
+class KGroupedData(DenseData):
+    """The MoE weight gradient: one step quantizes the activation gradient A
+    [M, K] and the activations B [N, K] (1x128 along the token axis K), then
+    runs the k-grouped GEMM into FP32 D [G, M, N].  FLOPs count the valid
+    tokens (not the padding of the segments)."""
+
+    def __init__(self, spec, device):
+        import torch
+        import moe_grouped_gemm_act_b200 as dg
+        self.dg = dg
+        a, b, lay = KGroupedOracleSample.generate(spec)
+        self.sample_src = KGroupedOracleSample.source(a, b)
+        G, m, n, k = spec["groups"], spec["m"], spec["n"], lay.k_total
+        a32 = torch.from_numpy(a).to(device)
+        b32 = torch.from_numpy(b).to(device)
+        qa = torch.empty((m, k), dtype=torch.uint8, device=device)
+        sfa = torch.empty((k // 128, dg.dg_get_tma_aligned_size(m, 4)), dtype=torch.float32,
+                          device=device)
+        qb = torch.empty((n, k), dtype=torch.uint8, device=device)
+        sfb = torch.empty((k // 128, dg.dg_get_tma_aligned_size(n, 4)), dtype=torch.float32,
+                          device=device)
+        d = torch.empty((G, m, n), dtype=torch.float32, device=device)
+        ks = torch.from_numpy(lay.k_sizes).to(device)
+        self.m = m
+        self.groups = G
+        self.k_total = k
+        tokens = int(lay.counts.sum())
+        self.shapes = [dict(n=n, k=tokens, a32=a32, b32=b32, qa=qa, sfa=sfa, qb=qb, sfb=sfb,
+                            d=d, k_sizes=ks, x_host=a, b_host=b, ws=None)]
+        torch.cuda.synchronize()
+
+    def gemm_bytes(self) -> float:
+        s = self.shapes[0]
+        m, n, k = self.m, s["n"], self.k_total
+        return (m + n) * k + 4 * (m + n) * (k // 128) + 4 * self.groups * m * n + 4 * self.groups
+
+    def gemm(self, s):
+        self.dg.dg_k_grouped_fp8_gemm_nt_contiguous(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"],
+                                                    s["k_sizes"])
+
+    def step(self):
+        s = self.shapes[0]
+        self.dg.dg_quantize_1x128(s["a32"], q=s["qa"], sf=s["sfa"])
+        self.dg.dg_quantize_1x128(s["b32"], q=s["qb"], sf=s["sfb"])
+        self.gemm(s)
+
+    def launches_per_step(self) -> int:
+        return 3
+
+    def input_bytes(self) -> float:
+        s = self.shapes[0]
+        return (s["a32"].numel() + s["b32"].numel()) * 4
+
+    def make_host(self):
+        s = self.shapes[0]
+        self.host = [dict(a=torch_pin(s["x_host"]), b=torch_pin(s["b_host"]),
+                          k_sizes=s["k_sizes"].cpu().pin_memory(),
+                          d=torch_empty_pinned(s["d"]))]
+        h = self.host[0]
+        self.h2d = (h["a"].numel() + h["b"].numel() + h["k_sizes"].numel()) * 4
+        self.d2h = h["d"].numel() * 4
+
+    def e2e_step(self, device):
+        s, h = self.shapes[0], self.host[0]
+        a = h["a"].to(device, non_blocking=True)
+        b = h["b"].to(device, non_blocking=True)
+        ks = h["k_sizes"].to(device, non_blocking=True)
+        qa, sfa = self.dg.dg_quantize_1x128(a)
+        qb, sfb = self.dg.dg_quantize_1x128(b)
+        self.dg.dg_k_grouped_fp8_gemm_nt_contiguous(qa, sfa, qb, sfb, s["d"], ks)
         h["d"].copy_(s["d"], non_blocking=True)
 
 
@@ -559,6 +642,65 @@ class GroupedOracleSample:
         return time.perf_counter() - t0, flops
 
 
+class KGroupedOracleSample:
+    """The CPU oracle on a bounded sample of the weight gradient: the first
+    ``rows`` rows of A and ``cols`` rows of B (rows and columns of every
+    D[g]) over the full K.  One run = quantize both samples (1x128) and run
+    the oracle's k-grouped GEMM; both operands are quantized per step on the
+    GPU too."""
+
+    @staticmethod
+    def generate(spec):
+        """The workload's host inputs: A [M, K], B [N, K] with zeros on the
+        padding tokens of every segment, and the layout."""
+        lay = inputs.k_grouped_layout(spec["tokens"], spec["groups"], seed=spec["seed"])
+        a = inputs.activations(spec["m"], lay.k_total, seed=spec["seed"] + 1, outliers=True)
+        b = inputs.activations(spec["n"], lay.k_total, seed=spec["seed"] + 2)
+        valid = np.zeros(lay.k_total, bool)
+        start = 0
+        for cnt, size in zip(lay.counts, lay.k_sizes):
+            valid[start:start + int(cnt)] = True
+            start += int(size)
+        a[:, ~valid] = 0.0
+        b[:, ~valid] = 0.0
+        return a, b, lay
+
+    @staticmethod
+    def source(a, b, rows: int = 64, cols: int = 1024):
+        return a[:rows].copy(), b[:cols].copy()
+
+    def __init__(self, spec, rows: int, cols: int, src=None):
+        lay = inputs.k_grouped_layout(spec["tokens"], spec["groups"], seed=spec["seed"])
+        if src is None:
+            a, b, _ = self.generate(spec)
+            src = self.source(a, b, rows, cols)
+        self.a, self.b = src[0][:rows], src[1][:cols]
+        self.k_sizes = lay.k_sizes
+        self.tokens = int(lay.counts.sum())
+        self.desc = (f"{len(self.a)} rows x {len(self.b)} columns of every D[g], full K "
+                     f"({self.tokens} tokens, k-grouped oracle)")
+
+    def run(self) -> tuple[float, float]:
+        """Returns (seconds, FLOPs) of one pass."""
+        from oracle import gemm as og, quant as oq
+        t0 = time.perf_counter()
+        qa, alpha = oq.quantize_1x128(self.a)
+        qb, beta = oq.quantize_1x128(self.b)
+        og.k_grouped_contiguous_f64(qa, alpha, qb, beta, self.k_sizes)
+        return time.perf_counter() - t0, 2.0 * len(self.a) * len(self.b) * self.tokens
+
+
+def make_sampler(spec, rows: int, cols: int, data=None):
+    """The oracle sample of a workload (from the GPU arm's host inputs when
+    ``data`` is given)."""
+    if spec["kind"] == "dense":
+        return OracleSample(spec, rows, cols)
+    src = None if data is None else data.sample_src
+    if spec["kind"] == "kgrouped":
+        return KGroupedOracleSample(spec, rows, cols, src=src)
+    return GroupedOracleSample(spec, rows, cols, src=src)
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -576,10 +718,7 @@ def run_reference(args, rank: int) -> None:
     if rank != 0:
         return
     spec = workload_spec(args.workload)
-    if spec["kind"] == "dense":
-        sampler = OracleSample(spec, args.ref_rows, args.ref_cols)
-    else:
-        sampler = GroupedOracleSample(spec, args.ref_rows, args.ref_cols)
+    sampler = make_sampler(spec, args.ref_rows, args.ref_cols)
     for _ in range(args.warmup):
         sampler.run()
     secs, flops = 0.0, 0.0
@@ -631,7 +770,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     torch.cuda.set_device(device)
     dg.load_library()
     spec = workload_spec(args.workload)
-    data = DenseData(spec, device) if spec["kind"] == "dense" else GroupedData(spec, device)
+    data = {"dense": DenseData, "kgrouped": KGroupedData}.get(spec["kind"], GroupedData)(
+        spec, device)
 
     def barrier():
         if world > 1:
@@ -719,11 +859,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        if spec["kind"] == "dense":
-            sampler = OracleSample(spec, args.ref_rows, args.ref_cols)
-        else:
-            sampler = GroupedOracleSample(spec, args.ref_rows, args.ref_cols,
-                                          src=data.sample_src)
+        sampler = make_sampler(spec, args.ref_rows, args.ref_cols, data)
         sampler.run()
         secs, fl = 0.0, 0.0
         while secs < 10.0:          # about 10 s of CPU work
@@ -737,11 +873,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3", "data": "synthetic",
-        "config": {"workload": spec["desc"], "m" if spec["kind"] == "dense" else "valid_rows": data.m,
+        "config": {"workload": spec["desc"], "valid_rows" if spec["kind"] in ("contiguous", "masked") else "m": data.m,
                    "nk": [[s["n"], s["k"]] for s in data.shapes],
                    "l2": "not flushed: each step streams %.0f MB of inputs (> 126 MB L2)"
-                         % ((sum(s["a32"].numel() * 4 + s["qb"].numel() for s in data.shapes))
-                            / 1e6),
+                         % (data.input_bytes() / 1e6),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "per_shape": per_shape},
         "roofline": roof,
@@ -761,7 +896,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="prefill",
                     choices=["prefill", "prefill_acc", "decode64", "decode128", "contiguous",
-                             "masked"])
+                             "masked", "kgrouped"])
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--ref-rows", type=int, default=16,
                     help="rows of A per shape in the oracle's timed sample")

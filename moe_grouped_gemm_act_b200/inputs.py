@@ -110,3 +110,6 @@ DECODE_M = [64, 128]
 DECODE_SEEDS = dict(seed_a=4, seed_b=5)
 CONTIGUOUS = dict(groups=8, n=4096, k=7168, tokens=32768, seed=6)
 MASKED = dict(groups=32, m_max=256, n=7168, k=2048, seed=7)
+# the weight gradient of the contiguous workload's GEMM: D[g] [4096, 7168] over
+# each expert's tokens
+K_GROUPED = dict(groups=8, m=4096, n=7168, tokens=32768, seed=8)

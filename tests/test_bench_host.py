@@ -37,8 +37,8 @@ def test_grouped_oracle_sample_takes_experts_with_rows():
 
 def test_workload_specs_name_their_bound():
     for name, bound in [("prefill", "tensor"), ("prefill_acc", "tensor"), ("decode64", "hbm"),
-                        ("decode128", "hbm"),
-                        ("contiguous", "tensor"), ("masked", "hbm")]:
+                        ("decode128", "hbm"), ("contiguous", "tensor"), ("masked", "hbm"),
+                        ("kgrouped", "tensor")]:
         assert bench.workload_spec(name)["bound"] == bound
     with pytest.raises(SystemExit):
         bench.workload_spec("nope")
@@ -68,3 +68,21 @@ def test_code_key_ignores_comments_but_not_code():
     assert bench.gemm_source_hash([other]) != key
     assert bench.gemm_source_hash([lit]) != key       # text inside a literal is code
     assert bench.strip_comments("a/*x*/b") == "a b"
+
+
+def test_k_grouped_oracle_sample():
+    spec = dict(kind="kgrouped", groups=3, m=40, n=136, tokens=300, seed=5)
+    a, b, lay = bench.KGroupedOracleSample.generate(spec)
+    assert a.shape == (40, lay.k_total) and b.shape == (136, lay.k_total)
+    # padding tokens are zero in both operands
+    start = 0
+    for cnt, size in zip(lay.counts, lay.k_sizes):
+        assert not a[:, start + int(cnt):start + int(size)].any()
+        assert not b[:, start + int(cnt):start + int(size)].any()
+        start += int(size)
+    s = bench.make_sampler(spec, rows=8, cols=64)
+    secs, flops = s.run()
+    assert secs > 0 and flops == 2.0 * 8 * 64 * 300
+    # the GPU arm's host slices give the same sample
+    s2 = bench.KGroupedOracleSample(spec, 8, 64, src=bench.KGroupedOracleSample.source(a, b))
+    assert np.array_equal(s2.a, s.a) and np.array_equal(s2.b, s.b)
