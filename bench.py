@@ -904,7 +904,7 @@ def main():
                     help="columns of D per shape in the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu DRAM bytes per GEMM launch, when measured for this build")
+                    help="ncu DRAM bytes per GEMM launch, when measured on the current sources")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
