@@ -271,16 +271,19 @@ class DenseData:
     def flops(self) -> float:
         return sum(2.0 * self.m * s["n"] * s["k"] for s in self.shapes)
 
-    def gemm_bytes(self) -> float:
-        """Algorithmic bytes of the GEMM launches (A, alpha, B, beta, D)."""
-        tot = 0.0
-        for s in self.shapes:
-            n, k = s["n"], s["k"]
-            tot += self.m * k + 4 * self.m * (k // 128) + n * k + \
-                4 * (-(-n // 128)) * (k // 128) + 2 * self.m * n
-            if self.acc:
-                tot += 4 * self.m * n  # C
+    def shape_bytes(self, s) -> float:
+        """Algorithmic bytes of one shape's GEMM launch (A, alpha, B, beta, D,
+        and C when accumulating)."""
+        n, k = s["n"], s["k"]
+        tot = self.m * k + 4 * self.m * (k // 128) + n * k + \
+            4 * (-(-n // 128)) * (k // 128) + 2 * self.m * n
+        if self.acc:
+            tot += 4 * self.m * n  # C
         return tot
+
+    def gemm_bytes(self) -> float:
+        """Algorithmic bytes of the GEMM launches of one step."""
+        return sum(self.shape_bytes(s) for s in self.shapes)
 
     def gemm(self, s):
         if self.acc:
@@ -403,6 +406,9 @@ class GroupedData(DenseData):
                             index=index, x_host=x)]
         torch.cuda.synchronize()
 
+    def shape_bytes(self, s) -> float:
+        return self.gemm_bytes()
+
     def gemm_bytes(self) -> float:
         s = self.shapes[0]
         n, k, v = s["n"], s["k"], self.m
@@ -472,6 +478,9 @@ class KGroupedData(DenseData):
                             d=d, k_sizes=ks, x_host=a, b_host=b, ws=None)]
         torch.cuda.synchronize()
 
+    def shape_bytes(self, s) -> float:
+        return self.gemm_bytes()
+
     def gemm_bytes(self) -> float:
         s = self.shapes[0]
         m, n, k = self.m, s["n"], self.k_total
@@ -512,6 +521,24 @@ class KGroupedData(DenseData):
         qb, sfb = self.dg.dg_quantize_1x128(b)
         self.dg.dg_k_grouped_fp8_gemm_nt_contiguous(qa, sfa, qb, sfb, s["d"], ks)
         h["d"].copy_(s["d"], non_blocking=True)
+
+
+def per_shape_report(data, per_shape_ms, bound: str, peak: float) -> list:
+    """Each shape's GEMM time, TFLOP/s and fraction of the roofline peak:
+    TFLOP/s over the FP8 peak for tensor-bound work, algorithmic GB/s over
+    the copy bandwidth for HBM-bound work."""
+    out = []
+    for s, ms in zip(data.shapes, per_shape_ms):
+        secs = ms * 1e-3
+        row = {"n": s["n"], "k": s["k"], "gemm_us": 1e3 * ms,
+               "tflops": 2.0 * data.m * s["n"] * s["k"] / secs / 1e12}
+        if bound == "tensor":
+            row["frac"] = row["tflops"] / peak
+        else:
+            row["gbs"] = data.shape_bytes(s) / secs / 1e9
+            row["frac"] = row["gbs"] / peak
+        out.append(row)
+    return out
 
 
 def torch_pin(a):
@@ -853,9 +880,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                 "frac": achieved / peak, "peak_source": f"{pk['source']} copy bandwidth"}
     roof["traffic"] = args.traffic if args.traffic is not None else measured_traffic(args.workload)
     roof["traffic_unit"] = "bytes per GEMM launch (ncu dram read + write)"
-    per_shape = [{"n": s["n"], "k": s["k"], "gemm_us": 1e3 * ms,
-                  "tflops": 2.0 * data.m * s["n"] * s["k"] / (ms * 1e-3) / 1e12}
-                 for s, ms in zip(data.shapes, per_shape_ms)]
+    per_shape = per_shape_report(data, per_shape_ms, spec["bound"], peak)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

@@ -86,3 +86,18 @@ def test_k_grouped_oracle_sample():
     # the GPU arm's host slices give the same sample
     s2 = bench.KGroupedOracleSample(spec, 8, 64, src=bench.KGroupedOracleSample.source(a, b))
     assert np.array_equal(s2.a, s.a) and np.array_equal(s2.b, s.b)
+
+
+def test_per_shape_report_fractions():
+    from types import SimpleNamespace
+    shapes = [dict(n=256, k=1024), dict(n=512, k=2048)]
+    data = SimpleNamespace(m=128, shapes=shapes, acc=False)
+    data.shape_bytes = lambda s: bench.DenseData.shape_bytes(data, s)
+    rows = bench.per_shape_report(data, [0.5, 2.0], "tensor", 1000.0)
+    assert rows[0]["tflops"] == pytest.approx(2 * 128 * 256 * 1024 / 0.5e-3 / 1e12)
+    assert rows[1]["frac"] == pytest.approx(rows[1]["tflops"] / 1000.0)
+    assert rows[0]["gemm_us"] == pytest.approx(500.0)
+    hb = bench.per_shape_report(data, [0.5, 2.0], "hbm", 6000.0)
+    want = 128 * 1024 + 4 * 128 * 8 + 256 * 1024 + 4 * 2 * 8 + 2 * 128 * 256
+    assert hb[0]["gbs"] == pytest.approx(want / 0.5e-3 / 1e9)
+    assert hb[0]["frac"] == pytest.approx(hb[0]["gbs"] / 6000.0)
