@@ -75,6 +75,27 @@ def fp8_gemm_nt(qa, alpha, qb, beta) -> np.ndarray:
     return bf16.to_bits(fp8_gemm_nt_f64(qa, alpha, qb, beta))
 
 
+LAYOUTS = ("nt", "nn", "tn", "tt")
+
+
+def fp8_gemm_f64(layout: str, qa_stored, alpha, qb_stored, beta) -> np.ndarray:
+    """The Fig. 13-1 formula for the four operand layouts of the Deep dive,
+    section 3 (D = A @ B.T for "nt"; the first letter says whether A is used
+    as stored or transposed, the second whether B is).  Stored shapes:
+    "nt" A [M, K], B [N, K]; "nn" A [M, K], B [K, N]; "tn" A [K, M],
+    B [K, N]; "tt" A [K, M], B [N, K].  The scales do not depend on the
+    layout: alpha [M, K/128] per row of A and 128-wide K group, beta
+    [ceil(N/128), K/128] per 128 x 128 block of B (in its [N, K] view).
+    Reading: the layouts only change how A and B are stored; D is still
+    [M, N] = sum over K, so the oracle views both operands as [M, K] and
+    [N, K] and evaluates the NT formula."""
+    if layout not in LAYOUTS:
+        raise ValueError(f"layout must be one of {LAYOUTS}")
+    qa = qa_stored.T if layout[0] == "t" else qa_stored
+    qb = qb_stored if layout[1] == "t" else qb_stored.T
+    return fp8_gemm_nt_f64(np.ascontiguousarray(qa), alpha, np.ascontiguousarray(qb), beta)
+
+
 def fp8_gemm_nt_accumulate_f64(qa, alpha, qb, beta, c) -> np.ndarray:
     """float64 C + A B^T (Deep dive, section 3: the NT GEMM's D = C + A @ B.T
     form), with C float32 [M, N] taken exactly and added to the float64

@@ -264,3 +264,40 @@ def test_accumulate_rounds_once_after_adding_c():
     assert gemm.fp8_gemm_nt_accumulate(qa, one, qb, one, c)[0, 0] == 0x3F81
     twice = bf16.to_bits(bf16.round_f64(gemm.fp8_gemm_nt_f64(qa, one, qb, one)) + c)
     assert twice[0, 0] == 0x3F80
+
+
+# ------------------------------------------------------------- operand layouts
+@pytest.mark.parametrize("layout,spec", [("nt", "mk,nk->mn"), ("nn", "mk,kn->mn"),
+                                         ("tn", "km,kn->mn"), ("tt", "km,nk->mn")])
+def test_layouts_match_an_einsum_over_the_stored_operands(layout, spec):
+    # the stored operands are contracted as they lie (no transposes), with
+    # each element's scale looked up by its logical (row, K) position
+    m, n, k = 24, 200, 384
+    qa, alpha, qb, beta = small_case(m=m, n=n, k=k, seed=120)
+    a_st = qa if layout[0] == "n" else np.ascontiguousarray(qa.T)
+    b_st = qb if layout[1] == "t" else np.ascontiguousarray(qb.T)
+    av = e4m3.decode(a_st)
+    bv = e4m3.decode(b_st)
+    ka = np.arange(k) // 128
+    sa = alpha[:, ka] if layout[0] == "n" else alpha[:, ka].T          # like a_st
+    sb_nk = beta[np.arange(n) // 128][:, ka]                            # [N, K]
+    sb = sb_nk if layout[1] == "t" else sb_nk.T                         # like b_st
+    want = np.einsum(spec, av * sa, bv * sb)
+    got = gemm.fp8_gemm_f64(layout, a_st, alpha, b_st, beta)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
+def test_layout_names_are_checked():
+    qa, alpha, qb, beta = small_case(m=8, n=16, k=128, seed=121)
+    with pytest.raises(ValueError):
+        gemm.fp8_gemm_f64("tx", qa, alpha, qb, beta)
+
+
+def test_a_layout_mix_up_is_caught():
+    # reading an "nn" B as if it were stored [N, K] fails the einsum pin
+    m, n, k = 16, 128, 128
+    qa, alpha, qb, beta = small_case(m=m, n=n, k=k, seed=122)
+    b_kn = np.ascontiguousarray(qb.T)
+    right = gemm.fp8_gemm_f64("nn", qa, alpha, b_kn, beta)
+    wrong = gemm.fp8_gemm_nt_f64(qa, alpha, np.ascontiguousarray(b_kn[:n, :k]), beta)
+    assert not np.allclose(right, wrong)
