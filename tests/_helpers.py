@@ -8,6 +8,8 @@ element, and the FP32 promotion plus the tensor cores' internal accumulation
 order add far less; the rms term absorbs cancellation near zero.
 """
 
+import os
+
 import numpy as np
 import torch
 
@@ -71,3 +73,21 @@ def check_f32(got: np.ndarray, want_f64: np.ndarray, what: str = "") -> None:
     worst = np.max(np.abs(diff) - (REL_ELEM * np.abs(want) + ABS_RMS * rms))
     assert fro <= REL_FRO, f"{what}: relative Frobenius error {fro:.3e}"
     assert worst <= 0, f"{what}: element bound exceeded by {worst:.3e}"
+
+
+class env:
+    """Temporarily set library tuning variables (read at each call)."""
+
+    def __init__(self, **kv):
+        self.kv = {k: str(v) for k, v in kv.items()}
+
+    def __enter__(self):
+        self.old = {k: os.environ.get(k) for k in self.kv}
+        os.environ.update(self.kv)
+
+    def __exit__(self, *a):
+        for k, v in self.old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v

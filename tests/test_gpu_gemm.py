@@ -3,8 +3,6 @@ C ABI): shapes spanning several tiles with ragged tails, every N-tile instance,
 split K, the exact-integer special case, untouched padding / masked rows,
 determinism and CUDA-graph replay of the masked call."""
 
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -13,29 +11,11 @@ import moe_grouped_gemm_act_b200 as dg
 from moe_grouped_gemm_act_b200 import inputs
 from oracle import bf16, e4m3, gemm, quant
 
-from _helpers import bits_of, check_gemm, dev, sfa_batched_to_device, sfa_to_device
+from _helpers import bits_of, check_gemm, dev, env, sfa_batched_to_device, sfa_to_device
 
 pytestmark = pytest.mark.gpu
 
 SENTINEL = 0x7FC1  # a NaN bit pattern no GEMM result can produce
-
-
-class env:
-    """Temporarily set library tuning variables (read at each call)."""
-
-    def __init__(self, **kv):
-        self.kv = {k: str(v) for k, v in kv.items()}
-
-    def __enter__(self):
-        self.old = {k: os.environ.get(k) for k in self.kv}
-        os.environ.update(self.kv)
-
-    def __exit__(self, *a):
-        for k, v in self.old.items():
-            if v is None:
-                os.environ.pop(k, None)
-            else:
-                os.environ[k] = v
 
 
 def dense_case(m, n, k, seed, outliers=True):

@@ -4,8 +4,6 @@ empty groups (also the first and the last), with and without C, exact
 integers, a weight-gradient-shaped layout, determinism, and segment sizes
 that break the layout's rules reported through the device status word."""
 
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -14,25 +12,9 @@ import moe_grouped_gemm_act_b200 as dg
 from moe_grouped_gemm_act_b200 import inputs
 from oracle import e4m3, gemm, quant
 
-from _helpers import check_f32, dev, sfa_to_device
+from _helpers import check_f32, dev, env, sfa_to_device
 
 pytestmark = pytest.mark.gpu
-
-
-class env:
-    def __init__(self, **kv):
-        self.kv = {k: str(v) for k, v in kv.items()}
-
-    def __enter__(self):
-        self.old = {k: os.environ.get(k) for k in self.kv}
-        os.environ.update(self.kv)
-
-    def __exit__(self, *a):
-        for k, v in self.old.items():
-            if v is None:
-                os.environ.pop(k, None)
-            else:
-                os.environ[k] = v
 
 
 def make_case(m, n, k_sizes, seed, with_c=True):
