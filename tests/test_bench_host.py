@@ -101,3 +101,78 @@ def test_per_shape_report_fractions():
     want = 128 * 1024 + 4 * 128 * 8 + 256 * 1024 + 4 * 2 * 8 + 2 * 128 * 256
     assert hb[0]["gbs"] == pytest.approx(want / 0.5e-3 / 1e9)
     assert hb[0]["frac"] == pytest.approx(hb[0]["gbs"] / 6000.0)
+
+
+def test_k_grouped_bench_data_on_the_host(monkeypatch):
+    # the weight-gradient workload's host logic, with a stand-in for the
+    # library (records the calls) and CPU tensors: no kernel runs here
+    import torch
+    calls = []
+
+    class FakeDG:
+        @staticmethod
+        def dg_get_tma_aligned_size(n, e):
+            return -(-n // 4) * 4
+
+        @staticmethod
+        def dg_quantize_1x128(x, q=None, sf=None):
+            calls.append(("quantize", tuple(x.shape)))
+            m, k = x.shape
+            return (torch.zeros((m, k), dtype=torch.uint8) if q is None else q,
+                    torch.zeros((k // 128, -(-m // 4) * 4)) if sf is None else sf)
+
+        @staticmethod
+        def dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, k_sizes, c=None):
+            calls.append(("kgrouped", tuple(a.shape), tuple(b.shape), tuple(d.shape),
+                          tuple(k_sizes.tolist())))
+            return d
+
+    import moe_grouped_gemm_act_b200 as dg_mod
+    for name in ("dg_get_tma_aligned_size", "dg_quantize_1x128",
+                 "dg_k_grouped_fp8_gemm_nt_contiguous"):
+        monkeypatch.setattr(dg_mod, name, getattr(FakeDG, name))
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a: None)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    spec = dict(name="kgrouped", kind="kgrouped", bound="tensor", groups=3, m=64, n=136,
+                tokens=300, seed=5, desc="test")
+    data = bench.KGroupedData(spec, torch.device("cpu"))
+    lay = inputs.k_grouped_layout(300, 3, seed=5)
+    k = lay.k_total
+    assert data.flops() == 2.0 * 64 * 136 * 300
+    assert data.gemm_bytes() == (64 + 136) * k + 4 * (64 + 136) * (k // 128) + \
+        4 * 3 * 64 * 136 + 4 * 3
+    assert data.input_bytes() == (64 + 136) * k * 4
+    assert data.launches_per_step() == 3
+    data.step()
+    assert calls == [("quantize", (64, k)), ("quantize", (136, k)),
+                     ("kgrouped", (64, k), (136, k), (3, 64, 136), tuple(lay.k_sizes))]
+    calls.clear()
+    data.make_host()
+    assert data.h2d == ((64 + 136) * k + 3) * 4 and data.d2h == 3 * 64 * 136 * 4
+    data.e2e_step(torch.device("cpu"))
+    assert [c[0] for c in calls] == ["quantize", "quantize", "kgrouped"]
+    rows = bench.per_shape_report(data, [1.0], "tensor", 1000.0)
+    assert rows[0]["k"] == 300 and rows[0]["tflops"] == pytest.approx(2 * 64 * 136 * 300 / 1e-3 / 1e12)
+    sampler = bench.make_sampler(spec, 8, 16, data)
+    assert isinstance(sampler, bench.KGroupedOracleSample)
+    assert sampler.a.shape == (8, k) and sampler.b.shape == (16, k)
+
+
+def test_dense_and_grouped_byte_helpers():
+    import torch
+    d = object.__new__(bench.DenseData)
+    d.m, d.acc = 64, True
+    d.shapes = [dict(n=256, k=512, a32=torch.zeros(64, 512), qb=torch.zeros(256, 512,
+                                                                             dtype=torch.uint8))]
+    s = d.shapes[0]
+    base = 64 * 512 + 4 * 64 * 4 + 256 * 512 + 4 * 2 * 4 + 2 * 64 * 256
+    assert d.shape_bytes(s) == base + 4 * 64 * 256
+    assert d.gemm_bytes() == d.shape_bytes(s)
+    assert d.input_bytes() == 64 * 512 * 4 + 256 * 512
+    g = object.__new__(bench.GroupedData)
+    g.m, g.active = 100, 2
+    g.shapes = [dict(n=256, k=512, index=torch.zeros(3, dtype=torch.int32),
+                     a32=torch.zeros(128, 512), qb=torch.zeros(4, 256, 512, dtype=torch.uint8))]
+    assert g.shape_bytes(g.shapes[0]) == g.gemm_bytes()
+    rows = bench.per_shape_report(g, [0.01], "hbm", 6540.0)
+    assert rows[0]["gbs"] == pytest.approx(g.gemm_bytes() / 1e-5 / 1e9)
