@@ -43,7 +43,9 @@ def _max_worker(rank, world, port, out):
 
 def test_max_over_ranks_two_gloo_ranks():
     world = 2
-    with mp.Manager() as m:
+    # the manager's server process is spawned too: forking a process that
+    # already runs threads can deadlock the child
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_max_worker, args=(world, free_port(), out), nprocs=world, join=True)
         got = dict(out)
