@@ -17,7 +17,9 @@
  *   layout (A row-major [M, K], B row-major [N, K], D = A * B^T), LHS scales
  *   stored transposed (MN-major) and TMA-aligned, contiguous grouped layout
  *   with expert segments aligned to the M block, masked grouped layout with a
- *   per-expert valid row count.
+ *   per-expert valid row count; every GEMM as D = C + A @ B (the accumulating
+ *   NT form), the K-grouped contiguous form of the MoE weight gradient, and
+ *   sm_100's packed UE8M0 scale layout.
  *
  * Conventions shared by every entry point:
  *   - Every pointer argument marked "device" must point to device memory of
@@ -27,8 +29,9 @@
  *   - The return value is a dg_status code.  Argument errors are detected on
  *     the host before anything is launched and leave outputs untouched.
  *     Errors found by a kernel on the device (bad expert index, masked_m out
- *     of range, a pipeline wait that timed out) are recorded in a device
- *     status word read by dg_get_device_status().
+ *     of range, k-grouped sizes off the rules, a scale UE8M0 cannot hold, a
+ *     pipeline wait that timed out) are recorded in a device status word
+ *     read by dg_get_device_status().
  *   - The library keeps a small amount of per-device state (device
  *     properties, the device status word), created by the first call on that
  *     device.  Make one call before capturing any call into a CUDA graph.
@@ -56,7 +59,7 @@ typedef struct CUstream_st *dg_stream_t;
 #define DG_ERR_CUDA -4             /* a CUDA runtime/driver call failed        */
 #define DG_ERR_WORKSPACE -5        /* workspace missing or too small           */
 #define DG_ERR_TIMEOUT -6          /* device: a pipeline wait gave up          */
-#define DG_ERR_DEVICE_DATA -7      /* device: bad m_indices / masked_m data    */
+#define DG_ERR_DEVICE_DATA -7      /* device: bad index / count / size / scale */
 
 /* Input element types for the quantizers. */
 #define DG_DTYPE_F32 0

@@ -108,7 +108,7 @@ const char *dg_status_string(int status) {
     case DG_ERR_CUDA: return "CUDA error";
     case DG_ERR_WORKSPACE: return "workspace missing or too small";
     case DG_ERR_TIMEOUT: return "a pipeline wait on the device timed out";
-    case DG_ERR_DEVICE_DATA: return "invalid m_indices / masked_m data on the device";
+    case DG_ERR_DEVICE_DATA: return "invalid index, count, size or scale data on the device";
     default: return "unknown status";
   }
 }
