@@ -14,6 +14,10 @@
 // Limit: the array holds kNoAllocScratchBytes (32 MiB).  A shape whose
 // preferred K split needs more (dg_fp8_gemm_nt_workspace_size above that) is
 // rejected with DG_ERR_WORKSPACE; shapes that do not split need no scratch.
+// Every split the GEMM picks keeps split tiles x splits <= the SM count, so
+// the need is at most SMs x 128 x 256 x 4 bytes plus one counter per SM: about
+// 19.4 MB on a 148-SM B200, under the limit for any device of up to 256 SMs,
+// where the refusal cannot happen.
 //
 // All calls on a device share the one array and leave their partial sums in
 // it; the split-K arrival counters are cleared by every call before its
@@ -40,12 +44,12 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 constexpr int kMaxDevices = 64;
 
-struct ScratchSlot {
-  std::once_flag once;
-  void *ptr = nullptr;
-  int status = DG_ERR_CUDA;
-};
-ScratchSlot g_slots[kMaxDevices];
+// Per device: the resolved address, or nullptr while it is not known.  Only
+// a successful lookup is kept, so a first call that failed (for instance one
+// made inside a stream capture) does not disable the entry point: the next
+// call tries again.
+void *g_scratch[kMaxDevices] = {};
+std::mutex g_scratch_mutex;
 
 // Device address of the scratch array on the current device.  The first call
 // on a device resolves it (this also loads the array's module on that device,
@@ -53,19 +57,17 @@ ScratchSlot g_slots[kMaxDevices];
 int scratch_on_current_device(void **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DG_ERR_CUDA;
-  ScratchSlot &s = g_slots[dev];
-  std::call_once(s.once, [&s] {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch[dev] == nullptr) {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess && p != nullptr) {
-      s.ptr = p;
-      s.status = DG_OK;
-    } else {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
       (void)cudaGetLastError();  // do not leave this error for the caller's next check
-      s.status = DG_ERR_CUDA;
+      return DG_ERR_CUDA;
     }
-  });
-  *out = s.ptr;
-  return s.status;
+    g_scratch[dev] = p;
+  }
+  *out = g_scratch[dev];
+  return DG_OK;
 }
 
 }  // namespace
@@ -83,7 +85,9 @@ extern "C" int dg_fp8_gemm_nt_noalloc(const uint8_t *A, const float *sfa, int64_
   void *scratch = nullptr;
   const int rc = scratch_on_current_device(&scratch);
   if (rc != DG_OK) return rc;
-  // the dense entry point validates the rest and launches with the scratch
-  return dg_fp8_gemm_nt(A, sfa, ld_sfa, B, sfb, D, M, N, K, scratch, kNoAllocScratchBytes,
+  // the dense entry point validates the rest and launches with the scratch,
+  // offered as exactly the bytes the size query reports, so that it picks the
+  // same tile form and split as dg_fp8_gemm_nt given that workspace
+  return dg_fp8_gemm_nt(A, sfa, ld_sfa, B, sfb, D, M, N, K, scratch, need > 16 ? need : 16,
                         stream);
 }
