@@ -211,10 +211,17 @@ size_t dg_fp8_gemm_nt_workspace_size(int64_t M, int64_t N, int64_t K);
  * the workspace.  Nothing is allocated and no allocating routine is called.
  *   - Returns DG_ERR_WORKSPACE (nothing launched) when the shape's preferred
  *     K split needs more than 32 MiB, i.e. when
- *     dg_fp8_gemm_nt_workspace_size(M, N, K) > 32 MiB.
+ *     dg_fp8_gemm_nt_workspace_size(M, N, K) > 32 MiB.  The split tiles
+ *     times their splits never exceed the SM count, so the need is at most
+ *     SMs x 128 KiB plus 4 bytes per SM (about 19.4 MB on a 148-SM B200):
+ *     devices of up to 256 SMs never see this error.
+ *   - Uses exactly the tile form and split that dg_fp8_gemm_nt picks when
+ *     given dg_fp8_gemm_nt_workspace_size(M, N, K) bytes of workspace, so
+ *     both give identical bits.
  *   - The first call on a device looks up the array's device address (and
  *     loads that code on the device); make that first call before any stream
- *     capture.
+ *     capture.  A lookup that fails returns DG_ERR_CUDA and is retried by
+ *     the next call.
  *   - All calls share the one array and leave their partial sums in it; each
  *     call clears the part that must start at zero before its kernel runs.
  *     Calls whose kernels overlap on the GPU (unordered streams) race on the

@@ -128,6 +128,45 @@ def _need_cuda(*ts: torch.Tensor) -> None:
             raise ValueError("tensors must be contiguous")
 
 
+def _expect(t: torch.Tensor | None, name: str, dtype: torch.dtype, shape: tuple) -> None:
+    """Raises ValueError unless t has this dtype and shape.  A shape entry of
+    None accepts any extent; a pair (lo, "ld") accepts any multiple of 4 that
+    is at least lo (the leading dimension of an MN-major scale tensor).  The C
+    ABI takes raw pointers and cannot check extents, so every tensor is
+    checked here before the call."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != len(shape):
+        raise ValueError(f"{name} must have {len(shape)} dimensions, got shape {tuple(t.shape)}")
+    for i, (got, want) in enumerate(zip(t.shape, shape)):
+        if want is None:
+            continue
+        if isinstance(want, tuple):
+            lo = want[0]
+            if got < lo or got % 4:
+                raise ValueError(f"{name}: dimension {i} is {got}; it must be a multiple of 4 "
+                                 f">= {lo} (shape {tuple(t.shape)})")
+        elif got != want:
+            raise ValueError(f"{name}: dimension {i} is {got}, expected {want} "
+                             f"(shape {tuple(t.shape)})")
+
+
+def _gemm_operands(a, sfa, b, sfb, m, n, k, groups=None, a_batch=None):
+    """Checks the FP8 operands and their scales of an NT GEMM: A [.., M, K]
+    uint8 with MN-major 1x128 scales [.., K/128, ld >= M], B [.., N, K] uint8
+    with 128x128 scales [.., ceil(N/128), K/128]."""
+    if k % 128:
+        return  # the C ABI rejects it (DG_ERR_INVALID_ARG) before touching memory
+    lead_a = () if a_batch is None else (a_batch,)
+    lead_b = () if groups is None else (groups,)
+    _expect(a, "a", torch.uint8, lead_a + (m, k))
+    _expect(sfa, "sfa", torch.float32, lead_a + (k // 128, (m, "ld")))
+    _expect(b, "b", torch.uint8, lead_b + (n, k))
+    _expect(sfb, "sfb", torch.float32, lead_b + (-(-n // 128), k // 128))
+
+
 # ------------------------------------------------------------------ helpers
 def dg_get_mk_alignment_for_contiguous_layout() -> int:
     return load_library().dg_get_mk_alignment_for_contiguous_layout()
@@ -177,6 +216,11 @@ def dg_quantize_1x128(x: torch.Tensor, pow2: bool = False, q=None, sf=None,
         q = torch.empty(xb.shape, dtype=torch.uint8, device=x.device)
     if sf is None:
         sf = torch.empty((b, k // 128, ld), dtype=torch.float32, device=x.device)
+    _need_cuda(q, sf)
+    if k % 128 == 0:  # (otherwise the C ABI rejects the call)
+        _expect(q if q.dim() == 3 else q.unsqueeze(0), "q", torch.uint8, (b, m, k))
+        _expect(sf if sf.dim() == 3 else sf.unsqueeze(0), "sf", torch.float32,
+                (b, k // 128, (m, "ld")))
     rc = load_library().dg_quantize_1x128(
         _ptr(xb), dtype, b, m, k, k, _ptr(q), k, _ptr(sf), sf.shape[-1],
         DG_SCALE_POW2 if pow2 else DG_SCALE_FP32, _stream(stream))
@@ -222,10 +266,14 @@ def dg_pack_ue8m0(sf: torch.Tensor, m: int, packed=None, stream=None) -> torch.T
     sb = sf if batched else sf.unsqueeze(0)
     b, kg, ld = sb.shape
     words = -(-kg // 4)
+    if m > ld:
+        raise ValueError(f"m = {m} exceeds the scale rows' leading dimension {ld}")
     if packed is None:
         packed = torch.empty((b, words, dg_get_tma_aligned_size(m, 4)), dtype=torch.int32,
                              device=sf.device)
     _need_cuda(packed)
+    _expect(packed if packed.dim() == 3 else packed.unsqueeze(0), "packed", torch.int32,
+            (b, words, (m, "ld")))
     rc = load_library().dg_pack_ue8m0(_ptr(sb), b, m, kg, ld, _ptr(packed), packed.shape[-1],
                                       _stream(stream))
     _check(rc, "dg_pack_ue8m0")
@@ -240,6 +288,10 @@ def dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace: torch.Tensor | None = None,
     _need_cuda(a, sfa, b, sfb, d)
     m, k = a.shape
     n = b.shape[0]
+    _gemm_operands(a, sfa, b, sfb, m, n, k)
+    _expect(d, "d", torch.bfloat16, (m, n))
+    if workspace is not None:
+        _need_cuda(workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = load_library().dg_fp8_gemm_nt(
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d), m, n, k,
@@ -255,6 +307,11 @@ def dg_fp8_gemm_nt_accumulate(a, sfa, b, sfb, c, d, workspace: torch.Tensor | No
     _need_cuda(a, sfa, b, sfb, c, d)
     m, k = a.shape
     n = b.shape[0]
+    _gemm_operands(a, sfa, b, sfb, m, n, k)
+    _expect(c, "c", torch.float32, (m, n))
+    _expect(d, "d", torch.bfloat16, (m, n))
+    if workspace is not None:
+        _need_cuda(workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = load_library().dg_fp8_gemm_nt_accumulate(
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(c), _ptr(d), m, n, k,
@@ -272,6 +329,8 @@ def dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, d, stream=None) -> torch.Tensor:
     _need_cuda(a, sfa, b, sfb, d)
     m, k = a.shape
     n = b.shape[0]
+    _gemm_operands(a, sfa, b, sfb, m, n, k)
+    _expect(d, "d", torch.bfloat16, (m, n))
     rc = load_library().dg_fp8_gemm_nt_noalloc(
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d), m, n, k,
         _stream(stream))
@@ -286,6 +345,9 @@ def dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices,
     _need_cuda(a, sfa, b, sfb, d, m_indices)
     m_total, k = a.shape
     g, n, _ = b.shape
+    _gemm_operands(a, sfa, b, sfb, m_total, n, k, groups=g)
+    _expect(d, "d", torch.bfloat16, (m_total, n))
+    _expect(m_indices, "m_indices", torch.int32, (m_total,))
     rc = load_library().dg_m_grouped_fp8_gemm_nt_contiguous(
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d),
         _ptr(m_indices), m_total, n, k, g, _stream(stream))
@@ -300,6 +362,9 @@ def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m,
     _need_cuda(a, sfa, b, sfb, d, masked_m)
     g, m_max, k = a.shape
     n = b.shape[1]
+    _gemm_operands(a, sfa, b, sfb, m_max, n, k, groups=g, a_batch=g)
+    _expect(d, "d", torch.bfloat16, (g, m_max, n))
+    _expect(masked_m, "masked_m", torch.int32, (g,))
     rc = load_library().dg_m_grouped_fp8_gemm_nt_masked(
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d),
         _ptr(masked_m), g, m_max, n, k, _stream(stream))
@@ -320,6 +385,15 @@ def dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, k_sizes, c=None,
     m, k = a.shape
     n = b.shape[0]
     g = k_sizes.numel()
+    if k % 128 == 0:  # (otherwise the C ABI rejects the call)
+        _expect(a, "a", torch.uint8, (m, k))
+        _expect(sfa, "sfa", torch.float32, (k // 128, (m, "ld")))
+        _expect(b, "b", torch.uint8, (n, k))
+        _expect(sfb, "sfb", torch.float32, (k // 128, (n, "ld")))
+    _expect(d, "d", torch.float32, (g, m, n))
+    _expect(k_sizes, "k_sizes", torch.int32, (g,))
+    if c is not None:
+        _expect(c, "c", torch.float32, (g, m, n))
     rc = load_library().dg_k_grouped_fp8_gemm_nt_contiguous(
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), sfb.shape[-1], _ptr(c),
         _ptr(d), _ptr(k_sizes), g, m, n, k, _stream(stream))
