@@ -76,10 +76,36 @@ constexpr int kControlWarps = 4;        // producer, MMA issuer, 2 helpers (one 
 constexpr int kPromoWarps = 8;          // two column halves x four lane quarters
 constexpr int kPromoThreads = 32 * kPromoWarps;
 constexpr int kThreads = 32 * (kControlWarps + kPromoWarps);
+// Register split of the 256-wide tile: the block is launched with 168
+// registers per thread (65536 / 384, in steps of 8); the control warpgroup
+// gives up most of them so that each promotion thread can hold its 128
+// accumulators and a 64-column TMEM chunk.  Either split uses exactly the
+// launch allocation (40 x 128 + 232 x 256 = 56 x 128 + 224 x 256 = 168 x 384);
+// per schedule, the one with which ptxas spills least.
+constexpr int kLaunchRegs = 168;
+__host__ __device__ constexpr int ctrl_regs(int sched) {
+  return (sched == kMasked || sched == kDenseCluster) ? 56 : 40;
+}
+__host__ __device__ constexpr int promo_regs(int sched) {
+  return (sched == kMasked || sched == kDenseCluster) ? 224 : 232;
+}
+static_assert(ctrl_regs(kDense) * 32 * kControlWarps + promo_regs(kDense) * kPromoThreads <=
+                  kLaunchRegs * kThreads,
+              "register split exceeds the launch allocation");
+static_assert(ctrl_regs(kMasked) * 32 * kControlWarps + promo_regs(kMasked) * kPromoThreads <=
+                  kLaunchRegs * kThreads,
+              "register split exceeds the launch allocation");
 constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
 constexpr int kCAhead = 8;              // K blocks between the C prefetch and the tile's end
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 constexpr int kClusterNoFit = 1;        // launch_instance: clusters do not fit one wave
+
+// Test hook: the K-block iteration whose loads CTA 0's producer leaves out
+// (-1: none).  Nothing then completes that stage's `full` barrier, so the MMA
+// warp's bounded wait on it runs out: the way the tests exercise the abort
+// path without faulting anything.  Set from the host only while the
+// DG_TEST_STARVE_LOAD variable is present.
+static __device__ int g_starve_load_it = -1;
 
 // How a schedule's epilogue stages the output tile in shared memory: 0 not
 // at all, 1 the BF16 tile, 2 the FP32 tile (D = C + A B^T adds C as it
@@ -88,10 +114,9 @@ __host__ __device__ constexpr int staged_epilogue(int sched) {
   return sched == kDenseAcc ? 2 : (sched == kDense || sched == kMasked) ? 1 : 0;
 }
 
-template <int BN, int STAGES, int NBUF, bool PAIR, int STAGED, bool KG = false>
+template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false>
 struct Layout {
-  // the pair form keeps half of the B tile (BN/2 rows) in each CTA
-  static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK;
+  static constexpr uint32_t kBBytes = BN * BK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   // With STAGED, staging of the output for coalesced stores: 128 rows x
   // kOutCols BF16 (kind 1: a 256-wide tile goes out in two column halves) or
@@ -232,15 +257,7 @@ __device__ __forceinline__ int masked_rows(const GemmParams &p, int e) {
 }
 
 // ------------------------------------------------------------------ the kernel
-//
-// PAIR: a 2-CTA cluster computes a 256 x BN tile with cta_group::2 MMAs
-// (M = 256).  Each CTA loads its own 128 rows of A and half of the B tile
-// (BN/2 rows), so every SM pulls half of B from L2 instead of all of it; both
-// CTAs' TMA loads complete on rank 0's `full` barrier, rank 0 issues the MMAs
-// and commits to the `empty` / `tmem_full` barriers of both CTAs, and the
-// promotion warps of both CTAs release TMEM buffers on rank 0's `tmem_empty`
-// barrier.  Each CTA promotes and stores its own 128 rows.
-template <int BN, int STAGES, int NBUF, int SCHED, bool PAIR>
+template <int BN, int STAGES, int NBUF, int SCHED>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
@@ -251,13 +268,18 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   constexpr int kStaged = staged_epilogue(SCHED);
   constexpr bool kDenseLike = SCHED == kDense || SCHED == kDenseAcc;
   constexpr bool kKG = SCHED == kKGrouped;
-  using L = Layout<BN, STAGES, NBUF, PAIR, kStaged, kKG>;
-  constexpr int TM = PAIR ? 2 * BM : BM;   // rows per tile
-  static_assert(!PAIR || SCHED == kDense, "the pair form serves dense GEMMs");
+  using L = Layout<BN, STAGES, NBUF, kStaged, kKG>;
   constexpr int W = BN / 2;                 // columns per promotion thread
-  // columns per TMEM load chunk: the whole slice up to 64; for BN = 256 the
-  // 128 accumulators leave room for 16-column chunks under 168 registers
-  constexpr int LW = W <= 64 ? W : 16;
+  // BN = 256 runs with the warpgroup register split (promo_regs per promotion
+  // thread), the narrower tiles fit the launch allocation as they are.  The
+  // contiguous schedule keeps the launch allocation: with the split, ptxas
+  // spills in its promotion loop (measured 40 % slower).
+  constexpr bool kRegSplit = BN == 256 && SCHED != kContiguous;
+  // columns per TMEM load chunk: the whole slice up to 64 (one wait per
+  // chunk; the buffer is handed back after the last chunk's wait, so the
+  // fewer chunks, the sooner the MMA warp can reuse it); 16 for a 256-wide
+  // tile without the register split (128 accumulators under 168 registers)
+  constexpr int LW = W <= 64 ? W : kRegSplit ? 64 : 16;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(W % LW == 0 && (LW == 8 || LW == 16 || LW == 32 || LW == 64), "TMEM chunk");
 
@@ -284,9 +306,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0;   // 0 issues the pair's MMAs
-  const int u_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int u_stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int u_first = static_cast<int>(blockIdx.x);
+  const int u_stride = static_cast<int>(gridDim.x);
 
   // ---------------------------------------------------------------- setup
   // the next kernel of the stream may begin its own set-up as our CTAs leave
@@ -300,7 +321,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), PAIR ? 2 * kPromoWarps : kPromoWarps);
+      mbar_init(tempty_bar(b), kPromoWarps);
     }
     mbar_init(drain_bar, 1);
     mbar_init(epi_bar, kPromoThreads);
@@ -309,13 +330,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    if constexpr (PAIR) {
-      tmem_alloc_pair(smem_u32(s_tmem), L::kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(smem_u32(s_tmem), L::kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc(smem_u32(s_tmem), L::kTmemCols);
+    tmem_relinquish();
   }
   // nothing above touched global memory; from here on the previous kernel's
   // results (A, the scales, the index arrays) are visible
@@ -383,18 +399,21 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   }
   tc_fence_before();
   __syncthreads();
-  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int units = num_units(p, SCHED, s_prefix);
   const int kg_total = p.num_k_blocks;
 
+  if (warp < kControlWarps) {
+  // the control warpgroup (all four warps) hands its spare registers over
+  if constexpr (kRegSplit) setmaxnreg_dec<ctrl_regs(SCHED)>();
   if (warp == 0) {
     // ============================================================ producer
     // bytes per stage: the A box (128 rows, or 64 when M <= 64: the MMA then
     // reads stale rows 64-127, which only reach output rows that are never
     // stored) and the B box
     const uint32_t stage_tx = static_cast<uint32_t>(p.a_box_rows) * BK + L::kBBytes;
+    const int starve_it = blockIdx.x == 0 ? g_starve_load_it : -1;
     int it = 0;
     bool alive = true;
     for (int u = u_first; u < units && alive; u += u_stride) {
@@ -403,8 +422,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         t.group = block_expert(p, t.m_blk, true);
         if (t.group < 0) continue;
       }
-      const int a_row = t.m_blk * TM + static_cast<int>(rank) * BM;
-      const int b_row = t.n_blk * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
+      const int a_row = t.m_blk * BM;
+      const int b_row = t.n_blk * BN;
       // D = C + A B^T: the epilogue's C rows are asked into L2 kCAhead K
       // blocks before the tile's last one -- late enough that the operand
       // stream of a long K does not evict them first, early enough to cover
@@ -429,16 +448,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!mbar_wait(empty_bar(s), ph ^ 1, s_abort, p.status)) { alive = false; break; }
-        if (lane == 0) {
+        if (lane == 0 && it != starve_it) {
           const uint32_t sa = base + s * L::kStageBytes;
-          if constexpr (PAIR) {
-            // both CTAs' stage bytes complete on rank 0's full barrier, whose
-            // single arrival (with the pair's byte count) comes from rank 0
-            const uint32_t fb = mapa_shared(full_bar(s), 0);
-            if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2 * stage_tx);
-            tma_load_3d_pair(sa, &tmap_a, fb, kb * BK, a_row, t.slab);
-            tma_load_3d_pair(sa + kABytes, &tmap_b, fb, kb * BK, b_row, t.group);
-          } else if constexpr (kKG) {
+          if constexpr (kKG) {
             // B is one [N][K] tensor for all groups
             mbar_arrive_expect_tx(full_bar(s), stage_tx + beta_bytes);
             tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, 0);
@@ -455,12 +467,18 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         __syncwarp();
       }
     }
+    // No copy may still be writing this CTA's shared memory when it exits:
+    // wait (bounded, and not cut short by the abort flag) for the `full`
+    // barrier of each of the last STAGES iterations armed above.  Earlier
+    // iterations were consumed by the MMA warp, so their copies landed.
+    volatile int never = 0;
+    for (int i = max(0, it - STAGES); i < it; ++i)
+      if (i != starve_it) mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &never, p.status);
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    // (in the pair form only rank 0 issues; rank 1's warp 1 idles)
-    constexpr uint32_t idesc = idesc_e4m3_f32(TM, BN);
+    constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
     int it = 0, acc_it = 0;
-    bool alive = rank == 0;
+    bool alive = true;
     for (int u = u_first; u < units && alive; u += u_stride) {
       Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
       if constexpr (SCHED == kContiguous) {
@@ -483,42 +501,27 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           for (int k = 0; k < BK / 32; ++k) {
             // +32 bytes along K inside the swizzled 128-byte row = +2 in the
             // descriptor's 16-byte address field
-            if constexpr (PAIR) {
-              umma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
-            } else {
-              umma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
-            }
+            umma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
           }
           // publish the buffer first: the promotion is on the critical path,
           // the producer has STAGES - 1 blocks of slack
-          if constexpr (PAIR) {
-            umma_commit_pair(mapa_shared(tfull_bar(buf), 0));
-            umma_commit_pair(mapa_shared(tfull_bar(buf), 1));
-            umma_commit_pair(mapa_shared(empty_bar(s), 0));
-            umma_commit_pair(mapa_shared(empty_bar(s), 1));
-          } else {
-            umma_commit(tfull_bar(buf));
-            umma_commit(empty_bar(s));
-          }
+          umma_commit(tfull_bar(buf));
+          umma_commit(empty_bar(s));
         }
         __syncwarp();
       }
     }
-    if (rank == 0) {
+    {
       // every MMA issued above must complete before TMEM is freed (bounded,
       // and not cut short by the abort flag)
-      if (lane == 0) {
-        if constexpr (PAIR) {
-          umma_commit_pair(mapa_shared(drain_bar, 0));
-        } else {
-          umma_commit(drain_bar);
-        }
-      }
+      if (lane == 0) umma_commit(drain_bar);
       __syncwarp();
       volatile int never = 0;
       mbar_wait(drain_bar, 0, &never, p.status);
     }
-  } else if (warp >= kControlWarps) {
+  }
+  } else {
+    if constexpr (kRegSplit) setmaxnreg_inc<promo_regs(SCHED)>();
     // ============================================================ promotion
     const int pw = warp - kControlWarps;   // 0..7
     const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
@@ -526,8 +529,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
     const int nb_total = (p.n + 127) / 128;
-    // TMEM buffers are handed back on rank 0's barrier (the MMA issuer's)
-    const uint32_t tempty_target0 = PAIR ? mapa_shared(tempty_bar(0), 0) : tempty_bar(0);
     int it = 0;
     bool alive = true;
     // every promotion thread arrives, then waits for the phase (bounded)
@@ -540,7 +541,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     };
     for (int u = u_first; u < units && alive; u += u_stride) {
       Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
-      const int row = t.m_blk * TM + static_cast<int>(rank) * BM + row_in_tile;
+      const int row = t.m_blk * BM + row_in_tile;
       bool row_ok;
       if constexpr (SCHED == kContiguous) {
         t.group = block_expert(p, t.m_blk, false);
@@ -637,13 +638,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
               // all of this buffer has been read: hand it back to the MMA warp
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) {
-                if constexpr (PAIR) {
-                  mbar_arrive_cluster(tempty_target0 + 8u * buf);
-                } else {
-                  mbar_arrive(tempty_bar(buf));
-                }
-              }
+              if (lane == 0) mbar_arrive(tempty_bar(buf));
             }
 #pragma unroll
             for (int c = 0; c < LW; c += 2)
@@ -688,7 +683,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (!epi_sync()) break;
         if (*s_abort) break;
         __threadfence();
-        const int row0 = t.m_blk * TM + static_cast<int>(rank) * BM;
+        const int row0 = t.m_blk * BM;
         const int valid = min(BM, p.rows - row0);
         const int slots = valid * (BN / 4);
         const int share = (slots + p.splits - 1) / p.splits;
@@ -820,7 +815,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const uint32_t s_out = base + L::kOutOff;
         uint8_t *s_rowok = smem + L::kRowOkOff;
         const int ptid = threadIdx.x - kControlWarps * 32;
-        const int64_t row0 = static_cast<int64_t>(t.m_blk) * TM;
+        const int64_t row0 = static_cast<int64_t>(t.m_blk) * BM;
         if (half == 0) s_rowok[row_in_tile] = row_ok ? 1 : 0;
 #pragma unroll
         for (int ph = 0; ph < kPhases; ++ph) {
@@ -879,8 +874,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const uint32_t s_out = base + L::kOutOff;
         uint8_t *s_rowok = smem + L::kRowOkOff;
         const int ptid = threadIdx.x - kControlWarps * 32;
-        const int64_t slab_row0 = static_cast<int64_t>(t.slab) * p.rows + t.m_blk * TM +
-                                  static_cast<int>(rank) * BM;
+        const int64_t slab_row0 = static_cast<int64_t>(t.slab) * p.rows + t.m_blk * BM;
         if (half == 0) s_rowok[row_in_tile] = row_ok ? 1 : 0;
 #pragma unroll
         for (int ph = 0; ph < kPhases; ++ph) {
@@ -969,17 +963,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  // in the pair form neither CTA leaves (or frees TMEM) while rank 0's MMAs
-  // may still read the peer's shared memory: rank 0 drained them above
-  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
-  if (warp == 1) {
-    if constexpr (PAIR) {
-      tmem_dealloc_pair(tmem_base, L::kTmemCols);
-    } else {
-      tmem_dealloc(tmem_base, L::kTmemCols);
-    }
-  }
+  if (warp == 1) tmem_dealloc(tmem_base, L::kTmemCols);
 }
 
 // ------------------------------------------------------------------ host side
@@ -990,12 +975,10 @@ struct Candidate {
 // flight; NBUF fills the 512 TMEM columns (at most 8 buffers).
 constexpr Candidate kCandidates[] = {
     {256, 4, 2}, {128, 6, 4}, {64, 8, 8}, {32, 8, 8}, {16, 8, 8}};
-// The pair form: 256 x 256 tiles, half of B per CTA (32 KB stages).
-constexpr Candidate kPairCandidate = {256, 6, 2};
 
-template <int BN, int STAGES, int NBUF, bool PAIR, int STAGED, bool KG = false>
+template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false>
 constexpr int smem_bytes_for(int extra) {
-  return 1024 + Layout<BN, STAGES, NBUF, PAIR, STAGED, KG>::kTableOff + extra;
+  return 1024 + Layout<BN, STAGES, NBUF, STAGED, KG>::kTableOff + extra;
 }
 
 bool print_configs() {
@@ -1003,23 +986,35 @@ bool print_configs() {
   return e && *e && *e != '0';
 }
 
-template <int BN, int STAGES, int NBUF, int SCHED, bool PAIR>
+template <int BN, int STAGES, int NBUF, int SCHED>
 int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                     int grid, int extra_smem, cudaStream_t stream, bool coop) {
-  const int smem = smem_bytes_for<BN, STAGES, NBUF, PAIR, staged_epilogue(SCHED),
+  const int smem = smem_bytes_for<BN, STAGES, NBUF, staged_epilogue(SCHED),
                                   SCHED == kKGrouped>(extra_smem);
-  auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED, PAIR>;
+  auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED>;
   static int configured_smem[64] = {0};  // per device; grows only
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DG_ERR_CUDA;
+  if constexpr (BN == 256) {
+    // the warpgroup register split needs the full launch allocation: never
+    // launch an instance compiled to fewer registers (its promotion warps
+    // would wait for registers that never come)
+    static int regs_checked = 0;  // 1 ok, -1 too few
+    if (regs_checked == 0) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return DG_ERR_CUDA;
+      regs_checked = fa.numRegs >= kLaunchRegs ? 1 : -1;
+    }
+    if (regs_checked < 0) return DG_ERR_CUDA;
+  }
   if (smem > configured_smem[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return DG_ERR_CUDA;
     configured_smem[dev] = smem;
   }
-  // clusters: the CTA pair, or the `splits` CTAs of a tile
-  const int cluster = PAIR ? 2 : SCHED == kDenseCluster ? p.splits : 1;
+  // clusters: the `splits` CTAs of a tile
+  const int cluster = SCHED == kDenseCluster ? p.splits : 1;
   if constexpr (SCHED == kDenseCluster) {
     // every cluster must be resident at once (one wave): ask the occupancy
     // calculator how many clusters of this size fit (cached per device)
@@ -1092,18 +1087,15 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
 template <int BN, int STAGES, int NBUF>
 int single_smem(int sched, int extra) {
   switch (staged_epilogue(sched)) {
-    case 1: return smem_bytes_for<BN, STAGES, NBUF, false, 1>(extra);
-    case 2: return smem_bytes_for<BN, STAGES, NBUF, false, 2>(extra);
+    case 1: return smem_bytes_for<BN, STAGES, NBUF, 1>(extra);
+    case 2: return smem_bytes_for<BN, STAGES, NBUF, 2>(extra);
     default:
-      return sched == kKGrouped ? smem_bytes_for<BN, STAGES, NBUF, false, 0, true>(extra)
-                                : smem_bytes_for<BN, STAGES, NBUF, false, 0>(extra);
+      return sched == kKGrouped ? smem_bytes_for<BN, STAGES, NBUF, 0, true>(extra)
+                                : smem_bytes_for<BN, STAGES, NBUF, 0>(extra);
   }
 }
 
-int config_smem(int bn, bool pair, int extra, int sched) {
-  if (pair)
-    return smem_bytes_for<kPairCandidate.bn, kPairCandidate.stages, kPairCandidate.nbuf, true,
-                          staged_epilogue(kDense)>(extra);
+int config_smem(int bn, int extra, int sched) {
   switch (bn) {
     case 256: return single_smem<256, 4, 2>(sched, extra);
     case 128: return single_smem<128, 6, 4>(sched, extra);
@@ -1124,24 +1116,17 @@ int max_smem_per_block() {
 }
 
 template <int SCHED>
-int dispatch(int bn, bool pair, const CUtensorMap &ta, const CUtensorMap &tb,
-             const GemmParams &p, int grid, int extra, cudaStream_t st) {
+int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+             int grid, int extra, cudaStream_t st) {
   // splits that wait for each other through global memory need all CTAs
   // resident; a cluster's splits are co-scheduled by construction
   const bool coop = p.splits > 1 && SCHED != kDenseCluster;
-  if (pair) {
-    if constexpr (SCHED == kDense) {
-      return launch_instance<kPairCandidate.bn, kPairCandidate.stages, kPairCandidate.nbuf,
-                             SCHED, true>(ta, tb, p, grid, extra, st, false);
-    }
-    return DG_ERR_INVALID_ARG;
-  }
   switch (bn) {
-    case 256: return launch_instance<256, 4, 2, SCHED, false>(ta, tb, p, grid, extra, st, coop);
-    case 128: return launch_instance<128, 6, 4, SCHED, false>(ta, tb, p, grid, extra, st, coop);
-    case 64: return launch_instance<64, 8, 8, SCHED, false>(ta, tb, p, grid, extra, st, coop);
-    case 32: return launch_instance<32, 8, 8, SCHED, false>(ta, tb, p, grid, extra, st, coop);
-    case 16: return launch_instance<16, 8, 8, SCHED, false>(ta, tb, p, grid, extra, st, coop);
+    case 256: return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st, coop);
+    case 128: return launch_instance<128, 6, 4, SCHED>(ta, tb, p, grid, extra, st, coop);
+    case 64: return launch_instance<64, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
+    case 32: return launch_instance<32, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
+    case 16: return launch_instance<16, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
     default: return DG_ERR_INVALID_ARG;
   }
 }
@@ -1199,7 +1184,6 @@ size_t split_ws_bytes(int64_t tiles, int splits, int bn) {
 
 struct Choice {
   int bn, splits;
-  bool pair;
   int64_t full_tiles;  // dense: tiles computed whole; the rest are split
 };
 
@@ -1217,20 +1201,17 @@ double estimate_tail(int64_t waves, int64_t k, int bn, int s) {
 // may split only the tiles of a last, partial wave (spreading them over all
 // CTAs).  Either needs a workspace that holds the split tiles' FP32 partials
 // (`ws_bytes`).  Tile forms whose shared memory (with `extra` bytes of
-// masked prefix tables) exceeds `max_smem` are skipped.  The pair form
-// (2-CTA clusters) is opt-in (DG_PAIR=1): on B200 it halves each SM's B
-// traffic but measured no faster than the single-CTA 256-wide tile, both
-// being bound by the TMEM round trip.
+// masked prefix tables) exceeds `max_smem` are skipped.
 Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, int num_sms,
                      size_t ws_bytes, int extra = 0, int max_smem = 232448) {
   const int64_t m_blocks = (rows + BM - 1) / BM;
   const int64_t k_blocks = k / BK;
   const int64_t m_blocks_eff =
       (sched == kMasked || sched == kKGrouped) ? m_blocks * groups : m_blocks;
-  Choice c{128, 1, false, 0};
+  Choice c{128, 1, 0};
   double best = 1e300;
   for (const Candidate &cand : kCandidates) {
-    if (config_smem(cand.bn, false, extra, sched) > max_smem) continue;
+    if (config_smem(cand.bn, extra, sched) > max_smem) continue;
     const int64_t tiles = m_blocks * ((n + cand.bn - 1) / cand.bn);
     for (int s = 1; s <= 16; ++s) {
       if (s > 1 && (sched != kDense || m_blocks > 2)) break;
@@ -1240,7 +1221,7 @@ Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, 
       const double e = estimate(m_blocks_eff, n, k, cand.bn, s, num_sms);
       if (e < best * 0.97) {
         best = e;
-        c = {cand.bn, s, false, 0};
+        c = {cand.bn, s, 0};
       }
     }
     if (sched == kDense && m_blocks > 2) {
@@ -1251,7 +1232,7 @@ Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, 
         const double e = std::max(estimate_tail(waves, k, cand.bn, s), bytes / (23.0 * num_sms));
         if (e < best * 0.97) {
           best = e;
-          c = {cand.bn, s, false, waves * num_sms};
+          c = {cand.bn, s, waves * num_sms};
         }
       }
     }
@@ -1270,8 +1251,55 @@ size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int num_sms) {
   return (split_ws_bytes(tiles, c.splits, c.bn) + 255) & ~static_cast<size_t>(255);
 }
 
+// Test knobs of the abort path (both unset in normal use):
+// DG_TEST_STARVE_LOAD=i makes CTA 0's producer leave out the loads of its
+// iteration i, DG_TEST_WAIT_LIMIT_US=t lowers every wait's limit to t
+// microseconds.  They are written to the device before this call's kernel and
+// put back after it, in stream order.
+struct TestKnobs {
+  bool on = false;
+  int starve = -1;
+  unsigned long long limit_ns = kWaitLimitNs;
+};
+
+static TestKnobs test_knobs() {
+  TestKnobs k;
+  if (const char *e = getenv("DG_TEST_STARVE_LOAD")) {
+    k.on = true;
+    k.starve = atoi(e);
+  }
+  if (const char *e = getenv("DG_TEST_WAIT_LIMIT_US")) {
+    k.on = true;
+    k.limit_ns = strtoull(e, nullptr, 10) * 1000ull;
+  }
+  return k;
+}
+
+static int set_test_knobs(const TestKnobs &k, cudaStream_t stream) {
+  if (cudaMemcpyToSymbolAsync(g_starve_load_it, &k.starve, sizeof(int), 0,
+                              cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyToSymbolAsync(g_wait_limit_ns, &k.limit_ns, sizeof(k.limit_ns), 0,
+                              cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return DG_ERR_CUDA;
+  return DG_OK;
+}
+
+static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
+                         cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws);
+
 int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
                     cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws) {
+  const TestKnobs knobs = test_knobs();
+  if (!knobs.on) return launch_fp8_gemm_impl(sched, A, B, p, stream, num_sms, ws_bytes, ws);
+  int rc = set_test_knobs(knobs, stream);
+  if (rc) return rc;
+  rc = launch_fp8_gemm_impl(sched, A, B, p, stream, num_sms, ws_bytes, ws);
+  const int rc2 = set_test_knobs(TestKnobs{}, stream);
+  return rc ? rc : rc2;
+}
+
+static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
+                         cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws) {
   const int64_t rows = p.rows, n = p.n, k = p.k;
   p.num_k_blocks = static_cast<int>(k / BK);
   if (ws == nullptr) ws_bytes = 0;
@@ -1285,34 +1313,19 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   const Choice choice =
       choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes, extra, max_smem);
   int bn = choice.bn, splits = choice.splits;
-  bool pair = choice.pair;
   int64_t full_tiles = choice.full_tiles;
   bool splits_forced = false;  // DG_SPLITS: exactly this many, or none
   // D = C + A B^T (dense only): single-CTA tiles, splits through the
   // workspace (the FP32 tile is staged in the 32 KB the BF16 tile uses, so
   // every tile form still fits)
   const bool acc = p.c != nullptr;
-  // Tuning / test overrides: DG_PAIR=0/1 disables / forces the pair form
-  // (dense only), DG_BLOCK_N forces the N tile of the single-CTA form,
-  // DG_SPLITS splits every tile's K, DG_TAIL_SPLITS only the last partial
-  // wave's tiles (dense, single-CTA; both need enough workspace).
-  if (const char *e = getenv("DG_PAIR")) {
-    if (*e == '0') {
-      if (pair) {
-        pair = false;
-        bn = 256;
-      }
-    } else if (*e == '1' && sched == kDense && !acc && num_sms >= 2) {
-      pair = true;
-      bn = kPairCandidate.bn;
-      splits = 1;
-      full_tiles = 0;
-    }
-  }
+  // Tuning / test overrides: DG_BLOCK_N forces the N tile, DG_SPLITS splits
+  // every tile's K, DG_TAIL_SPLITS only the last partial wave's tiles (dense;
+  // both need enough workspace).
   if (const char *e = getenv("DG_BLOCK_N")) {
     const int v = atoi(e);
     for (const Candidate &c : kCandidates)
-      if (c.bn == v && !pair && v != bn) {
+      if (c.bn == v && v != bn) {
         bn = v;
         splits = 1;  // the split chosen for another width does not carry over
         full_tiles = 0;
@@ -1321,7 +1334,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   if (const char *e = getenv("DG_SPLITS")) {
     // every tile split v ways (v = 1: no split)
     const int v = atoi(e);
-    if (v >= 1 && !pair) {
+    if (v >= 1) {
       const int64_t tiles = ((rows + BM - 1) / BM) * ((n + bn - 1) / bn);
       if (v > 1 && (sched != kDense || ws == nullptr || split_ws_bytes(tiles, v, bn) > ws_bytes ||
                     v > p.num_k_blocks))
@@ -1335,7 +1348,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   if (const char *e = getenv("DG_TAIL_SPLITS")) {
     // the tiles of a partial last wave split v ways, after whole waves
     const int v = atoi(e);
-    if (v >= 2 && !pair && sched == kDense) {
+    if (v >= 2 && sched == kDense) {
       const int64_t tiles = ((rows + BM - 1) / BM) * ((n + bn - 1) / bn);
       const int64_t waves = tiles / num_sms, tail = tiles % num_sms;
       if (waves == 0 || tail == 0 || tail * v > num_sms || v > p.num_k_blocks)
@@ -1345,11 +1358,9 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
       full_tiles = waves * num_sms;
     }
   }
-  if (config_smem(bn, pair, extra, pair ? kDense : (sched == kDense && acc ? kDenseAcc : sched)) >
-      max_smem)
+  if (config_smem(bn, extra, sched == kDense && acc ? kDenseAcc : sched) > max_smem)
     return DG_ERR_INVALID_ARG;  // too many experts
-  const int tile_rows = pair ? 2 * BM : BM;
-  p.num_m_blocks = static_cast<int>((rows + tile_rows - 1) / tile_rows);
+  p.num_m_blocks = static_cast<int>((rows + BM - 1) / BM);
   p.num_n_blocks = static_cast<int>((n + bn - 1) / bn);
   p.splits = splits;
   p.full_tiles = splits > 1 ? static_cast<int>(full_tiles) : 0;
@@ -1360,7 +1371,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   // form a cluster and reduce through distributed shared memory, needing no
   // workspace or arrival counters, when all clusters fit in one wave
   // (DG_CLUSTER_SPLIT=0 forces the workspace path).
-  bool try_cluster = sched == kDense && !acc && !pair && splits > 1 && splits <= 8 &&
+  bool try_cluster = sched == kDense && !acc && splits > 1 && splits <= 8 &&
                      p.full_tiles == 0 && all_tiles * splits <= num_sms;
   if (const char *e = getenv("DG_CLUSTER_SPLIT"))
     if (*e == '0') try_cluster = false;
@@ -1383,11 +1394,10 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
 
   // ------------------------------------------------ tensor maps
   CUtensorMap ta, tb;
-  p.a_box_rows = (sched == kDense && !pair && rows <= BM / 2) ? BM / 2 : BM;
+  p.a_box_rows = (sched == kDense && rows <= BM / 2) ? BM / 2 : BM;
   int rc = make_tmap(&ta, A, k, rows, sched == kMasked ? p.groups : 1, p.a_box_rows);
   if (rc) return rc;
-  rc = make_tmap(&tb, B, k, n, (sched == kDense || sched == kKGrouped) ? 1 : p.groups,
-                 pair ? bn / 2 : bn);
+  rc = make_tmap(&tb, B, k, n, (sched == kDense || sched == kKGrouped) ? 1 : p.groups, bn);
   if (rc) return rc;
 
   // ------------------------------------------------ grid
@@ -1401,12 +1411,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   } else {
     units = p.full_tiles + (all_tiles - p.full_tiles) * splits;
   }
-  int grid;
-  if (pair) {
-    grid = 2 * static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms / 2)));
-  } else {
-    grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
-  }
+  int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
   if (try_cluster) {
     // the chosen split, else (unless forced) fewer splits while the grid
     // still keeps 3/5 of the SMs busy
@@ -1417,7 +1422,7 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
       if (sc < chosen && all_tiles * sc * 5 < static_cast<int64_t>(num_sms) * 3) break;
       p.splits = sc;
       grid = static_cast<int>(all_tiles * sc);
-      rc = dispatch<kDenseCluster>(bn, false, ta, tb, p, grid, extra, stream);
+      rc = dispatch<kDenseCluster>(bn, ta, tb, p, grid, extra, stream);
     }
     if (rc == kClusterNoFit) {
       p.splits = chosen;
@@ -1437,19 +1442,19 @@ int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
   }
   if (print_configs()) {
     fprintf(stderr,
-            "[dg] gemm sched=%d rows=%lld n=%lld k=%lld groups=%d: %s BN=%d splits=%d "
+            "[dg] gemm sched=%d rows=%lld n=%lld k=%lld groups=%d: BN=%d splits=%d "
             "whole=%d grid=%d units=%lld\n",
             sched, static_cast<long long>(rows), static_cast<long long>(n),
-            static_cast<long long>(k), p.groups, pair ? "pair" : "single", bn, splits,
+            static_cast<long long>(k), p.groups, bn, splits,
             p.full_tiles, grid, static_cast<long long>(units));
   }
   switch (sched) {
     case kDense:
-      return acc ? dispatch<kDenseAcc>(bn, false, ta, tb, p, grid, extra, stream)
-                 : dispatch<kDense>(bn, pair, ta, tb, p, grid, extra, stream);
-    case kContiguous: return dispatch<kContiguous>(bn, false, ta, tb, p, grid, extra, stream);
-    case kMasked: return dispatch<kMasked>(bn, false, ta, tb, p, grid, extra, stream);
-    case kKGrouped: return dispatch<kKGrouped>(bn, false, ta, tb, p, grid, extra, stream);
+      return acc ? dispatch<kDenseAcc>(bn, ta, tb, p, grid, extra, stream)
+                 : dispatch<kDense>(bn, ta, tb, p, grid, extra, stream);
+    case kContiguous: return dispatch<kContiguous>(bn, ta, tb, p, grid, extra, stream);
+    case kMasked: return dispatch<kMasked>(bn, ta, tb, p, grid, extra, stream);
+    case kKGrouped: return dispatch<kKGrouped>(bn, ta, tb, p, grid, extra, stream);
     default: return DG_ERR_INVALID_ARG;
   }
 }

@@ -2,7 +2,7 @@
 // mbarriers (with bounded waits), TMA tensor loads, and the tcgen05 family
 // (TMEM allocation, MMA issue, commit, TMEM loads, fences).
 //
-// Every wait in this library is bounded: it gives up after kWaitLimitNs of
+// Every wait in this library is bounded: it gives up after g_wait_limit_ns of
 // %globaltimer, records DG_ERR_TIMEOUT in the device status word and returns
 // false so that the caller can leave its loop and let the CTA exit cleanly.
 #pragma once
@@ -20,6 +20,11 @@ __device__ __forceinline__ void record_status(int *status, int code) {
 
 // Two seconds: far above any legitimate wait inside one kernel.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// The limit every bounded wait of a kernel compiled in this translation unit
+// applies (one copy per translation unit).  Its host side may lower it for a
+// test that starves a wait on purpose, so that the wait runs out quickly.
+static __device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -78,8 +83,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false (and
-// records DG_ERR_TIMEOUT in *status) after kWaitLimitNs, or soon after *abort
-// is set by another role of the CTA that already gave up.
+// records DG_ERR_TIMEOUT in *status) after g_wait_limit_ns, or soon after
+// *abort is set by another role of the CTA that already gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int *abort, int *status) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -89,7 +94,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > g_wait_limit_ns) {
       record_status(status, DG_ERR_TIMEOUT);
       *abort = 1;
       return false;
@@ -104,14 +109,14 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
 }
 
 // Spins until *counter >= target (acquire).  Returns false, recording
-// DG_ERR_TIMEOUT, after kWaitLimitNs.
+// DG_ERR_TIMEOUT, after g_wait_limit_ns.
 __device__ __forceinline__ bool wait_counter(const uint32_t *counter, uint32_t target,
                                              int *status) {
   if (ld_acquire_gpu(counter) >= target) return true;
   const uint64_t t0 = globaltimer();
   while (ld_acquire_gpu(counter) < target) {
     __nanosleep(64);
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > g_wait_limit_ns) {
       record_status(status, DG_ERR_TIMEOUT);
       return false;
     }
@@ -214,6 +219,22 @@ __device__ __forceinline__ void ffma2v(float &a0, float &a1, float x0, float x1,
       "mov.b64 {%0, %1}, d;\n\t}"
       : "+f"(a0), "+f"(a1)
       : "f"(x0), "f"(x1), "f"(s0), "f"(s1));
+}
+
+// ------------------------------------------------------------------ registers
+// Warp-specialised register split: a warpgroup lowers (dec) or raises (inc)
+// its per-thread register count.  All four warps of a warpgroup execute the
+// same instruction; an inc waits until the registers it asks for have been
+// released by dec's of other warpgroups, so the split must fit the block's
+// launch allocation (threads x registers per thread at launch).
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -333,9 +354,9 @@ __device__ __forceinline__ void reg_barrier(uint32_t *r) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i])::"memory");
 }
 
-// ------------------------------------------------------------------ CTA pairs
-// The pair form: two CTAs of a 2-CTA cluster (ranks 0 and 1) run one
-// cta_group::2 MMA of M = 256; rank 0 issues it.
+// ------------------------------------------------------------------ clusters
+// The split-K cluster reduction: the CTAs of a thread-block cluster read each
+// other's shared memory (distributed shared memory).
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -366,75 +387,6 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr) {
                : "r"(addr)
                : "memory");
   return v;
-}
-
-// Arrive on an mbarrier given by its cluster-window address (possibly in the
-// peer CTA).  Default (release, CTA-scope) semantics: the arrive only has to
-// follow this thread's completed TMEM reads, which tcgen05.wait::ld and
-// tcgen05.fence::before_thread_sync already order; a cluster-scope release
-// would add a full fence to the promotion's critical path.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
-// 3-D TMA load into this CTA's shared memory whose completion is counted on
-// an mbarrier of either CTA of the pair (`bar` is a cluster-window address).
-__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void *tmap,
-                                                 uint32_t bar, int32_t c0,
-                                                 int32_t c1, int32_t c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::"
-      "complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
-  asm volatile(
-      "tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-          dst),
-      "r"(ncols)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::
-                   : "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile(
-      "tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr),
-      "r"(ncols)
-      : "memory");
-}
-
-// D[tmem of both CTAs] (+)= A * B^T with M = 256: rows 0-127 of A and D in
-// rank 0, rows 128-255 in rank 1; B split along N between the two CTAs'
-// shared memory at the same offsets.  Issued by one thread of rank 0.
-__device__ __forceinline__ void umma_f8_pair(uint32_t d_tmem, uint64_t a_desc,
-                                             uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  const uint32_t z = 0;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, "
-      "%8, %9, %10, %11, %12}, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z),
-      "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z)
-      : "memory");
-}
-
-// Arrives once on the mbarrier at cluster-window address `bar` (this CTA's or
-// the peer's) when all tcgen05 operations issued so far by this thread have
-// completed.  Pair form; one call per target barrier.
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 "
-      "[%0];" ::"r"(bar)
-      : "memory");
 }
 
 // ------------------------------------------------------------------ UMMA descriptors
