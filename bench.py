@@ -7,9 +7,14 @@ One step = one pass of the whole hot path over one batch of synthetic input:
 for every (N, K) pair of the workload, quantize the FP32 activations A with the
 1x128 quantizer kernel, then run the FP8 GEMM against the pre-quantized
 (128x128) weights B.  Weights are quantized once before timing (they are
-offline-quantized model parameters).  The default workload is the dense
+offline-quantized model parameters).  The headline workload is the dense
 prefill set: M = 4096 and (N, K) in {(7168, 16384), (4096, 7168),
-(24576, 1536), (2112, 7168)}.
+(24576, 1536), (2112, 7168)}.  By default every workload of the metric is
+measured, one after the other: prefill (the line's value), decode at M = 64
+and 128, the contiguous and masked MoE layouts, the masked layout with
+power-of-two scales, the k-grouped weight gradient and D = C + A B^T; each
+of the others is listed under config.workloads with its own roofline,
+end-to-end rate and oracle sample.  ``--workload W`` measures one.
 
 Reported (one JSON line on rank 0):
 * value       whole-job TFLOP/s (2 M N K per GEMM, summed over shapes and
@@ -147,6 +152,11 @@ def workload_spec(name: str) -> dict:
         return dict(name=name, kind="masked", bound="hbm", **inputs.MASKED,
                     desc="m-grouped masked, G=32, M_max=256, N=7168 K=2048, "
                          "masked_m ~ U{0..256}")
+    if name == "masked_pow2":
+        return dict(name=name, kind="masked", bound="hbm", pow2=True, **inputs.MASKED,
+                    desc="m-grouped masked, G=32, M_max=256, N=7168 K=2048, "
+                         "masked_m ~ U{0..256}, every scale rounded up to a power of two "
+                         "(UE8M0-representable)")
     if name == "kgrouped":
         return dict(name=name, kind="kgrouped", bound="tensor", **inputs.K_GROUPED,
                     desc="k-grouped contiguous (MoE weight gradient), G=8, M=4096 N=7168, "
@@ -392,12 +402,13 @@ class GroupedData(DenseData):
             self.rows_total = lay.m_total
         w = inputs.weights((G, n, k), seed=spec["seed"] + 2)
         a32 = torch.from_numpy(x).to(device)
-        qb, sfb = dg.dg_quantize_128x128(torch.from_numpy(w).to(device))
+        self.pow2 = bool(spec.get("pow2"))
+        qb, sfb = dg.dg_quantize_128x128(torch.from_numpy(w).to(device), pow2=self.pow2)
         # host inputs for the oracle's timed sample (a few experts' rows and
         # the first columns of their weights)
         self.sample_src = GroupedOracleSample.source(spec, x, w, index.cpu().numpy())
         del w
-        qa, sfa = dg.dg_quantize_1x128(a32)
+        qa, sfa = dg.dg_quantize_1x128(a32, pow2=self.pow2)
         d = torch.empty(d_shape, dtype=torch.bfloat16, device=device)
         self.m = rows_valid
         self.active = active
@@ -423,6 +434,12 @@ class GroupedData(DenseData):
             self.dg.dg_m_grouped_fp8_gemm_nt_contiguous(s["qa"], s["sfa"], s["qb"], s["sfb"],
                                                         s["d"], s["index"])
 
+    def step(self):
+        """One pass of the hot path: quantize the activations, then GEMM."""
+        s = self.shapes[0]
+        self.dg.dg_quantize_1x128(s["a32"], pow2=self.pow2, q=s["qa"], sf=s["sfa"])
+        self.gemm(s)
+
     def make_host(self):
         s = self.shapes[0]
         self.host = [dict(a=torch_pin(s["x_host"]), qb=s["qb"].cpu().pin_memory(),
@@ -439,7 +456,7 @@ class GroupedData(DenseData):
         qb = h["qb"].to(device, non_blocking=True)
         sfb = h["sfb"].to(device, non_blocking=True)
         index = h["index"].to(device, non_blocking=True)
-        qa, sfa = self.dg.dg_quantize_1x128(a)
+        qa, sfa = self.dg.dg_quantize_1x128(a, pow2=self.pow2)
         if self.kind == "masked":
             self.dg.dg_m_grouped_fp8_gemm_nt_masked(qa, sfa, qb, sfb, s["d"], index)
         else:
@@ -618,12 +635,13 @@ class GroupedOracleSample:
         from oracle import quant as oq
         self.kind = spec["kind"]
         self.k = spec["k"]
+        self.pow2 = bool(spec.get("pow2"))
         if src is None:
             src = self.source(spec, *self._generate(spec))
         self.prepared = []
         for xr, wc in src:
             xr, wc = xr[:rows], wc[:cols]
-            qb, beta = oq.quantize_128x128(wc)
+            qb, beta = oq.quantize_128x128(wc, pow2=self.pow2)
             self.prepared.append((xr, qb, beta))
         c = min(cols, spec["n"])
         self.desc = (f"{rows} rows of each of the first {len(self.prepared)} experts with rows "
@@ -646,7 +664,7 @@ class GroupedOracleSample:
         """Returns (seconds, FLOPs) of one pass."""
         from oracle import gemm as og, quant as oq
         t0 = time.perf_counter()
-        qas = [oq.quantize_1x128(xr) for xr, _, _ in self.prepared]
+        qas = [oq.quantize_1x128(xr, pow2=self.pow2) for xr, _, _ in self.prepared]
         qb = np.stack([q for _, q, _ in self.prepared])
         beta = np.stack([b for _, _, b in self.prepared])
         n_rows = [len(xr) for xr, _, _ in self.prepared]
@@ -744,7 +762,8 @@ def run_reference(args, rank: int) -> None:
     """The oracle arm: rank 0 times the CPU oracle on bounded samples."""
     if rank != 0:
         return
-    spec = workload_spec(args.workload)
+    # the headline workload when all are measured
+    spec = workload_spec("prefill" if args.workload == "all" else args.workload)
     sampler = make_sampler(spec, args.ref_rows, args.ref_cols)
     for _ in range(args.warmup):
         sampler.run()
@@ -787,16 +806,20 @@ def job_throughput(work_per_step: float, steps: int, world: int, ms: float) -> f
     return work_per_step * steps * world / (ms * 1e-3)
 
 
-def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
+ALL_WORKLOADS = ["prefill", "decode64", "decode128", "contiguous", "masked", "masked_pow2",
+                 "kgrouped", "prefill_acc"]
+
+
+def measure_workload(name: str, args, rank: int, world: int, device, cpu_secs: float) -> dict:
+    """Times one workload on this rank and returns its bench fields (rank 0's
+    are the ones printed): whole-step throughput from CUDA-graph replays, the
+    GEMM kernel alone against its roofline, the end-to-end rate from pinned
+    host buffers, and the oracle on a bounded sample of the same work (rank 0,
+    N = 1 only, about ``cpu_secs`` of CPU time)."""
     import torch
     import torch.distributed as dist
 
-    import moe_grouped_gemm_act_b200 as dg
-
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    dg.load_library()
-    spec = workload_spec(args.workload)
+    spec = workload_spec(name)
     data = {"dense": DenseData, "kgrouped": KGroupedData}.get(spec["kind"], GroupedData)(
         spec, device)
 
@@ -811,7 +834,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     data.capture()
     nshape = len(data.shapes)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clocks:
+    with ClockSampler(device.index or 0) as clocks:
         for _ in range(args.warmup):
             data.step_graph.replay()
         barrier()
@@ -838,7 +861,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             ev[j][i][1].record()
     torch.cuda.synchronize()
     per_shape_ms = [statistics.mean(a.elapsed_time(b) for a, b in ev[j]) for j in range(nshape)]
-    gemm_ms = [sum(per_shape_ms)] * args.steps
+    gemm_ms = sum(per_shape_ms) * args.steps
 
     # ------------------------------------------------ end-to-end timing
     data.make_host()
@@ -857,10 +880,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     e2e_ms = e0.elapsed_time(e1) * args.steps / e2e_steps
 
     # ------------------------------------------------ max over ranks
-    total_ms, e2e_ms, gemm_total_ms = max_over_ranks([total_ms, e2e_ms, sum(gemm_ms)], world,
-                                                     device)
-    if rank != 0:
-        return
+    total_ms, e2e_ms, gemm_total_ms = max_over_ranks([total_ms, e2e_ms, gemm_ms], world, device)
 
     flops_step = data.flops()
     value = job_throughput(flops_step, args.steps, world, total_ms) / 1e12
@@ -878,28 +898,28 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         peak = pk["hbm"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{pk['source']} copy bandwidth"}
-    roof["traffic"] = args.traffic if args.traffic is not None else measured_traffic(args.workload)
+    roof["traffic"] = (args.traffic if args.traffic is not None and args.workload == name
+                       else measured_traffic(name))
     roof["traffic_unit"] = "bytes per GEMM launch (ncu dram read + write)"
     per_shape = per_shape_report(data, per_shape_ms, spec["bound"], peak)
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and cpu_secs > 0:
         sampler = make_sampler(spec, args.ref_rows, args.ref_cols, data)
         sampler.run()
         secs, fl = 0.0, 0.0
-        while secs < 10.0:          # about 10 s of CPU work
+        while secs < cpu_secs:
             s_, f_ = sampler.run()
             secs += s_
             fl += f_
         cpu = {"value": fl / secs / 1e12, "unit": "TFLOPS", "cores": blas_threads(),
                "kind": "oracle", "sample": f"{sampler.desc} ({secs:.1f} s on the host)"}
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3", "data": "synthetic",
-        "config": {"workload": spec["desc"], "valid_rows" if spec["kind"] in ("contiguous", "masked") else "m": data.m,
-                   "nk": [[s["n"], s["k"]] for s in data.shapes],
+    out = {
+        "workload": name, "desc": spec["desc"], "value": value, "unit": "TFLOPS",
+        "ms_per_step": total_ms / args.steps,
+        "config": {"workload": spec["desc"],
+                   "valid_rows" if spec["kind"] in ("contiguous", "masked") else "m": data.m,
+                   "nk": [[sh["n"], sh["k"]] for sh in data.shapes],
                    "l2": "not flushed: each step streams %.0f MB of inputs (> 126 MB L2)"
                          % (data.input_bytes() / 1e6),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -911,6 +931,46 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         "gpu_launches": data.launches_per_step() * args.steps,
         "clocks": clocks.summary(),
     }
+    del data
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+
+    import moe_grouped_gemm_act_b200 as dg
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dg.load_library()
+    names = ALL_WORKLOADS if args.workload == "all" else [args.workload]
+    cpu_secs = 0.0 if args.no_cpu_baseline else 10.0
+    results = []
+    for i, name in enumerate(names):
+        # the headline workload gets about 10 s of oracle time, the others 3 s
+        results.append(measure_workload(name, args, rank, world, device,
+                                        cpu_secs if i == 0 else min(cpu_secs, 3.0)))
+    if rank != 0:
+        return
+    head = results[0]
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3", "data": "synthetic",
+        "config": dict(head["config"]),
+        "roofline": head["roofline"],
+        "cpu_baseline": head["cpu_baseline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+    }
+    if len(results) > 1:
+        # every other workload of the metric, each with its own roofline,
+        # end-to-end rate, oracle sample and clocks
+        line["config"]["workloads"] = results[1:]
     print(json.dumps(line))
 
 
@@ -919,9 +979,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="prefill",
-                    choices=["prefill", "prefill_acc", "decode64", "decode128", "contiguous",
-                             "masked", "kgrouped"])
+    ap.add_argument("--workload", default="all", choices=["all", *ALL_WORKLOADS],
+                    help="one workload, or all of them (the default: the line's value is the "
+                         "prefill workload's, the others are listed under config.workloads)")
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--ref-rows", type=int, default=16,
                     help="rows of A per shape in the oracle's timed sample")

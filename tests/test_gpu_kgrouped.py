@@ -164,3 +164,44 @@ def test_host_argument_checks(cuda_device):
     assert call(M=0) == dg.DG_OK
     torch.cuda.synchronize()
     assert dg.dg_get_device_status() == dg.DG_OK
+
+
+def test_bench_size_sampled(cuda_device):
+    # the bench's weight-gradient workload at full size (8 experts, M 4096,
+    # N 7168, 32768 tokens along K, padding tokens zero), operands quantized on
+    # the device as the bench does; every D[g] compared on the first and last
+    # row of each 128-row tile and the first and last column of each 128-column
+    # block, plus random rows and columns
+    c = inputs.K_GROUPED
+    lay = inputs.k_grouped_layout(c["tokens"], c["groups"], seed=c["seed"])
+    a = inputs.activations(c["m"], lay.k_total, seed=c["seed"] + 1, outliers=True)
+    b = inputs.activations(c["n"], lay.k_total, seed=c["seed"] + 2)
+    valid = np.zeros(lay.k_total, bool)
+    start = 0
+    for cnt, size in zip(lay.counts, lay.k_sizes):
+        valid[start:start + int(cnt)] = True
+        start += int(size)
+    a[:, ~valid] = 0.0
+    b[:, ~valid] = 0.0
+    qa_d, sfa_d = dg.dg_quantize_1x128(torch.from_numpy(a).cuda())
+    qb_d, sfb_d = dg.dg_quantize_1x128(torch.from_numpy(b).cuda())
+    ks = dev(lay.k_sizes)
+    g_count, m, n = c["groups"], c["m"], c["n"]
+    d = torch.full((g_count, m, n), float("nan"), dtype=torch.float32, device="cuda")
+    dg.dg_k_grouped_fp8_gemm_nt_contiguous(qa_d, sfa_d, qb_d, sfb_d, d, ks)
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == dg.DG_OK
+    rng = np.random.default_rng(9)
+
+    def pick(size):
+        idx = [i for t in range(0, size, 128) for i in (t, min(t + 127, size - 1))]
+        return np.array(sorted(set(idx) | set(rng.choice(size, 32, replace=False).tolist())))
+
+    rows, cols = pick(m), pick(n)
+    qa, alpha = quant.quantize_1x128(a[rows])
+    qb, beta = quant.quantize_1x128(b[cols])
+    assert np.array_equal(qa_d.cpu().numpy()[rows], qa)
+    want = gemm.k_grouped_contiguous_f64(qa, alpha, qb, beta, lay.k_sizes)
+    got = d.cpu().numpy()[:, rows][:, :, cols]
+    for g in range(g_count):
+        check_f32(got[g], want[g], f"k-grouped bench size group {g}")
