@@ -70,6 +70,51 @@ def fp8_gemm_nt_f64(qa: np.ndarray, alpha: np.ndarray,
     return d
 
 
+def fp8_gemm_nt_rowscaled_f64(qa: np.ndarray, alpha: np.ndarray,
+                              qb: np.ndarray, beta_rows: np.ndarray) -> np.ndarray:
+    """float64 D [M, N] of the Fig. 13-1 formula with one scale per row of B
+    and 128-wide K group, beta_rows float [N, K/128], instead of one per
+    128 x 128 block (the scaling Fig. 13-1 gives A, applied to both operands;
+    a 128 x 128 block scale is the special case in which the 128 rows of a
+    block share their values).  alpha float [M, K/128] as in fp8_gemm_nt_f64.
+    Same order: per 128-wide K block, the block's partial product of the
+    decoded codes times the outer product of the block's scales, added in
+    float64."""
+    M, K = qa.shape
+    N, Kb = qb.shape
+    if K != Kb or K % GROUP:
+        raise ValueError("K mismatch or K not a multiple of 128")
+    kg = K // GROUP
+    if alpha.shape != (M, kg) or beta_rows.shape != (N, kg):
+        raise ValueError("scale shapes do not match the 1x128 grids of A and B")
+    a_vals = e4m3.decode(qa)
+    b_vals = e4m3.decode(qb)
+    alpha64 = np.asarray(alpha, np.float64)
+    beta64 = np.asarray(beta_rows, np.float64)
+    d = np.zeros((M, N), dtype=np.float64)
+    for g in range(kg):
+        ks = slice(g * GROUP, (g + 1) * GROUP)
+        d += (a_vals[:, ks] @ b_vals[:, ks].T) * (alpha64[:, g][:, None] * beta64[:, g][None, :])
+    return d
+
+
+def fp8_gemm_nt_ue8m0_f64(qa, sfa_packed, qb, sfb_packed) -> np.ndarray:
+    """float64 D [M, N] of the block-scaled GEMM whose scales are UE8M0 codes
+    in the packed layout (Lesson 13, Fig. 13-1 text: newer versions take
+    UE8M0 scales; Deep dive, section 3: four per 32-bit word, MN-major):
+    sfa_packed int32 [ceil(K/512), ld_a >= M] for the rows of A,
+    sfb_packed int32 [ceil(K/512), ld_b >= N] for the rows of B.  The codes
+    are decoded to their powers of two and the formula is evaluated as in
+    fp8_gemm_nt_rowscaled_f64."""
+    from . import ue8m0
+    M, K = qa.shape
+    N = qb.shape[0]
+    kg = K // GROUP
+    alpha = ue8m0.unpack_1x128(sfa_packed, M, kg)
+    beta_rows = ue8m0.unpack_1x128(sfb_packed, N, kg)
+    return fp8_gemm_nt_rowscaled_f64(qa, alpha, qb, beta_rows)
+
+
 def fp8_gemm_nt(qa, alpha, qb, beta) -> np.ndarray:
     """BF16 bit patterns (uint16 [M, N]) of the dense NT GEMM."""
     return bf16.to_bits(fp8_gemm_nt_f64(qa, alpha, qb, beta))

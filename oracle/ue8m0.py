@@ -68,3 +68,19 @@ def pack_1x128(alpha: np.ndarray) -> np.ndarray:
             if g < kg:
                 out[p] += codes[:, g].astype(np.int64) * (256 ** t)
     return out.astype(np.uint32).view(np.int32)
+
+
+def unpack_1x128(packed: np.ndarray, m: int, kg: int) -> np.ndarray:
+    """float64 scales [m, kg] (row i, group g) of the packed layout: the
+    inverse of ``pack_1x128`` on the first m rows of each word row (the
+    columns past m of a TMA-aligned ld are ignored)."""
+    words = np.asarray(packed).view(np.uint32).astype(np.int64)
+    if words.ndim != 2 or words.shape[0] != -(-kg // GROUPS_PER_WORD) or words.shape[1] < m:
+        raise ValueError("packed scales must be [ceil(kg/4), ld >= m]")
+    codes = np.zeros((m, kg), np.int64)
+    for g in range(kg):
+        p, t = divmod(g, GROUPS_PER_WORD)
+        codes[:, g] = (words[p, :m] >> (8 * t)) & 0xFF
+    out = decode(codes)
+    out[codes == 0] = 0.0   # code 0 stands for an all-zero group (scale +0)
+    return out

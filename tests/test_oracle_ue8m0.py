@@ -14,7 +14,7 @@ MN-major.  Pinned against:
 import numpy as np
 import pytest
 
-from oracle import quant, ue8m0
+from oracle import e4m3, gemm, quant, ue8m0
 from moe_grouped_gemm_act_b200 import inputs
 
 
@@ -99,3 +99,58 @@ def test_planted_layout_mistakes_are_caught(mutant):
                      [0x00000075, 0x00000000]], np.uint32)
     got = mutant(alpha).view(np.uint32)
     assert got.shape != want.shape or not np.array_equal(got, want)
+
+
+# ------------------------------------------------ unpacking and the UE8M0 GEMM
+def test_unpack_inverts_pack_including_zero_groups():
+    rng = np.random.default_rng(11)
+    for m, kg in [(5, 1), (130, 7), (64, 16)]:
+        sf = np.ldexp(1.0, rng.integers(-20, 21, size=(m, kg))).astype(np.float32)
+        sf[rng.random((m, kg)) < 0.1] = 0.0
+        packed = ue8m0.pack_1x128(sf)
+        wide = np.zeros((packed.shape[0], m + 3), np.int32)   # a TMA-aligned ld
+        wide[:, :m] = packed
+        assert np.array_equal(ue8m0.unpack_1x128(wide, m, kg), sf.astype(np.float64))
+
+
+def _pow2_case(m, n, k, seed):
+    x = inputs.activations(m, k, seed=seed, outliers=True)
+    w = inputs.weights((n, k), seed=seed + 1)
+    qa, alpha = quant.quantize_1x128(x, pow2=True)
+    qb, beta = quant.quantize_128x128(w, pow2=True)
+    return qa, alpha, qb, beta
+
+
+def test_ue8m0_gemm_with_block_scales_is_the_dense_oracle():
+    # B's 128 x 128 block scales written out per row (each row of a block
+    # carries its block's codes): the packed-code GEMM must reproduce the
+    # pinned Fig. 13-1 oracle exactly (same float64 operations)
+    qa, alpha, qb, beta = _pow2_case(150, 264, 640, seed=3)
+    beta_rows = beta[np.arange(264) // 128]
+    got = gemm.fp8_gemm_nt_ue8m0_f64(qa, ue8m0.pack_1x128(alpha), qb,
+                                     ue8m0.pack_1x128(beta_rows))
+    assert np.array_equal(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta))
+
+
+def test_rowscaled_gemm_matches_an_elementwise_restatement():
+    # distinct scales on every row of B (not block-constant), brute force
+    rng = np.random.default_rng(5)
+    m, n, k = 3, 5, 256
+    qa = e4m3.encode_rne(rng.integers(-6, 7, size=(m, k)).astype(np.float32))
+    qb = e4m3.encode_rne(rng.integers(-6, 7, size=(n, k)).astype(np.float32))
+    alpha = np.ldexp(1.0, rng.integers(-3, 4, size=(m, 2)))
+    beta = np.ldexp(1.0, rng.integers(-3, 4, size=(n, 2)))
+    a, b = e4m3.decode(qa), e4m3.decode(qb)
+    want = np.zeros((m, n))
+    for i in range(m):
+        for j in range(n):
+            for kk in range(k):
+                want[i, j] += alpha[i, kk // 128] * beta[j, kk // 128] * a[i, kk] * b[j, kk]
+    got = gemm.fp8_gemm_nt_rowscaled_f64(qa, alpha, qb, beta)
+    assert np.allclose(got, want, rtol=1e-12, atol=0)
+    # a mistake in the byte order of the packed words is caught
+    packed = ue8m0.pack_1x128(beta.astype(np.float32))
+    swapped = packed.view(np.uint8).reshape(packed.shape + (4,))[..., ::-1].copy().view(np.int32)
+    swapped = swapped.reshape(packed.shape)
+    bad = gemm.fp8_gemm_nt_ue8m0_f64(qa, ue8m0.pack_1x128(alpha.astype(np.float32)), qb, swapped)
+    assert not np.allclose(bad, want)
