@@ -161,6 +161,27 @@ int dg_pack_ue8m0(const float *sf, int64_t batch, int64_t M, int64_t Kg,
                   dg_stream_t stream);
 
 /*
+ * dg_pack_ue8m0_128x128 -- 128 x 128 block scales of B (Lesson 13, Fig. 13-1)
+ * written out in the packed UE8M0 layout one word row per row of B, the form
+ * the UE8M0 GEMMs read B's scales in (each of the 128 rows of a block repeats
+ * the block's words).
+ *
+ *   sf      device float [G][ceil(N/128)][Kg] row-major, as written by
+ *           dg_quantize_128x128 with DG_SCALE_POW2 (every scale +0 or a
+ *           normal power of two).
+ *   packed  device int32 [G][ceil(Kg/4)][ld_packed]: word (g, p, n) holds
+ *           groups 4p .. 4p+3 of block n/128 of expert g, group 4p+t in bits
+ *           8t .. 8t+7; groups past Kg are zero bytes.  Entries n >= N are not
+ *           written.
+ *   G >= 1, N >= 0 (0 is a no-op), Kg >= 1, ld_packed >= N and % 4 == 0;
+ *   both pointers 16-byte aligned.
+ * Scales UE8M0 cannot hold are recorded as DG_ERR_DEVICE_DATA, as in
+ * dg_pack_ue8m0.  Output is bit-exact.  Memory is caller-owned.
+ */
+int dg_pack_ue8m0_128x128(const float *sf, int64_t G, int64_t N, int64_t Kg,
+                          int32_t *packed, int64_t ld_packed, dg_stream_t stream);
+
+/*
  * dg_fp8_gemm_nt -- dense NT GEMM, D = A * B^T with 1x128 / 128x128 scales
  * (Lesson 13, Fig. 13-1; DeepGEMM launch article: gemm_fp8_fp8_bf16_nt).
  *
@@ -301,6 +322,52 @@ int dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *A, const float *sfa,
                                     const int32_t *masked_m, int G,
                                     int64_t M_max, int64_t N, int64_t K,
                                     dg_stream_t stream);
+
+/*
+ * dg_fp8_gemm_nt_ue8m0 -- dense NT GEMM with power-of-two scales given as
+ * packed UE8M0 codes (Lesson 13, Fig. 13-1 text: newer versions accept UE8M0
+ * scales; Deep dive, section 3: on sm_100 the scales are four UE8M0 values
+ * per 32-bit word, MN-major, TMA-aligned).  The formula is Fig. 13-1's with
+ * alpha = 2^(code_A - 127) per row of A and 128-wide K group and
+ * beta = 2^(code_B - 127) per row of B and K group.  Because every scale is a
+ * power of two, the tensor cores apply them (block-scaled MMA, one scale per
+ * row and 32-wide K slice) and the tile accumulates in FP32 over the whole of
+ * K; there is no per-block promotion on the CUDA cores.  A code of 0 stands
+ * for 2^-127 and may only scale an all-zero group (the quantizer's +0 scale).
+ *
+ *   A      device uint8 [M][K] E4M3, row-major (K-major).
+ *   sfa    device int32 [ceil(K/512)][ld_sfa], the layout dg_pack_ue8m0
+ *          writes: word (p, i) holds K groups 4p .. 4p+3 of row i;
+ *          ld_sfa >= M, % 4 == 0.
+ *   B      device uint8 [N][K] E4M3, row-major (K-major).
+ *   sfb    device int32 [ceil(K/512)][ld_sfb], one word row per row of B
+ *          (dg_pack_ue8m0 of per-row scales, or dg_pack_ue8m0_128x128 of
+ *          128 x 128 block scales); ld_sfb >= N, % 4 == 0.
+ *   D      device BF16 [M][N] row-major, written for all i < M, j < N.
+ *   M >= 0 (0 is a no-op), N > 0 with N % 8 == 0, K > 0 with K % 128 == 0;
+ *   A, B, D, sfa, sfb 16-byte aligned.
+ * No workspace: K is never split.  Deterministic.
+ */
+int dg_fp8_gemm_nt_ue8m0(const uint8_t *A, const int32_t *sfa, int64_t ld_sfa,
+                         const uint8_t *B, const int32_t *sfb, int64_t ld_sfb,
+                         void *D, int64_t M, int64_t N, int64_t K,
+                         dg_stream_t stream);
+
+/*
+ * dg_m_grouped_fp8_gemm_nt_masked_ue8m0 -- the masked MoE GEMM of
+ * dg_m_grouped_fp8_gemm_nt_masked with packed UE8M0 scales as in
+ * dg_fp8_gemm_nt_ue8m0: sfa device int32 [G][ceil(K/512)][ld_sfa]
+ * (ld_sfa >= M_max, % 4 == 0), sfb device int32 [G][ceil(K/512)][ld_sfb]
+ * (ld_sfb >= N, % 4 == 0).  Rows >= masked_m[g] of D are not written;
+ * masked_m outside [0, M_max] is clamped and recorded as DG_ERR_DEVICE_DATA.
+ *   1 <= G <= 1024, M_max >= 1, N % 8 == 0, K % 128 == 0.
+ */
+int dg_m_grouped_fp8_gemm_nt_masked_ue8m0(const uint8_t *A, const int32_t *sfa,
+                                          int64_t ld_sfa, const uint8_t *B,
+                                          const int32_t *sfb, int64_t ld_sfb, void *D,
+                                          const int32_t *masked_m, int G,
+                                          int64_t M_max, int64_t N, int64_t K,
+                                          dg_stream_t stream);
 
 /*
  * dg_k_grouped_fp8_gemm_nt_contiguous -- the K-grouped contiguous GEMM of

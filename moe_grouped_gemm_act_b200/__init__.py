@@ -11,12 +11,16 @@ Entry points (same names as the C ABI):
 * ``dg_quantize_1x128(x, pow2=False)`` -> (q, sf)    1 x 128 E4M3 activations
 * ``dg_quantize_128x128(w, pow2=False)`` -> (q, sf)  128 x 128 E4M3 weights
 * ``dg_pack_ue8m0(sf, m)`` -> packed int32 UE8M0 scales (4 K groups per word)
+* ``dg_pack_ue8m0_128x128(sf, n)`` -> B's 128 x 128 block scales packed per row
 * ``dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace=None)``
 * ``dg_fp8_gemm_nt_accumulate(a, sfa, b, sfb, c, d, workspace=None)``  D = C + A B^T
 * ``dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, d)``
 * ``dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices)``
 * ``dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m)``
 * ``dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, k_sizes, c=None)``
+* ``dg_fp8_gemm_nt_ue8m0(a, sfa, b, sfb, d)``, ``dg_m_grouped_fp8_gemm_nt_masked_ue8m0(
+  a, sfa, b, sfb, d, masked_m)``  power-of-two scales as packed UE8M0 words,
+  applied by the tensor cores
 * ``dg_get_device_status()``, helpers ``dg_get_tma_aligned_size``,
   ``dg_get_mk_alignment_for_contiguous_layout``, ``dg_set_num_sms``,
   ``dg_get_num_sms``, ``dg_fp8_gemm_nt_workspace_size``.
@@ -46,7 +50,8 @@ DG_ERR_TIMEOUT, DG_ERR_DEVICE_DATA = -6, -7
 EXPORTS = [
     "dg_status_string", "dg_get_mk_alignment_for_contiguous_layout",
     "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms",
-    "dg_quantize_1x128", "dg_quantize_128x128", "dg_pack_ue8m0", "dg_fp8_gemm_nt",
+    "dg_quantize_1x128", "dg_quantize_128x128", "dg_pack_ue8m0", "dg_pack_ue8m0_128x128",
+    "dg_fp8_gemm_nt", "dg_fp8_gemm_nt_ue8m0", "dg_m_grouped_fp8_gemm_nt_masked_ue8m0",
     "dg_fp8_gemm_nt_workspace_size", "dg_fp8_gemm_nt_noalloc", "dg_fp8_gemm_nt_accumulate",
     "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_nt_contiguous",
@@ -81,6 +86,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_quantize_1x128": (I, [P, I, I64, I64, I64, I64, P, I64, P, I64, I, P]),
         "dg_quantize_128x128": (I, [P, I64, I64, I64, P, P, I, P]),
         "dg_pack_ue8m0": (I, [P, I64, I64, I64, I64, P, I64, P]),
+        "dg_pack_ue8m0_128x128": (I, [P, I64, I64, I64, P, I64, P]),
+        "dg_fp8_gemm_nt_ue8m0": (I, [P, P, I64, P, P, I64, P, I64, I64, I64, P]),
+        "dg_m_grouped_fp8_gemm_nt_masked_ue8m0":
+            (I, [P, P, I64, P, P, I64, P, P, I, I64, I64, I64, P]),
         "dg_fp8_gemm_nt": (I, [P, P, I64, P, P, P, I64, I64, I64, P, SZ, P]),
         "dg_fp8_gemm_nt_workspace_size": (SZ, [I64, I64, I64]),
         "dg_fp8_gemm_nt_noalloc": (I, [P, P, I64, P, P, P, I64, I64, I64, P]),
@@ -280,6 +289,33 @@ def dg_pack_ue8m0(sf: torch.Tensor, m: int, packed=None, stream=None) -> torch.T
     return packed if batched else packed.view(words, packed.shape[-1])
 
 
+def dg_pack_ue8m0_128x128(sf: torch.Tensor, n: int, packed=None, stream=None) -> torch.Tensor:
+    """B's 128 x 128 block scales sf (float32 power-of-two values,
+    [ceil(n/128), Kg] or [G, ceil(n/128), Kg], as dg_quantize_128x128(pow2=True)
+    returns) written out per row of B in the packed UE8M0 layout: int32
+    [ceil(Kg/4), ld] (or [G, ceil(Kg/4), ld]), ld = dg_get_tma_aligned_size(n,
+    4); word (p, j) holds groups 4p .. 4p+3 of row j's block."""
+    _need_cuda(sf)
+    if sf.dtype != torch.float32:
+        raise ValueError("sf must be float32")
+    grouped = sf.dim() == 3
+    sb = sf if grouped else sf.unsqueeze(0)
+    g, nb, kg = sb.shape
+    if nb != -(-n // 128):
+        raise ValueError(f"sf has {nb} row blocks; n = {n} needs {-(-n // 128)}")
+    words = -(-kg // 4)
+    if packed is None:
+        packed = torch.empty((g, words, dg_get_tma_aligned_size(n, 4)), dtype=torch.int32,
+                             device=sf.device)
+    _need_cuda(packed)
+    _expect(packed if packed.dim() == 3 else packed.unsqueeze(0), "packed", torch.int32,
+            (g, words, (n, "ld")))
+    rc = load_library().dg_pack_ue8m0_128x128(_ptr(sb), g, n, kg, _ptr(packed),
+                                              packed.shape[-1], _stream(stream))
+    _check(rc, "dg_pack_ue8m0_128x128")
+    return packed if grouped else packed.view(words, packed.shape[-1])
+
+
 # ------------------------------------------------------------------ GEMMs
 def dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace: torch.Tensor | None = None,
                    stream=None) -> torch.Tensor:
@@ -398,4 +434,57 @@ def dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, k_sizes, c=None,
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), sfb.shape[-1], _ptr(c),
         _ptr(d), _ptr(k_sizes), g, m, n, k, _stream(stream))
     _check(rc, "dg_k_grouped_fp8_gemm_nt_contiguous")
+    return d
+
+
+def _ue8m0_scales(sfa, sfb, m, n, k, lead=()):
+    """Checks packed UE8M0 scale words: sfa [.., ceil(K/512), ld >= m],
+    sfb [.., ceil(K/512), ld >= n], int32."""
+    if k % 128:
+        return
+    words = -(-(k // 128) // 4)
+    _expect(sfa, "sfa", torch.int32, lead + (words, (m, "ld")))
+    _expect(sfb, "sfb", torch.int32, lead + (words, (n, "ld")))
+
+
+def dg_fp8_gemm_nt_ue8m0(a, sfa, b, sfb, d, stream=None) -> torch.Tensor:
+    """D = A * B^T with power-of-two scales as packed UE8M0 words applied by
+    the tensor cores: a [M, K] and b [N, K] uint8, sfa int32 [ceil(K/512),
+    ld_a] (dg_pack_ue8m0 of the 1x128 scales), sfb int32 [ceil(K/512), ld_b]
+    per row of B (dg_pack_ue8m0_128x128 of the 128x128 block scales); d a
+    preallocated bfloat16 [M, N] tensor, returned."""
+    _need_cuda(a, sfa, b, sfb, d)
+    m, k = a.shape
+    n = b.shape[0]
+    if k % 128 == 0:
+        _expect(a, "a", torch.uint8, (m, k))
+        _expect(b, "b", torch.uint8, (n, k))
+    _ue8m0_scales(sfa, sfb, m, n, k)
+    _expect(d, "d", torch.bfloat16, (m, n))
+    rc = load_library().dg_fp8_gemm_nt_ue8m0(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), sfb.shape[-1], _ptr(d), m, n, k,
+        _stream(stream))
+    _check(rc, "dg_fp8_gemm_nt_ue8m0")
+    return d
+
+
+def dg_m_grouped_fp8_gemm_nt_masked_ue8m0(a, sfa, b, sfb, d, masked_m,
+                                          stream=None) -> torch.Tensor:
+    """The masked m-grouped GEMM with packed UE8M0 scales: a [G, M_max, K],
+    sfa int32 [G, ceil(K/512), ld_a], b [G, N, K], sfb int32 [G, ceil(K/512),
+    ld_b] per row of B, masked_m int32 [G] on the device; rows >= masked_m[g]
+    of d are untouched."""
+    _need_cuda(a, sfa, b, sfb, d, masked_m)
+    g, m_max, k = a.shape
+    n = b.shape[1]
+    if k % 128 == 0:
+        _expect(a, "a", torch.uint8, (g, m_max, k))
+        _expect(b, "b", torch.uint8, (g, n, k))
+    _ue8m0_scales(sfa, sfb, m_max, n, k, lead=(g,))
+    _expect(d, "d", torch.bfloat16, (g, m_max, n))
+    _expect(masked_m, "masked_m", torch.int32, (g,))
+    rc = load_library().dg_m_grouped_fp8_gemm_nt_masked_ue8m0(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), sfb.shape[-1], _ptr(d),
+        _ptr(masked_m), g, m_max, n, k, _stream(stream))
+    _check(rc, "dg_m_grouped_fp8_gemm_nt_masked_ue8m0")
     return d

@@ -301,6 +301,75 @@ int dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sfa, int6
                          effective_num_sms(), 0, nullptr);
 }
 
+namespace {
+
+// Checks shared by the UE8M0 GEMMs (packed int32 scale words, four K groups
+// each, for the rows of A and of B).
+int check_gemm_ue8m0(const uint8_t *A, const int32_t *sfa, int64_t ld_sfa, const uint8_t *B,
+                     const int32_t *sfb, int64_t ld_sfb, const void *D, int64_t rows,
+                     int64_t N, int64_t K) {
+  if (rows < 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 8 != 0) return DG_ERR_INVALID_ARG;
+  if (rows == 0) return DG_OK;
+  if (!A || !sfa || !B || !sfb || !D) return DG_ERR_INVALID_ARG;
+  if (ld_sfa < rows || ld_sfb < N) return DG_ERR_INVALID_ARG;
+  if (rows > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return DG_ERR_INVALID_ARG;
+  if (ld_sfa % 4 != 0 || ld_sfb % 4 != 0) return DG_ERR_ALIGNMENT;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(sfa) || !aligned16(sfb) || !aligned16(D))
+    return DG_ERR_ALIGNMENT;
+  return DG_OK;
+}
+
+}  // namespace
+
+int dg_fp8_gemm_nt_ue8m0(const uint8_t *A, const int32_t *sfa, int64_t ld_sfa,
+                         const uint8_t *B, const int32_t *sfb, int64_t ld_sfb, void *D,
+                         int64_t M, int64_t N, int64_t K, dg_stream_t stream) {
+  int rc = check_gemm_ue8m0(A, sfa, ld_sfa, B, sfb, ld_sfb, D, M, N, K);
+  if (rc) return rc;
+  rc = check_device();
+  if (rc) return rc;
+  if (M == 0) return DG_OK;
+  GemmParams p{};
+  p.status = device_info()->status;
+  p.sfa = reinterpret_cast<const float *>(sfa);
+  p.ld_sfa = ld_sfa;
+  p.sfb = reinterpret_cast<const float *>(sfb);
+  p.ld_sfb = ld_sfb;
+  p.d = static_cast<uint16_t *>(D);
+  p.rows = static_cast<int>(M);
+  p.n = static_cast<int>(N);
+  p.k = static_cast<int>(K);
+  p.groups = 1;
+  return launch_fp8_gemm(kDenseUE8M0, A, B, p, reinterpret_cast<cudaStream_t>(stream),
+                         effective_num_sms(), 0, nullptr);
+}
+
+int dg_m_grouped_fp8_gemm_nt_masked_ue8m0(const uint8_t *A, const int32_t *sfa,
+                                          int64_t ld_sfa, const uint8_t *B,
+                                          const int32_t *sfb, int64_t ld_sfb, void *D,
+                                          const int32_t *masked_m, int G, int64_t M_max,
+                                          int64_t N, int64_t K, dg_stream_t stream) {
+  int rc = check_gemm_ue8m0(A, sfa, ld_sfa, B, sfb, ld_sfb, D, M_max, N, K);
+  if (rc) return rc;
+  if (!masked_m || G < 1 || G > 1024 || M_max < 1) return DG_ERR_INVALID_ARG;
+  rc = check_device();
+  if (rc) return rc;
+  GemmParams p{};
+  p.status = device_info()->status;
+  p.sfa = reinterpret_cast<const float *>(sfa);
+  p.ld_sfa = ld_sfa;
+  p.sfb = reinterpret_cast<const float *>(sfb);
+  p.ld_sfb = ld_sfb;
+  p.d = static_cast<uint16_t *>(D);
+  p.masked_m = masked_m;
+  p.rows = static_cast<int>(M_max);
+  p.n = static_cast<int>(N);
+  p.k = static_cast<int>(K);
+  p.groups = G;
+  return launch_fp8_gemm(kMaskedUE8M0, A, B, p, reinterpret_cast<cudaStream_t>(stream),
+                         effective_num_sms(), 0, nullptr);
+}
+
 int dg_get_device_status(dg_stream_t stream, int *status) {
   if (!status) return DG_ERR_INVALID_ARG;
   if (!device_info()) return DG_ERR_CUDA;

@@ -84,10 +84,10 @@ constexpr int kThreads = 32 * (kControlWarps + kPromoWarps);
 // per schedule, the one with which ptxas spills least.
 constexpr int kLaunchRegs = 168;
 __host__ __device__ constexpr int ctrl_regs(int sched) {
-  return (sched == kMasked || sched == kDenseCluster) ? 56 : 40;
+  return (sched == kMasked || sched == kDenseCluster || is_ue8m0(sched)) ? 56 : 40;
 }
 __host__ __device__ constexpr int promo_regs(int sched) {
-  return (sched == kMasked || sched == kDenseCluster) ? 224 : 232;
+  return (sched == kMasked || sched == kDenseCluster || is_ue8m0(sched)) ? 224 : 232;
 }
 static_assert(ctrl_regs(kDense) * 32 * kControlWarps + promo_regs(kDense) * kPromoThreads <=
                   kLaunchRegs * kThreads,
@@ -114,7 +114,17 @@ __host__ __device__ constexpr int staged_epilogue(int sched) {
   return sched == kDenseAcc ? 2 : (sched == kDense || sched == kMasked) ? 1 : 0;
 }
 
-template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false>
+// Scale-factor bytes per stage of the UE8M0 schedules: the K block's packed
+// word (four K groups) of each of the tile's 128 rows of A and 256 rows of
+// B, arranged as tcgen05.cp's 32-row x 16-byte sources: row r of a source
+// holds the words of tile rows r, r + 32, r + 64, r + 96.
+constexpr uint32_t kSfABytes = 512;
+constexpr uint32_t kSfStageBytes = kSfABytes + 1024;
+// TMEM columns of the scale factors: two slots (consecutive K blocks) of 4
+// (A) + 8 (B) columns, 16 apart.
+constexpr uint32_t kSfSlotCols = 16;
+
+template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false, bool UE = false>
 struct Layout {
   static constexpr uint32_t kBBytes = BN * BK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
@@ -139,8 +149,13 @@ struct Layout {
   static constexpr int kBetaSlots = KG ? STAGES + NBUF : 0;
   static constexpr uint32_t kBetaOff = (kPrefixOff + 15u) & ~15u;
   static constexpr uint32_t kBetaBytes = static_cast<uint32_t>(kBetaSlots) * BN * 4u;
-  static constexpr uint32_t kTableOff = kBetaOff + kBetaBytes;
-  static constexpr uint32_t kCols = BN * NBUF;
+  // UE8M0 schedules: a scale-factor area per stage (128-byte aligned)
+  static constexpr uint32_t kSfOff = (kBetaOff + kBetaBytes + 127u) & ~127u;
+  static constexpr uint32_t kSfBytes = UE ? STAGES * kSfStageBytes : 0u;
+  static constexpr uint32_t kTableOff = kSfOff + kSfBytes;
+  static_assert(!UE || BN == 256, "the UE8M0 scale-factor layout is laid out for 256-wide tiles");
+  // accumulator buffers, then (UE8M0) the scale-factor slots
+  static constexpr uint32_t kCols = BN * NBUF + (UE ? 2 * kSfSlotCols : 0);
   static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64
                                       : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
   static_assert(kCols <= 512, "TMEM holds 512 columns");
@@ -265,16 +280,20 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // dense and masked tiles leave through shared memory (coalesced row
   // stores); contiguous tiles store each thread's row segment directly
   // (measured 1 % faster for them)
-  constexpr int kStaged = staged_epilogue(SCHED);
-  constexpr bool kDenseLike = SCHED == kDense || SCHED == kDenseAcc;
-  constexpr bool kKG = SCHED == kKGrouped;
-  using L = Layout<BN, STAGES, NBUF, kStaged, kKG>;
+  // the UE8M0 schedules walk the tiles of their base schedule
+  constexpr bool kUE = is_ue8m0(SCHED);
+  constexpr int S = base_sched(SCHED);
+  static_assert(!kUE || NBUF == 1, "the UE8M0 schedules keep one accumulator per tile");
+  constexpr int kStaged = staged_epilogue(S);
+  constexpr bool kDenseLike = (S == kDense || S == kDenseAcc) && !kUE;
+  constexpr bool kKG = S == kKGrouped;
+  using L = Layout<BN, STAGES, NBUF, kStaged, kKG, kUE>;
   constexpr int W = BN / 2;                 // columns per promotion thread
   // BN = 256 runs with the warpgroup register split (promo_regs per promotion
   // thread), the narrower tiles fit the launch allocation as they are.  The
   // contiguous schedule keeps the launch allocation: with the split, ptxas
   // spills in its promotion loop (measured 40 % slower).
-  constexpr bool kRegSplit = BN == 256 && SCHED != kContiguous;
+  constexpr bool kRegSplit = BN == 256 && S != kContiguous;
   // columns per TMEM load chunk: the whole slice up to 64 (one wait per
   // chunk; the buffer is handed back after the last chunk's wait, so the
   // fewer chunks, the sooner the MMA warp can reuse it); 16 for a 256-wide
@@ -302,7 +321,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *s_flag = reinterpret_cast<int *>(smem + L::kMiscOff + 8);
   int *s_prefix = reinterpret_cast<int *>(smem + L::kTableOff);         // [groups + 1]
-  int *s_mblocks = s_prefix + (SCHED == kMasked ? p.groups + 1 : 0);   // [groups]
+  int *s_mblocks = s_prefix + (S == kMasked ? p.groups + 1 : 0);   // [groups]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -316,7 +335,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      // UE8M0: the producer's arrival with the byte count, plus one arrival
+      // per producer lane when its scale-factor copies have landed
+      mbar_init(full_bar(s), kUE ? 33 : 1);
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < NBUF; ++b) {
@@ -336,7 +357,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // nothing above touched global memory; from here on the previous kernel's
   // results (A, the scales, the index arrays) are visible
   grid_dependency_wait();
-  if constexpr (SCHED == kMasked) {
+  if constexpr (S == kMasked) {
     if (warp == 2) {
       // prefix[e] = sum_{e' < e} ceil(clamp(masked_m[e']) / 128) * n_blocks
       int running = 0;
@@ -401,7 +422,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int units = num_units(p, SCHED, s_prefix);
+  const int units = num_units(p, S, s_prefix);
   const int kg_total = p.num_k_blocks;
 
   if (warp < kControlWarps) {
@@ -417,8 +438,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     int it = 0;
     bool alive = true;
     for (int u = u_first; u < units && alive; u += u_stride) {
-      Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
-      if constexpr (SCHED == kContiguous) {
+      Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
+      if constexpr (S == kContiguous) {
         t.group = block_expert(p, t.m_blk, true);
         if (t.group < 0) continue;
       }
@@ -428,7 +449,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       // blocks before the tile's last one -- late enough that the operand
       // stream of a long K does not evict them first, early enough to cover
       // the DRAM latency the epilogue would otherwise wait on
-      const int c_kb = (SCHED == kDenseAcc && t.split == 0) ? max(t.k_begin, t.k_end - kCAhead)
+      const int c_kb = (S == kDenseAcc && t.split == 0) ? max(t.k_begin, t.k_end - kCAhead)
                                                             : -1;
       // k-grouped: the tile's slice of B's column scales for each K block
       // (N % 8 == 0, so a multiple of 32 bytes; 16-byte aligned because the
@@ -436,7 +457,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       const int b_col0 = t.n_blk * BN;
       const uint32_t beta_bytes = kKG ? static_cast<uint32_t>(min(BN, p.n - b_col0)) * 4u : 0u;
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
-        if constexpr (SCHED == kDenseAcc) {
+        if constexpr (S == kDenseAcc) {
           if (kb == c_kb) {
             const int col0 = t.n_blk * BN;
             const uint32_t bytes = static_cast<uint32_t>(min(BN, p.n - col0)) * 4u;
@@ -464,6 +485,31 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             tma_load_3d(sa + kABytes, &tmap_b, full_bar(s), kb * BK, b_row, t.group);
           }
         }
+        if constexpr (kUE) {
+          // The K block's packed scale words (four K groups each) of the
+          // tile's rows of A and B, one 4-byte cp.async per word, placed as
+          // tcgen05.cp's sources (lane l fills source row l); rows past the
+          // operands take the last row's word (their outputs are not
+          // stored).  Each lane then arrives on the stage's barrier once its
+          // copies have landed.
+          if (it != starve_it) {
+            const uint32_t sf = base + L::kSfOff + static_cast<uint32_t>(s) * kSfStageBytes +
+                                static_cast<uint32_t>(lane) * 16u;
+            const int kwords = (kg_total + 3) / 4;
+            const int32_t *wa = reinterpret_cast<const int32_t *>(p.sfa) +
+                                (static_cast<int64_t>(t.slab) * kwords + kb / 4) * p.ld_sfa;
+            const int32_t *wb = reinterpret_cast<const int32_t *>(p.sfb) +
+                                (static_cast<int64_t>(t.group) * kwords + kb / 4) * p.ld_sfb;
+#pragma unroll
+            for (int m1 = 0; m1 < 4; ++m1)
+              cp_async_4(sf + 4u * m1, wa + min(a_row + lane + 32 * m1, p.rows - 1));
+#pragma unroll
+            for (int n1 = 0; n1 < 8; ++n1)
+              cp_async_4(sf + kSfABytes + 512u * (n1 >> 2) + 4u * (n1 & 3),
+                         wb + min(b_row + lane + 32 * n1, p.n - 1));
+            cp_async_arrive_noinc(full_bar(s));
+          }
+        }
         __syncwarp();
       }
     }
@@ -475,13 +521,64 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     for (int i = max(0, it - STAGES); i < it; ++i)
       if (i != starve_it) mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &never, p.status);
   } else if (warp == 1) {
+   if constexpr (kUE) {
+    // ================================================ MMA issuer, UE8M0 scales
+    // The tensor cores apply the scales: each K block's 4 MMAs (kind::mxf8f6f4
+    // with block scaling) accumulate into the tile's single TMEM accumulator,
+    // which the promotion warps drain once per tile.  Before them, the block's
+    // scale words are copied from the stage into TMEM (alternating between
+    // two slots), replicated across the four lane quarters; tcgen05 copies and
+    // MMAs from this thread execute in order.
+    constexpr uint32_t idesc0 = idesc_mxf8_ue8m0(BM, BN);
+    const uint32_t acc_t = tmem_base;
+    const uint32_t sf_t = tmem_base + static_cast<uint32_t>(BN * NBUF);
+    int it = 0, tile_i = 0;
+    bool alive = true;
+    for (int u = u_first; u < units && alive; u += u_stride, ++tile_i) {
+      const Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
+      // the previous tile's accumulator has been read out
+      if (!mbar_wait(tempty_bar(0), (tile_i & 1) ^ 1, s_abort, p.status)) break;
+      tc_fence_after();
+      for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(full_bar(s), ph, s_abort, p.status)) { alive = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          // the scale words arrived through cp.async (generic proxy); make
+          // them visible to the tensor-core copy
+          fence_proxy_async_smem();
+          const uint32_t sf_s = base + L::kSfOff + static_cast<uint32_t>(s) * kSfStageBytes;
+          const uint32_t slot = sf_t + static_cast<uint32_t>(it & 1) * kSfSlotCols;
+          tmem_cp_32x128b_x4(slot, smem_desc_rows16(sf_s));
+          tmem_cp_32x128b_x4(slot + 4, smem_desc_rows16(sf_s + kSfABytes));
+          tmem_cp_32x128b_x4(slot + 8, smem_desc_rows16(sf_s + kSfABytes + 512));
+          // byte kb % 4 of each cell holds this K block's scale
+          const uint32_t byte = static_cast<uint32_t>(kb & 3);
+          const uint32_t idesc = idesc_sf_bytes(idesc0, byte);
+          const uint32_t sfa_t = slot | (byte << 30);
+          const uint32_t sfb_t = (slot + 4) | (byte << 30);
+          const uint32_t sa = base + s * L::kStageBytes;
+          const uint64_t adesc = smem_desc_k128_sw128(sa);
+          const uint64_t bdesc = smem_desc_k128_sw128(sa + kABytes);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            umma_mxf8_ue8m0(acc_t, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t, sfb_t,
+                            (kb > t.k_begin || k > 0) ? 1u : 0u);
+          umma_commit(empty_bar(s));
+          if (kb + 1 == t.k_end) umma_commit(tfull_bar(0));
+        }
+        __syncwarp();
+      }
+    }
+   } else {
     // ============================================================ MMA issuer
     constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
     int it = 0, acc_it = 0;
     bool alive = true;
     for (int u = u_first; u < units && alive; u += u_stride) {
-      Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
-      if constexpr (SCHED == kContiguous) {
+      Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
+      if constexpr (S == kContiguous) {
         if (block_expert(p, t.m_blk, false) < 0) continue;
       }
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it, ++acc_it) {
@@ -511,6 +608,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         __syncwarp();
       }
     }
+   }
     {
       // every MMA issued above must complete before TMEM is freed (bounded,
       // and not cut short by the abort flag)
@@ -530,6 +628,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
     const int nb_total = (p.n + 127) / 128;
     int it = 0;
+    int tile_i = 0;  // UE8M0: tiles drained so far (the accumulator's phase)
     bool alive = true;
     // every promotion thread arrives, then waits for the phase (bounded)
     uint32_t epi_phase = 0;
@@ -540,27 +639,51 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       return ok;
     };
     for (int u = u_first; u < units && alive; u += u_stride) {
-      Tile t = unit_to_tile(p, SCHED, u, s_prefix, s_mblocks);
+      Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
       const int row = t.m_blk * BM + row_in_tile;
       bool row_ok;
-      if constexpr (SCHED == kContiguous) {
+      if constexpr (S == kContiguous) {
         t.group = block_expert(p, t.m_blk, false);
         if (t.group < 0) continue;
         row_ok = row < p.rows && __ldg(p.m_indices + row) == t.group;
-      } else if constexpr (SCHED == kMasked) {
+      } else if constexpr (S == kMasked) {
         row_ok = row < masked_rows(p, t.slab);
       } else {
         row_ok = row < p.rows;
       }
       const int col0 = t.n_blk * BN + half * W;  // first column of this thread
-      // a thread's W columns (W divides 128 or equals 128) lie in one beta block
-      const int nb = min(col0, p.n - 1) / 128;
-      const float *sfb_ptr =
-          p.sfb + (static_cast<int64_t>(t.group) * nb_total + nb) * kg_total;
 
       float acc[W];
 #pragma unroll
       for (int c = 0; c < W; ++c) acc[c] = 0.0f;
+
+      if constexpr (kUE) {
+        // The tensor cores applied the scales and summed the whole K range
+        // in TMEM: read this thread's row segment of the accumulator once and
+        // hand it back to the MMA warp for the next tile.
+        if (!mbar_wait(tfull_bar(0), tile_i & 1, s_abort, p.status)) {
+          alive = false;
+          break;
+        }
+        ++tile_i;
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < W; c0 += LW) {
+          uint32_t r[LW];
+          tmem_ld<LW>(tmem_base + t_lane + half * W + c0, r);
+          tmem_wait_ld();
+          reg_barrier<LW>(r);
+#pragma unroll
+          for (int c = 0; c < LW; ++c) acc[c0 + c] = __uint_as_float(r[c]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(0));
+      } else {
+      // a thread's W columns (W divides 128 or equals 128) lie in one beta block
+      const int nb = min(col0, p.n - 1) / 128;
+      const float *sfb_ptr =
+          p.sfb + (static_cast<int64_t>(t.group) * nb_total + nb) * kg_total;
 
       // This thread's row scale alpha is loaded two K blocks ahead into
       // registers (one coalesced 128-byte load per warp and block); rows past
@@ -647,6 +770,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           }
         }
       }
+      }  // (not UE8M0)
       if (!alive) break;
 
       // ---------------------------------------------------------- epilogue
@@ -724,7 +848,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             const int c4 = f / valid, r = f - c4 * valid;
             const int col = t.n_blk * BN + 4 * c4;
             if (ok[q] && col < p.n) {
-              if constexpr (SCHED == kDenseAcc) {
+              if constexpr (S == kDenseAcc) {
                 const float4 cv = __ldg(reinterpret_cast<const float4 *>(
                     p.c + static_cast<int64_t>(row0 + r) * p.n + col));
                 sum[q].x += cv.x;
@@ -766,7 +890,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
         continue;
       }
-      if constexpr (SCHED == kDenseCluster) {
+      if constexpr (S == kDenseCluster) {
         // Leave this split's FP32 partial in this CTA's shared memory (the
         // stage ring, drained: every block's MMAs have completed) for the
         // cluster reduction after the role loops.  Layout [128 rows][BN/4]
@@ -921,11 +1045,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // The splits of a tile are the CTAs of one cluster (rank = split).  Every
   // thread of every CTA passes both cluster barriers, whatever happened in
   // its role loop, so none can strand the others.
-  if constexpr (SCHED == kDenseCluster) {
+  if constexpr (S == kDenseCluster) {
     __syncwarp();
     cluster_sync();  // all partials written
     if (warp >= kControlWarps && !*s_abort) {
-      const Tile t = unit_to_tile(p, SCHED, static_cast<int>(blockIdx.x), s_prefix, s_mblocks);
+      const Tile t = unit_to_tile(p, S, static_cast<int>(blockIdx.x), s_prefix, s_mblocks);
       constexpr int kChunksF = BN / 4;
       constexpr int kSwF = kChunksF < 8 ? kChunksF : 8;
       const int split = static_cast<int>(cluster_ctarank());
@@ -976,9 +1100,14 @@ struct Candidate {
 constexpr Candidate kCandidates[] = {
     {256, 4, 2}, {128, 6, 4}, {64, 8, 8}, {32, 8, 8}, {16, 8, 8}};
 
-template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false>
+// The UE8M0 schedules' one tile form: 256 wide, one accumulator (the tile
+// sums all of K in TMEM), three stages (the fourth does not fit beside the
+// per-stage scale-factor areas and the output staging).
+constexpr Candidate kUECandidate = {256, 3, 1};
+
+template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false, bool UE = false>
 constexpr int smem_bytes_for(int extra) {
-  return 1024 + Layout<BN, STAGES, NBUF, STAGED, KG>::kTableOff + extra;
+  return 1024 + Layout<BN, STAGES, NBUF, STAGED, KG, UE>::kTableOff + extra;
 }
 
 bool print_configs() {
@@ -989,8 +1118,8 @@ bool print_configs() {
 template <int BN, int STAGES, int NBUF, int SCHED>
 int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                     int grid, int extra_smem, cudaStream_t stream, bool coop) {
-  const int smem = smem_bytes_for<BN, STAGES, NBUF, staged_epilogue(SCHED),
-                                  SCHED == kKGrouped>(extra_smem);
+  const int smem = smem_bytes_for<BN, STAGES, NBUF, staged_epilogue(base_sched(SCHED)),
+                                  SCHED == kKGrouped, is_ue8m0(SCHED)>(extra_smem);
   auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED>;
   static int configured_smem[64] = {0};  // per device; grows only
   int dev = 0;
@@ -1096,6 +1225,10 @@ int single_smem(int sched, int extra) {
 }
 
 int config_smem(int bn, int extra, int sched) {
+  if (is_ue8m0(sched))
+    // (both UE8M0 schedules stage the BF16 tile: kind 1)
+    return smem_bytes_for<kUECandidate.bn, kUECandidate.stages, kUECandidate.nbuf,
+                          staged_epilogue(kDense), false, true>(extra);
   switch (bn) {
     case 256: return single_smem<256, 4, 2>(sched, extra);
     case 128: return single_smem<128, 6, 4>(sched, extra);
@@ -1121,13 +1254,18 @@ int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmPar
   // splits that wait for each other through global memory need all CTAs
   // resident; a cluster's splits are co-scheduled by construction
   const bool coop = p.splits > 1 && SCHED != kDenseCluster;
-  switch (bn) {
-    case 256: return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st, coop);
-    case 128: return launch_instance<128, 6, 4, SCHED>(ta, tb, p, grid, extra, st, coop);
-    case 64: return launch_instance<64, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
-    case 32: return launch_instance<32, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
-    case 16: return launch_instance<16, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
-    default: return DG_ERR_INVALID_ARG;
+  if constexpr (is_ue8m0(SCHED)) {
+    return launch_instance<kUECandidate.bn, kUECandidate.stages, kUECandidate.nbuf, SCHED>(
+        ta, tb, p, grid, extra, st, false);
+  } else {
+    switch (bn) {
+      case 256: return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st, coop);
+      case 128: return launch_instance<128, 6, 4, SCHED>(ta, tb, p, grid, extra, st, coop);
+      case 64: return launch_instance<64, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
+      case 32: return launch_instance<32, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
+      case 16: return launch_instance<16, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
+      default: return DG_ERR_INVALID_ARG;
+    }
   }
 }
 
@@ -1307,9 +1445,35 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
   // ------------------------------------------------ choose the tile form
   // masked launches keep per-expert row-block counts and prefix sums in
   // shared memory
-  const int extra = sched == kMasked ? 8 * (p.groups + 1)
+  const int extra = base_sched(sched) == kMasked ? 8 * (p.groups + 1)
                     : sched == kKGrouped ? 4 * (p.groups + 1) : 0;
   const int max_smem = max_smem_per_block();
+  if (is_ue8m0(sched)) {
+    // one tile form, no K split: the whole tile sums K in TMEM
+    if (config_smem(kUECandidate.bn, extra, sched) > max_smem) return DG_ERR_INVALID_ARG;
+    const int bn = kUECandidate.bn;
+    p.num_m_blocks = static_cast<int>((rows + BM - 1) / BM);
+    p.num_n_blocks = static_cast<int>((n + bn - 1) / bn);
+    p.splits = 1;
+    p.full_tiles = 0;
+    p.ws = nullptr;
+    p.a_box_rows = BM;
+    CUtensorMap ta, tb;
+    const bool masked = base_sched(sched) == kMasked;
+    int rc = make_tmap(&ta, A, k, rows, masked ? p.groups : 1, BM);
+    if (rc) return rc;
+    rc = make_tmap(&tb, B, k, n, masked ? p.groups : 1, bn);
+    if (rc) return rc;
+    const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks *
+                          (masked ? p.groups : 1);
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
+    if (print_configs())
+      fprintf(stderr, "[dg] gemm sched=%d (UE8M0) rows=%lld n=%lld k=%lld groups=%d grid=%d\n",
+              sched, static_cast<long long>(rows), static_cast<long long>(n),
+              static_cast<long long>(k), p.groups, grid);
+    return masked ? dispatch<kMaskedUE8M0>(bn, ta, tb, p, grid, extra, stream)
+                  : dispatch<kDenseUE8M0>(bn, ta, tb, p, grid, extra, stream);
+  }
   const Choice choice =
       choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes, extra, max_smem);
   int bn = choice.bn, splits = choice.splits;

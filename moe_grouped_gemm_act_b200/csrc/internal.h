@@ -38,9 +38,22 @@ inline cudaLaunchAttribute pdl_attribute() {
 // kKGrouped: the groups split K; group g computes its own FP32
 // D[g] = C[g] + A_g B_g^T over its K segment, with 1x128 scales on both
 // operands (one B scale per column and K block).
+// kDenseUE8M0 / kMaskedUE8M0: the dense and masked tiles with power-of-two
+// scales given as packed UE8M0 codes, applied by the tensor cores
+// (block-scaled MMA): the tile accumulates in TMEM over all of K and the
+// promotion warps only drain it for the epilogue.
 enum Sched : int {
-  kDense = 0, kContiguous = 1, kMasked = 2, kDenseCluster = 3, kDenseAcc = 4, kKGrouped = 5
+  kDense = 0, kContiguous = 1, kMasked = 2, kDenseCluster = 3, kDenseAcc = 4, kKGrouped = 5,
+  kDenseUE8M0 = 6, kMaskedUE8M0 = 7
 };
+
+// The tile schedule (work list, row validity, epilogue) a schedule follows.
+__host__ __device__ constexpr int base_sched(int sched) {
+  return sched == kDenseUE8M0 ? kDense : sched == kMaskedUE8M0 ? kMasked : sched;
+}
+__host__ __device__ constexpr bool is_ue8m0(int sched) {
+  return sched == kDenseUE8M0 || sched == kMaskedUE8M0;
+}
 
 // Kernel parameters besides the two tensor maps.  Row coordinates are inside
 // one "slab": the whole of A for dense and contiguous, one expert's M_max rows
@@ -48,10 +61,13 @@ enum Sched : int {
 // it does not use (so the struct, and every other schedule's code, stays as
 // it was).
 struct GemmParams {
-  const float *sfa;      // MN-major alpha: [slab][K/128][ld_sfa]
+  const float *sfa;      // MN-major alpha: [slab][K/128][ld_sfa]; UE8M0: packed
+                         // int32 words [slab][ceil(K/512)][ld_sfa]
   int64_t ld_sfa;
   const float *sfb;      // beta: [group][ceil(N/128)][K/128]; k-grouped:
-                         // MN-major [K/128][ld_sfb], one scale per column
+                         // MN-major [K/128][ld_sfb], one scale per column;
+                         // UE8M0: int32 words [group][ceil(K/512)][ld_sfb]
+                         // per row of B
   union {
     uint16_t *d;         // BF16 output [slab][rows][N]
     float *d_f32;        // k-grouped: FP32 output [group][rows][N]
@@ -67,7 +83,7 @@ struct GemmParams {
   float *ws;             // split-K partials (nullptr: no split)
   union {
     uint32_t *ws_ticket;  // split-K arrival counters, one per output tile
-    int64_t ld_sfb;       // k-grouped: row stride of the B scales
+    int64_t ld_sfb;       // k-grouped and UE8M0: row stride of the B scales
   };
   int rows;              // dense: M; contiguous: M_total; masked: M_max
   int n, k;

@@ -406,6 +406,20 @@ __device__ __forceinline__ uint64_t smem_desc_k128_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory descriptor of a no-swizzle K-major source whose rows are 16
+// bytes, stored contiguously (8-row core matrices of 128 bytes, one after
+// the other): the source of tcgen05.cp's 32x128b shape.  Stride byte offset
+// = 128 (next 8 rows), leading byte offset 128 (unused: one 16-byte column),
+// version 1, layout type 0 (no swizzle).  saddr 16-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);      // start address
+  d |= static_cast<uint64_t>(128 >> 4) << 16;              // leading byte offset
+  d |= static_cast<uint64_t>(128 >> 4) << 32;              // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                     // version
+  return d;
+}
+
 // Instruction descriptor: kind::f8f6f4, A and B E4M3 (format 0), both
 // K-major, FP32 accumulator (c_format 1), shape M x N.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {
@@ -413,6 +427,61 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {
          (0u << 7) | (0u << 10) |                   // A, B: E4M3
          (static_cast<uint32_t>(n >> 3) << 17) |    // N / 8
          (static_cast<uint32_t>(m >> 4) << 24);     // M / 16
+}
+
+// Instruction descriptor of the block-scaled kind::mxf8f6f4: A and B E4M3
+// (format 0), both K-major, UE8M0 scale factors (scale format 1 at bit 23),
+// shape M x N; the FP32 accumulator is implied.  The byte of each 32-bit
+// scale-factor cell to use (one of four K groups packed per cell) goes to
+// bits 29-30 (A) and 4-5 (B), and to bits 30-31 of the scale-factor TMEM
+// addresses given to the MMA.
+__host__ __device__ constexpr uint32_t idesc_mxf8_ue8m0(int m, int n) {
+  return (0u << 7) | (0u << 10) |                   // A, B: E4M3
+         (static_cast<uint32_t>(n >> 3) << 17) |    // N / 8
+         (1u << 23) |                               // scale factors UE8M0
+         (static_cast<uint32_t>(m >> 4) << 24);     // M / 16
+}
+
+__host__ __device__ constexpr uint32_t idesc_sf_bytes(uint32_t idesc, uint32_t byte) {
+  return idesc | (byte << 29) | (byte << 4);
+}
+
+// D[tmem] (+)= (A * 2^sfa) * (B * 2^sfb)^T, kind::mxf8f6f4 with one UE8M0
+// scale factor per row of A and of B for the MMA's 32-wide K slice, read
+// from TMEM at sfa_tmem / sfb_tmem (the byte within each cell in the top two
+// address bits and in the instruction descriptor).  One thread issues.
+__device__ __forceinline__ void umma_mxf8_ue8m0(uint32_t d_tmem, uint64_t a_desc,
+                                                uint64_t b_desc, uint32_t idesc,
+                                                uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Shared memory -> TMEM: 32 rows of 128 bits (smem_desc_rows16 source) into
+// 32 lanes x 4 columns at taddr, the same data written into each of the four
+// 32-lane subpartitions (the replicated layout the block-scaled MMA reads
+// its scale factors from).  Asynchronous; tcgen05 operations issued by the
+// same thread after it (the MMAs that read these columns) see its result.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+               : "memory");
+}
+
+// 4-byte asynchronous copy global -> shared (both 4-byte aligned).
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Arrives on `bar` (counting as one of its expected arrivals) once every
+// cp.async this thread issued before has completed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 }  // namespace dg
