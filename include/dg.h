@@ -118,6 +118,26 @@ int dg_quantize_1x128(const void *x, int x_dtype, int64_t batch, int64_t M,
                       float *sf, int64_t ld_sf, int flags, dg_stream_t stream);
 
 /*
+ * dg_quantize_128x1 -- the 1 x 128 activation quantization of Lesson 13,
+ * Fig. 13-1 (groups of 128 consecutive K elements of one row of the logical
+ * [M][K] operand) for an operand stored with K outermost, x [K][M]: the
+ * group of column m and K group g is x[128 g .. 128 g + 127][m].  This is how
+ * the TN / TT GEMMs and the TN k-grouped GEMM take their transposed operands.
+ *
+ *   x       device float or BF16 (x_dtype) [K][ld_x], ld_x >= M.
+ *   q       device uint8 [K][ld_q] E4M3 codes, ld_q >= M.
+ *   sf      device float [K/128][ld_sf], MN-major (sf[g * ld_sf + m]), the
+ *           layout the GEMMs read; ld_sf >= M, % 4 == 0.
+ *   flags   DG_SCALE_FP32 or DG_SCALE_POW2.
+ *   M >= 0 (0 is a no-op), K % 128 == 0, K / 128 <= 65535; pointers
+ *   16-byte aligned.
+ * Bit-exact with dg_quantize_1x128 applied to the transposed operand.
+ */
+int dg_quantize_128x1(const void *x, int x_dtype, int64_t K, int64_t M,
+                      int64_t ld_x, uint8_t *q, int64_t ld_q, float *sf,
+                      int64_t ld_sf, int flags, dg_stream_t stream);
+
+/*
  * dg_quantize_128x128 -- 128 x 128 weight block quantization (Lesson 13,
  * Fig. 13-1: "one scale beta per 128 x 128 block, quantized offline").
  *
@@ -210,10 +230,41 @@ int dg_fp8_gemm_nt(const uint8_t *A, const float *sfa, int64_t ld_sfa,
                    int64_t N, int64_t K, void *workspace,
                    size_t workspace_bytes, dg_stream_t stream);
 
-/* Workspace size in bytes with which dg_fp8_gemm_nt uses the K split its
- * tile heuristic prefers for this shape on the current device (0 when that
- * choice does not split K; the result depends on the SM count in effect,
- * see dg_set_num_sms).  A multiple of 256 bytes. */
+/*
+ * dg_fp8_gemm_nn, dg_fp8_gemm_tn, dg_fp8_gemm_tt -- the dense GEMM with the
+ * other operand layouts ("DeepGEMM architecture deep dive", section 3: every
+ * GEMM is D = C + A @ B, NT by default, and sm_100 supports NT, TN, NN and
+ * TT).  The first letter says how A is used, the second how B is: N as
+ * stored, T transposed, with D = A * B^T always [M][N]:
+ *   NN  A [M][K] (K-major) and B stored [K][N] (N contiguous);
+ *   TN  A stored [K][M] (M contiguous) and B stored [K][N];
+ *   TT  A stored [K][M] and B [N][K] (K-major).
+ * The scales keep their logical meaning: sfa is alpha per row of A and
+ * 128-wide K group (device float [K/128][ld_sfa], MN-major, as for NT) and
+ * sfb is beta per 128 x 128 block of B's [N][K] view ([ceil(N/128)][K/128]).
+ * An operand stored with K outermost is loaded as MN-major tiles, so its row
+ * stride must be a multiple of 16 bytes: M % 16 == 0 for TN and TT, N % 16
+ * == 0 for NN and TN (DG_ERR_ALIGNMENT otherwise).  Everything else --
+ * arguments, workspace use, errors, determinism -- is as in dg_fp8_gemm_nt
+ * (the tile is 128 or 256 columns wide).
+ */
+int dg_fp8_gemm_nn(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                   const uint8_t *B, const float *sfb, void *D, int64_t M,
+                   int64_t N, int64_t K, void *workspace,
+                   size_t workspace_bytes, dg_stream_t stream);
+int dg_fp8_gemm_tn(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                   const uint8_t *B, const float *sfb, void *D, int64_t M,
+                   int64_t N, int64_t K, void *workspace,
+                   size_t workspace_bytes, dg_stream_t stream);
+int dg_fp8_gemm_tt(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                   const uint8_t *B, const float *sfb, void *D, int64_t M,
+                   int64_t N, int64_t K, void *workspace,
+                   size_t workspace_bytes, dg_stream_t stream);
+
+/* Workspace size in bytes with which dg_fp8_gemm_nt (and the NN, TN, TT
+ * forms) use the K split the tile heuristic prefers for this shape on the
+ * current device (0 when that choice does not split K; the result depends on
+ * the SM count in effect, see dg_set_num_sms).  A multiple of 256 bytes. */
 size_t dg_fp8_gemm_nt_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -251,6 +302,32 @@ size_t dg_fp8_gemm_nt_workspace_size(int64_t M, int64_t N, int64_t K);
 int dg_fp8_gemm_nt_noalloc(const uint8_t *A, const float *sfa, int64_t ld_sfa,
                            const uint8_t *B, const float *sfb, void *D, int64_t M,
                            int64_t N, int64_t K, dg_stream_t stream);
+
+/*
+ * dg_fp8_gemm_nt_quantize -- dg_fp8_gemm_nt with the FP8 cast of its output
+ * fused into the epilogue ("DeepGEMM architecture deep dive", section 3:
+ * users should fuse the FP8 cast into the kernel that produces the data).
+ * D is not written as BF16; each row's 128-column groups leave the GEMM
+ * already quantized 1 x 128 (Lesson 13, Fig. 13-1), in the layouts the next
+ * GEMM takes as its A and alpha.  The result is bit-identical to rounding D
+ * to BF16 and then calling dg_quantize_1x128 on it (DG_DTYPE_BF16, the same
+ * flags), for the tile form this call uses (256-wide tiles, K not split; a
+ * dg_fp8_gemm_nt that splits K may round a few elements of D differently).
+ *
+ *   A, sfa, ld_sfa, B, sfb, M, K   as in dg_fp8_gemm_nt.
+ *   N      N % 128 == 0 (whole groups).
+ *   Dq     device uint8 [M][N] E4M3 codes, 16-byte aligned.
+ *   sfd    device float [N/128][ld_sfd], MN-major: the scale of row i, column
+ *          group g at sfd[g * ld_sfd + i]; ld_sfd >= M, % 4 == 0, 16-byte
+ *          aligned.
+ *   flags  DG_SCALE_FP32 or DG_SCALE_POW2 (scales rounded up to powers of
+ *          two, UE8M0-representable).
+ * No workspace: K is never split.  Deterministic.
+ */
+int dg_fp8_gemm_nt_quantize(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                            const uint8_t *B, const float *sfb, uint8_t *Dq,
+                            float *sfd, int64_t ld_sfd, int64_t M, int64_t N,
+                            int64_t K, int flags, dg_stream_t stream);
 
 /*
  * dg_fp8_gemm_nt_accumulate -- D = C + A * B^T (Deep dive, section 3: the NT
@@ -412,6 +489,26 @@ int dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sfa,
  * error recorded since the last read (DG_ERR_TIMEOUT, DG_ERR_DEVICE_DATA).
  * Returns DG_OK, or DG_ERR_CUDA if the synchronization itself failed.
  */
+/*
+ * dg_k_grouped_fp8_gemm_tn_contiguous -- the K-grouped GEMM of
+ * dg_k_grouped_fp8_gemm_nt_contiguous with both operands stored with the
+ * token axis K outermost, as a weight gradient's activations and output
+ * gradients are ("DeepGEMM architecture deep dive", section 3, the grouped
+ * GEMM table: K-grouped, FP8 TN):
+ *   A  device uint8 [K][M] (M contiguous), M % 16 == 0;
+ *   B  device uint8 [K][N] (N contiguous), N % 16 == 0;
+ * sfa [K/128][ld_sfa] and sfb [K/128][ld_sfb], C, D, k_sizes and everything
+ * else as in the NT form: D[g][i][j] = C[g][i][j] + the sum over group g's
+ * K segment (per 128-wide K block, scaled by alpha[i] and beta[j] of the
+ * block) of A[k][i] * B[k][j].
+ */
+int dg_k_grouped_fp8_gemm_tn_contiguous(const uint8_t *A, const float *sfa,
+                                        int64_t ld_sfa, const uint8_t *B,
+                                        const float *sfb, int64_t ld_sfb,
+                                        const float *C, float *D,
+                                        const int32_t *k_sizes, int G, int64_t M,
+                                        int64_t N, int64_t K, dg_stream_t stream);
+
 int dg_get_device_status(dg_stream_t stream, int *status);
 
 #ifdef __cplusplus

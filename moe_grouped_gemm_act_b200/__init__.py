@@ -10,14 +10,22 @@ Entry points (same names as the C ABI):
 
 * ``dg_quantize_1x128(x, pow2=False)`` -> (q, sf)    1 x 128 E4M3 activations
 * ``dg_quantize_128x128(w, pow2=False)`` -> (q, sf)  128 x 128 E4M3 weights
+* ``dg_quantize_128x1(x, pow2=False)`` -> (q, sf)  1 x 128-along-K groups of an
+  operand stored [K, M] (K outermost)
 * ``dg_pack_ue8m0(sf, m)`` -> packed int32 UE8M0 scales (4 K groups per word)
 * ``dg_pack_ue8m0_128x128(sf, n)`` -> B's 128 x 128 block scales packed per row
 * ``dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace=None)``
 * ``dg_fp8_gemm_nt_accumulate(a, sfa, b, sfb, c, d, workspace=None)``  D = C + A B^T
 * ``dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, d)``
+* ``dg_fp8_gemm_nt_quantize(a, sfa, b, sfb, pow2=False)`` -> (dq, sfd)  the
+  output quantized 1 x 128 in the epilogue (E4M3 codes and MN-major scales)
+* ``dg_fp8_gemm_nn / _tn / _tt(a, sfa, b, sfb, d, workspace=None)``  the other
+  operand layouts (A stored [K, M] for T, B stored [K, N] for N)
 * ``dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices)``
 * ``dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m)``
 * ``dg_k_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, k_sizes, c=None)``
+* ``dg_k_grouped_fp8_gemm_tn_contiguous(a, sfa, b, sfb, d, k_sizes, c=None)``
+  (a [K, M] and b [K, N])
 * ``dg_fp8_gemm_nt_ue8m0(a, sfa, b, sfb, d)``, ``dg_m_grouped_fp8_gemm_nt_masked_ue8m0(
   a, sfa, b, sfb, d, masked_m)``  power-of-two scales as packed UE8M0 words,
   applied by the tensor cores
@@ -50,8 +58,11 @@ DG_ERR_TIMEOUT, DG_ERR_DEVICE_DATA = -6, -7
 EXPORTS = [
     "dg_status_string", "dg_get_mk_alignment_for_contiguous_layout",
     "dg_get_tma_aligned_size", "dg_set_num_sms", "dg_get_num_sms",
-    "dg_quantize_1x128", "dg_quantize_128x128", "dg_pack_ue8m0", "dg_pack_ue8m0_128x128",
+    "dg_quantize_1x128", "dg_quantize_128x1", "dg_quantize_128x128", "dg_pack_ue8m0",
+    "dg_pack_ue8m0_128x128",
     "dg_fp8_gemm_nt", "dg_fp8_gemm_nt_ue8m0", "dg_m_grouped_fp8_gemm_nt_masked_ue8m0",
+    "dg_fp8_gemm_nn", "dg_fp8_gemm_tn", "dg_fp8_gemm_tt", "dg_k_grouped_fp8_gemm_tn_contiguous",
+    "dg_fp8_gemm_nt_quantize",
     "dg_fp8_gemm_nt_workspace_size", "dg_fp8_gemm_nt_noalloc", "dg_fp8_gemm_nt_accumulate",
     "dg_m_grouped_fp8_gemm_nt_contiguous",
     "dg_m_grouped_fp8_gemm_nt_masked", "dg_k_grouped_fp8_gemm_nt_contiguous",
@@ -85,12 +96,19 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "dg_get_num_sms": (I, []),
         "dg_quantize_1x128": (I, [P, I, I64, I64, I64, I64, P, I64, P, I64, I, P]),
         "dg_quantize_128x128": (I, [P, I64, I64, I64, P, P, I, P]),
+        "dg_quantize_128x1": (I, [P, I, I64, I64, I64, P, I64, P, I64, I, P]),
         "dg_pack_ue8m0": (I, [P, I64, I64, I64, I64, P, I64, P]),
         "dg_pack_ue8m0_128x128": (I, [P, I64, I64, I64, P, I64, P]),
         "dg_fp8_gemm_nt_ue8m0": (I, [P, P, I64, P, P, I64, P, I64, I64, I64, P]),
         "dg_m_grouped_fp8_gemm_nt_masked_ue8m0":
             (I, [P, P, I64, P, P, I64, P, P, I, I64, I64, I64, P]),
         "dg_fp8_gemm_nt": (I, [P, P, I64, P, P, P, I64, I64, I64, P, SZ, P]),
+        "dg_fp8_gemm_nn": (I, [P, P, I64, P, P, P, I64, I64, I64, P, SZ, P]),
+        "dg_fp8_gemm_nt_quantize": (I, [P, P, I64, P, P, P, P, I64, I64, I64, I64, I, P]),
+        "dg_fp8_gemm_tn": (I, [P, P, I64, P, P, P, I64, I64, I64, P, SZ, P]),
+        "dg_fp8_gemm_tt": (I, [P, P, I64, P, P, P, I64, I64, I64, P, SZ, P]),
+        "dg_k_grouped_fp8_gemm_tn_contiguous":
+            (I, [P, P, I64, P, P, I64, P, P, P, I, I64, I64, I64, P]),
         "dg_fp8_gemm_nt_workspace_size": (SZ, [I64, I64, I64]),
         "dg_fp8_gemm_nt_noalloc": (I, [P, P, I64, P, P, P, I64, I64, I64, P]),
         "dg_fp8_gemm_nt_accumulate": (I, [P, P, I64, P, P, P, P, I64, I64, I64, P, SZ, P]),
@@ -239,6 +257,32 @@ def dg_quantize_1x128(x: torch.Tensor, pow2: bool = False, q=None, sf=None,
     return q, sf
 
 
+def dg_quantize_128x1(x: torch.Tensor, pow2: bool = False, q=None, sf=None, stream=None):
+    """1 x 128-along-K quantization of an operand stored [K, M] (float32 or
+    bfloat16): returns (q uint8 [K, M], sf float32 [K/128, ld]) with ld =
+    dg_get_tma_aligned_size(M, 4); sf[g, m] is the scale of column m's K
+    group g.  Bit-exact with dg_quantize_1x128 of x.T."""
+    _need_cuda(x)
+    k, m = x.shape
+    dtype = {torch.float32: DG_DTYPE_F32, torch.bfloat16: DG_DTYPE_BF16}.get(x.dtype)
+    if dtype is None:
+        raise ValueError("x must be float32 or bfloat16")
+    if q is None:
+        q = torch.empty((k, m), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty((k // 128, dg_get_tma_aligned_size(m, 4)), dtype=torch.float32,
+                         device=x.device)
+    _need_cuda(q, sf)
+    if k % 128 == 0:
+        _expect(q, "q", torch.uint8, (k, m))
+        _expect(sf, "sf", torch.float32, (k // 128, (m, "ld")))
+    rc = load_library().dg_quantize_128x1(
+        _ptr(x), dtype, k, m, m, _ptr(q), m, _ptr(sf), sf.shape[-1],
+        DG_SCALE_POW2 if pow2 else DG_SCALE_FP32, _stream(stream))
+    _check(rc, "dg_quantize_128x1")
+    return q, sf
+
+
 def dg_quantize_128x128(w: torch.Tensor, pow2: bool = False, stream=None):
     """128 x 128 quantization of w [N, K] or [G, N, K] float32.
 
@@ -336,6 +380,73 @@ def dg_fp8_gemm_nt(a, sfa, b, sfb, d, workspace: torch.Tensor | None = None,
     return d
 
 
+def _fp8_gemm_layout(name, a_t, b_t, a, sfa, b, sfb, d, workspace, stream):
+    """The dense GEMM with A stored [K, M] when a_t, B stored [K, N] when b_t
+    (else [M, K] and [N, K]); the scales keep their logical layouts."""
+    _need_cuda(a, sfa, b, sfb, d)
+    if a_t:
+        k, m = a.shape
+    else:
+        m, k = a.shape
+    n = b.shape[1] if b_t else b.shape[0]
+    if k % 128 == 0:
+        _expect(a, "a", torch.uint8, (k, m) if a_t else (m, k))
+        _expect(b, "b", torch.uint8, (k, n) if b_t else (n, k))
+        _expect(sfa, "sfa", torch.float32, (k // 128, (m, "ld")))
+        _expect(sfb, "sfb", torch.float32, (-(-n // 128), k // 128))
+    _expect(d, "d", torch.bfloat16, (m, n))
+    if workspace is not None:
+        _need_cuda(workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = getattr(load_library(), name)(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d), m, n, k,
+        _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, name)
+    return d
+
+
+def dg_fp8_gemm_nt_quantize(a, sfa, b, sfb, pow2: bool = False, dq=None, sfd=None,
+                            stream=None):
+    """D = A * B^T quantized 1 x 128 in the GEMM's epilogue: returns (dq uint8
+    [M, N] E4M3 codes, sfd float32 [N/128, ld] MN-major scales, ld =
+    dg_get_tma_aligned_size(M, 4)) -- bit-identical to dg_quantize_1x128 of
+    the BF16 result of the same tile form.  N % 128 == 0."""
+    _need_cuda(a, sfa, b, sfb)
+    m, k = a.shape
+    n = b.shape[0]
+    _gemm_operands(a, sfa, b, sfb, m, n, k)
+    if n % 128:
+        raise ValueError(f"N = {n} must be a multiple of 128")
+    if dq is None:
+        dq = torch.empty((m, n), dtype=torch.uint8, device=a.device)
+    if sfd is None:
+        sfd = torch.empty((n // 128, dg_get_tma_aligned_size(m, 4)), dtype=torch.float32,
+                          device=a.device)
+    _need_cuda(dq, sfd)
+    _expect(dq, "dq", torch.uint8, (m, n))
+    _expect(sfd, "sfd", torch.float32, (n // 128, (m, "ld")))
+    rc = load_library().dg_fp8_gemm_nt_quantize(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(dq), _ptr(sfd),
+        sfd.shape[-1], m, n, k, DG_SCALE_POW2 if pow2 else DG_SCALE_FP32, _stream(stream))
+    _check(rc, "dg_fp8_gemm_nt_quantize")
+    return dq, sfd
+
+
+def dg_fp8_gemm_nn(a, sfa, b, sfb, d, workspace=None, stream=None) -> torch.Tensor:
+    """D = A * B^T with A [M, K] and B stored [K, N] (N contiguous, N % 16 == 0)."""
+    return _fp8_gemm_layout("dg_fp8_gemm_nn", False, True, a, sfa, b, sfb, d, workspace, stream)
+
+
+def dg_fp8_gemm_tn(a, sfa, b, sfb, d, workspace=None, stream=None) -> torch.Tensor:
+    """D = A * B^T with A stored [K, M] and B stored [K, N] (M, N % 16 == 0)."""
+    return _fp8_gemm_layout("dg_fp8_gemm_tn", True, True, a, sfa, b, sfb, d, workspace, stream)
+
+
+def dg_fp8_gemm_tt(a, sfa, b, sfb, d, workspace=None, stream=None) -> torch.Tensor:
+    """D = A * B^T with A stored [K, M] (M % 16 == 0) and B [N, K]."""
+    return _fp8_gemm_layout("dg_fp8_gemm_tt", True, False, a, sfa, b, sfb, d, workspace, stream)
+
+
 def dg_fp8_gemm_nt_accumulate(a, sfa, b, sfb, c, d, workspace: torch.Tensor | None = None,
                               stream=None) -> torch.Tensor:
     """D = C + A * B^T: as dg_fp8_gemm_nt, with c a float32 [M, N] tensor added
@@ -405,6 +516,33 @@ def dg_m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m,
         _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), _ptr(d),
         _ptr(masked_m), g, m_max, n, k, _stream(stream))
     _check(rc, "dg_m_grouped_fp8_gemm_nt_masked")
+    return d
+
+
+def dg_k_grouped_fp8_gemm_tn_contiguous(a, sfa, b, sfb, d, k_sizes, c=None,
+                                        stream=None) -> torch.Tensor:
+    """The k-grouped GEMM with both operands stored with the token axis K
+    outermost: a [K, M], b [K, N] uint8 (M, N % 16 == 0), scales and the rest
+    as in dg_k_grouped_fp8_gemm_nt_contiguous."""
+    _need_cuda(a, sfa, b, sfb, d, k_sizes)
+    if c is not None:
+        _need_cuda(c)
+    k, m = a.shape
+    n = b.shape[1]
+    g = k_sizes.numel()
+    if k % 128 == 0:
+        _expect(a, "a", torch.uint8, (k, m))
+        _expect(sfa, "sfa", torch.float32, (k // 128, (m, "ld")))
+        _expect(b, "b", torch.uint8, (k, n))
+        _expect(sfb, "sfb", torch.float32, (k // 128, (n, "ld")))
+    _expect(d, "d", torch.float32, (g, m, n))
+    _expect(k_sizes, "k_sizes", torch.int32, (g,))
+    if c is not None:
+        _expect(c, "c", torch.float32, (g, m, n))
+    rc = load_library().dg_k_grouped_fp8_gemm_tn_contiguous(
+        _ptr(a), _ptr(sfa), sfa.shape[-1], _ptr(b), _ptr(sfb), sfb.shape[-1], _ptr(c),
+        _ptr(d), _ptr(k_sizes), g, m, n, k, _stream(stream))
+    _check(rc, "dg_k_grouped_fp8_gemm_tn_contiguous")
     return d
 
 

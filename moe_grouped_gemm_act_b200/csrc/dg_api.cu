@@ -147,6 +147,23 @@ int dg_quantize_1x128(const void *x, int x_dtype, int64_t batch, int64_t M, int6
                                reinterpret_cast<cudaStream_t>(stream), effective_num_sms());
 }
 
+int dg_quantize_128x1(const void *x, int x_dtype, int64_t K, int64_t M, int64_t ld_x,
+                      uint8_t *q, int64_t ld_q, float *sf, int64_t ld_sf, int flags,
+                      dg_stream_t stream) {
+  if (!x || !q || !sf) return DG_ERR_INVALID_ARG;
+  if (x_dtype != DG_DTYPE_F32 && x_dtype != DG_DTYPE_BF16) return DG_ERR_INVALID_ARG;
+  if (flags & ~DG_SCALE_POW2) return DG_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || K % 128 != 0) return DG_ERR_INVALID_ARG;
+  if (ld_x < M || ld_q < M || ld_sf < M) return DG_ERR_INVALID_ARG;
+  if (ld_sf % 4 != 0) return DG_ERR_ALIGNMENT;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(sf)) return DG_ERR_ALIGNMENT;
+  int rc = check_device();
+  if (rc) return rc;
+  if (M == 0) return DG_OK;
+  return launch_quantize_128x1(x, x_dtype, K, M, ld_x, q, ld_q, sf, ld_sf, flags,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
 int dg_quantize_128x128(const float *w, int64_t G, int64_t N, int64_t K, uint8_t *q,
                         float *sf, int flags, dg_stream_t stream) {
   if (!w || !q || !sf) return DG_ERR_INVALID_ARG;
@@ -189,6 +206,91 @@ int dg_fp8_gemm_nt(const uint8_t *A, const float *sfa, int64_t ld_sfa, const uin
   p.groups = 1;
   return launch_fp8_gemm(kDense, A, B, p, reinterpret_cast<cudaStream_t>(stream),
                          effective_num_sms(), workspace_bytes, workspace);
+}
+
+namespace {
+
+// D = A * B^T with A and B stored as `layout` says (the transposed forms keep
+// K outermost for the operand they transpose; its row stride, M or N bytes,
+// must be a multiple of 16 for the tensor memory accelerator).
+int fp8_gemm_layout(int layout, const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                    const uint8_t *B, const float *sfb, void *D, int64_t M, int64_t N, int64_t K,
+                    void *workspace, size_t workspace_bytes, dg_stream_t stream) {
+  int rc = check_gemm_common(A, sfa, ld_sfa, B, sfb, D, M, N, K);
+  if (rc) return rc;
+  if (a_mn_major(layout) && M % 16 != 0) return DG_ERR_ALIGNMENT;
+  if (b_mn_major(layout) && N % 16 != 0) return DG_ERR_ALIGNMENT;
+  if (workspace && !aligned16(workspace)) return DG_ERR_ALIGNMENT;
+  if (!workspace) workspace_bytes = 0;
+  rc = check_device();
+  if (rc) return rc;
+  if (M == 0) return DG_OK;
+  GemmParams p{};
+  p.status = device_info()->status;
+  p.sfa = sfa;
+  p.ld_sfa = ld_sfa;
+  p.sfb = sfb;
+  p.d = static_cast<uint16_t *>(D);
+  p.rows = static_cast<int>(M);
+  p.n = static_cast<int>(N);
+  p.k = static_cast<int>(K);
+  p.groups = 1;
+  return launch_fp8_gemm(kDense, A, B, p, reinterpret_cast<cudaStream_t>(stream),
+                         effective_num_sms(), workspace_bytes, workspace, layout);
+}
+
+}  // namespace
+
+int dg_fp8_gemm_nn(const uint8_t *A, const float *sfa, int64_t ld_sfa, const uint8_t *B,
+                   const float *sfb, void *D, int64_t M, int64_t N, int64_t K,
+                   void *workspace, size_t workspace_bytes, dg_stream_t stream) {
+  return fp8_gemm_layout(kLayoutNN, A, sfa, ld_sfa, B, sfb, D, M, N, K, workspace,
+                         workspace_bytes, stream);
+}
+
+int dg_fp8_gemm_tn(const uint8_t *A, const float *sfa, int64_t ld_sfa, const uint8_t *B,
+                   const float *sfb, void *D, int64_t M, int64_t N, int64_t K,
+                   void *workspace, size_t workspace_bytes, dg_stream_t stream) {
+  return fp8_gemm_layout(kLayoutTN, A, sfa, ld_sfa, B, sfb, D, M, N, K, workspace,
+                         workspace_bytes, stream);
+}
+
+int dg_fp8_gemm_tt(const uint8_t *A, const float *sfa, int64_t ld_sfa, const uint8_t *B,
+                   const float *sfb, void *D, int64_t M, int64_t N, int64_t K,
+                   void *workspace, size_t workspace_bytes, dg_stream_t stream) {
+  return fp8_gemm_layout(kLayoutTT, A, sfa, ld_sfa, B, sfb, D, M, N, K, workspace,
+                         workspace_bytes, stream);
+}
+
+int dg_fp8_gemm_nt_quantize(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                            const uint8_t *B, const float *sfb, uint8_t *Dq, float *sfd,
+                            int64_t ld_sfd, int64_t M, int64_t N, int64_t K, int flags,
+                            dg_stream_t stream) {
+  int rc = check_gemm_common(A, sfa, ld_sfa, B, sfb, Dq, M, N, K);
+  if (rc) return rc;
+  if (flags & ~DG_SCALE_POW2) return DG_ERR_INVALID_ARG;
+  if (N % 128 != 0) return DG_ERR_INVALID_ARG;
+  if (M > 0 && (!sfd || ld_sfd < M)) return DG_ERR_INVALID_ARG;
+  if (ld_sfd % 4 != 0) return DG_ERR_ALIGNMENT;
+  if (sfd && !aligned16(sfd)) return DG_ERR_ALIGNMENT;
+  rc = check_device();
+  if (rc) return rc;
+  if (M == 0) return DG_OK;
+  GemmParams p{};
+  p.status = device_info()->status;
+  p.sfa = sfa;
+  p.ld_sfa = ld_sfa;
+  p.sfb = sfb;
+  p.dq = Dq;
+  p.sfd = sfd;
+  p.ld_sfd = ld_sfd;
+  p.q_flags = flags;
+  p.rows = static_cast<int>(M);
+  p.n = static_cast<int>(N);
+  p.k = static_cast<int>(K);
+  p.groups = 1;
+  return launch_fp8_gemm(kDenseQuant, A, B, p, reinterpret_cast<cudaStream_t>(stream),
+                         effective_num_sms(), 0, nullptr);
 }
 
 int dg_fp8_gemm_nt_accumulate(const uint8_t *A, const float *sfa, int64_t ld_sfa,
@@ -270,13 +372,16 @@ int dg_m_grouped_fp8_gemm_nt_masked(const uint8_t *A, const float *sfa, int64_t 
                          effective_num_sms(), 0, nullptr);
 }
 
-int dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sfa, int64_t ld_sfa,
-                                        const uint8_t *B, const float *sfb, int64_t ld_sfb,
-                                        const float *C, float *D, const int32_t *k_sizes,
-                                        int G, int64_t M, int64_t N, int64_t K,
-                                        dg_stream_t stream) {
+namespace {
+
+int k_grouped(int layout, const uint8_t *A, const float *sfa, int64_t ld_sfa, const uint8_t *B,
+              const float *sfb, int64_t ld_sfb, const float *C, float *D,
+              const int32_t *k_sizes, int G, int64_t M, int64_t N, int64_t K,
+              dg_stream_t stream) {
   int rc = check_gemm_common(A, sfa, ld_sfa, B, sfb, D, M, N, K);
   if (rc) return rc;
+  if (a_mn_major(layout) && M % 16 != 0) return DG_ERR_ALIGNMENT;
+  if (b_mn_major(layout) && N % 16 != 0) return DG_ERR_ALIGNMENT;
   if (G < 1 || G > 1024) return DG_ERR_INVALID_ARG;
   if (M == 0) return DG_OK;
   if (!k_sizes || ld_sfb < N) return DG_ERR_INVALID_ARG;
@@ -298,7 +403,27 @@ int dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sfa, int6
   p.k = static_cast<int>(K);
   p.groups = G;
   return launch_fp8_gemm(kKGrouped, A, B, p, reinterpret_cast<cudaStream_t>(stream),
-                         effective_num_sms(), 0, nullptr);
+                         effective_num_sms(), 0, nullptr, layout);
+}
+
+}  // namespace
+
+int dg_k_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                                        const uint8_t *B, const float *sfb, int64_t ld_sfb,
+                                        const float *C, float *D, const int32_t *k_sizes,
+                                        int G, int64_t M, int64_t N, int64_t K,
+                                        dg_stream_t stream) {
+  return k_grouped(kLayoutNT, A, sfa, ld_sfa, B, sfb, ld_sfb, C, D, k_sizes, G, M, N, K,
+                   stream);
+}
+
+int dg_k_grouped_fp8_gemm_tn_contiguous(const uint8_t *A, const float *sfa, int64_t ld_sfa,
+                                        const uint8_t *B, const float *sfb, int64_t ld_sfb,
+                                        const float *C, float *D, const int32_t *k_sizes,
+                                        int G, int64_t M, int64_t N, int64_t K,
+                                        dg_stream_t stream) {
+  return k_grouped(kLayoutTN, A, sfa, ld_sfa, B, sfb, ld_sfb, C, D, k_sizes, G, M, N, K,
+                   stream);
 }
 
 namespace {

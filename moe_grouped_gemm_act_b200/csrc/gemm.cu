@@ -65,6 +65,7 @@
 #include "dg.h"
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_math.cuh"
 
 namespace dg {
 
@@ -112,6 +113,12 @@ static __device__ int g_starve_load_it = -1;
 // leaves).
 __host__ __device__ constexpr int staged_epilogue(int sched) {
   return sched == kDenseAcc ? 2 : (sched == kDense || sched == kMasked) ? 1 : 0;
+}
+
+// The staging kind an instance uses (every schedule, including the UE8M0
+// and quantizing forms).
+__host__ __device__ constexpr int instance_staging(int sched) {
+  return sched == kDenseQuant ? 0 : staged_epilogue(base_sched(sched));
 }
 
 // Scale-factor bytes per stage of the UE8M0 schedules: the K block's packed
@@ -272,7 +279,7 @@ __device__ __forceinline__ int masked_rows(const GemmParams &p, int e) {
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int BN, int STAGES, int NBUF, int SCHED>
+template <int BN, int STAGES, int NBUF, int SCHED, int LAYOUT = kLayoutNT>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
@@ -284,8 +291,18 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   constexpr bool kUE = is_ue8m0(SCHED);
   constexpr int S = base_sched(SCHED);
   static_assert(!kUE || NBUF == 1, "the UE8M0 schedules keep one accumulator per tile");
-  constexpr int kStaged = staged_epilogue(S);
-  constexpr bool kDenseLike = (S == kDense || S == kDenseAcc) && !kUE;
+  // operands stored with K outermost (T of A, N of B) are MN-major tiles in
+  // shared memory: K rows of 128 values, B in BN / 128 such columns
+  constexpr bool kAmn = a_mn_major(LAYOUT);
+  constexpr bool kBmn = b_mn_major(LAYOUT);
+  static_assert(LAYOUT == kLayoutNT || ((S == kDense || S == kDenseCluster || S == kKGrouped) &&
+                                         !kUE && (!kBmn || BN % 128 == 0)),
+                "transposed layouts serve the dense and k-grouped schedules");
+  // the quantizing epilogue writes each thread's row group itself
+  constexpr bool kQ = SCHED == kDenseQuant;
+  constexpr int kStaged = instance_staging(SCHED);
+  constexpr bool kDenseLike = (S == kDense || S == kDenseAcc) && !kUE && !kQ;
+  static_assert(!kQ || BN == 256, "the quantizing epilogue needs whole 128-column groups");
   constexpr bool kKG = S == kKGrouped;
   using L = Layout<BN, STAGES, NBUF, kStaged, kKG, kUE>;
   constexpr int W = BN / 2;                 // columns per promotion thread
@@ -471,18 +488,26 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (!mbar_wait(empty_bar(s), ph ^ 1, s_abort, p.status)) { alive = false; break; }
         if (lane == 0 && it != starve_it) {
           const uint32_t sa = base + s * L::kStageBytes;
+          // (the k-grouped form's B is one [N][K] tensor for all groups)
+          const int b_slab = kKG ? 0 : t.group;
+          mbar_arrive_expect_tx(full_bar(s), stage_tx + beta_bytes);
+          if constexpr (kAmn) {
+            tma_load_3d(sa, &tmap_a, full_bar(s), a_row, kb * BK, t.slab);
+          } else {
+            tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, t.slab);
+          }
+          if constexpr (kBmn) {
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              tma_load_3d(sa + kABytes + j * (BK * 128), &tmap_b, full_bar(s), b_row + 128 * j,
+                          kb * BK, b_slab);
+          } else {
+            tma_load_3d(sa + kABytes, &tmap_b, full_bar(s), kb * BK, b_row, b_slab);
+          }
           if constexpr (kKG) {
-            // B is one [N][K] tensor for all groups
-            mbar_arrive_expect_tx(full_bar(s), stage_tx + beta_bytes);
-            tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, 0);
-            tma_load_3d(sa + kABytes, &tmap_b, full_bar(s), kb * BK, b_row, 0);
             bulk_load(base + L::kBetaOff + static_cast<uint32_t>(it % L::kBetaSlots) * (BN * 4u),
                       p.sfb + static_cast<int64_t>(kb) * p.ld_sfb + b_col0, beta_bytes,
                       full_bar(s));
-          } else {
-            mbar_arrive_expect_tx(full_bar(s), stage_tx);
-            tma_load_3d(sa, &tmap_a, full_bar(s), kb * BK, a_row, t.slab);
-            tma_load_3d(sa + kABytes, &tmap_b, full_bar(s), kb * BK, b_row, t.group);
           }
         }
         if constexpr (kUE) {
@@ -573,7 +598,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
    } else {
     // ============================================================ MMA issuer
-    constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+    constexpr uint32_t idesc = idesc_e4m3_f32_major(BM, BN, kAmn, kBmn);
+    // advancing one 32-wide K slice: +32 bytes inside a K-major 128-byte row
+    // (+2 in the descriptor's 16-byte address field), or +32 rows of 128
+    // bytes of an MN-major tile (+256)
+    constexpr uint64_t kAStep = kAmn ? 256 : 2, kBStep = kBmn ? 256 : 2;
     int it = 0, acc_it = 0;
     bool alive = true;
     for (int u = u_first; u < units && alive; u += u_stride) {
@@ -591,15 +620,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         tc_fence_after();
         if (lane == 0) {
           const uint32_t sa = base + s * L::kStageBytes;
-          const uint64_t adesc = smem_desc_k128_sw128(sa);
-          const uint64_t bdesc = smem_desc_k128_sw128(sa + kABytes);
+          const uint64_t adesc = kAmn ? smem_desc_mn_sw128(sa, BK * 128)
+                                      : smem_desc_k128_sw128(sa);
+          const uint64_t bdesc = kBmn ? smem_desc_mn_sw128(sa + kABytes, BK * 128)
+                                      : smem_desc_k128_sw128(sa + kABytes);
           const uint32_t d = tmem_base + buf * BN;
 #pragma unroll
-          for (int k = 0; k < BK / 32; ++k) {
-            // +32 bytes along K inside the swizzled 128-byte row = +2 in the
-            // descriptor's 16-byte address field
-            umma_f8(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < BK / 32; ++k)
+            umma_f8(d, adesc + kAStep * k, bdesc + kBStep * k, idesc, k > 0 ? 1u : 0u);
           // publish the buffer first: the promotion is on the critical path,
           // the producer has STAGES - 1 blocks of slack
           umma_commit(tfull_bar(buf));
@@ -907,7 +935,36 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
         continue;  // one unit per CTA in this schedule
       }
-      if constexpr (!kStaged) {
+      if constexpr (kQ) {
+        // D quantized 1 x 128 along N: this thread's 128 columns are one
+        // group of its row.  As the 1x128 quantizer would do on the BF16
+        // result: round to BF16, amax, s = amax / 448 (or its power of two
+        // above), codes E4M3_RNE(x / s); the codes go out 16 bytes at a time
+        // and the scale to the MN-major [N/128][ld] layout (consecutive rows
+        // of a warp: one 128-byte store).
+        if (row_ok && col0 < p.n) {
+          float amax = 0.0f;
+#pragma unroll
+          for (int c = 0; c < W; ++c) {
+            acc[c] = __bfloat162float(__float2bfloat16_rn(acc[c]));
+            amax = fmaxf(amax, fabsf(acc[c]));
+          }
+          const float sc = group_scale(amax, p.q_flags);
+          const bool fast = sc >= kFastDivMin;
+          const float y = fast ? __frcp_rn(sc) : 0.0f;
+          uint8_t *qrow = p.dq + static_cast<int64_t>(row) * p.n + col0;
+#pragma unroll
+          for (int c = 0; c < W; c += 16) {
+            uint4 w;
+            w.x = encode4(acc + c, sc, y, fast);
+            w.y = encode4(acc + c + 4, sc, y, fast);
+            w.z = encode4(acc + c + 8, sc, y, fast);
+            w.w = encode4(acc + c + 12, sc, y, fast);
+            *reinterpret_cast<uint4 *>(qrow + c) = w;
+          }
+          p.sfd[static_cast<int64_t>(col0 / 128) * p.ld_sfd + row] = sc;
+        }
+      } else if constexpr (!kStaged) {
         // each thread stores its row segment (valid rows), 16 bytes at a time
         if (row_ok) {
           uint16_t *drow = p.d + (static_cast<int64_t>(t.slab) * p.rows + row) * p.n;
@@ -1115,12 +1172,12 @@ bool print_configs() {
   return e && *e && *e != '0';
 }
 
-template <int BN, int STAGES, int NBUF, int SCHED>
+template <int BN, int STAGES, int NBUF, int SCHED, int LAYOUT = kLayoutNT>
 int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                     int grid, int extra_smem, cudaStream_t stream, bool coop) {
-  const int smem = smem_bytes_for<BN, STAGES, NBUF, staged_epilogue(base_sched(SCHED)),
+  const int smem = smem_bytes_for<BN, STAGES, NBUF, instance_staging(SCHED),
                                   SCHED == kKGrouped, is_ue8m0(SCHED)>(extra_smem);
-  auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED>;
+  auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED, LAYOUT>;
   static int configured_smem[64] = {0};  // per device; grows only
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DG_ERR_CUDA;
@@ -1248,6 +1305,30 @@ int max_smem_per_block() {
   return v;
 }
 
+// The transposed layouts: tiles 256 or 128 wide (a whole number of
+// 128-value MN-major columns of B).
+template <int SCHED, int LAYOUT>
+int dispatch_layout(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+                    int grid, int extra, cudaStream_t st) {
+  const bool coop = p.splits > 1 && SCHED != kDenseCluster;
+  switch (bn) {
+    case 256: return launch_instance<256, 4, 2, SCHED, LAYOUT>(ta, tb, p, grid, extra, st, coop);
+    case 128: return launch_instance<128, 6, 4, SCHED, LAYOUT>(ta, tb, p, grid, extra, st, coop);
+    default: return DG_ERR_INVALID_ARG;
+  }
+}
+
+template <int SCHED>
+int dispatch_any_layout(int layout, int bn, const CUtensorMap &ta, const CUtensorMap &tb,
+                        const GemmParams &p, int grid, int extra, cudaStream_t st) {
+  switch (layout) {
+    case kLayoutNN: return dispatch_layout<SCHED, kLayoutNN>(bn, ta, tb, p, grid, extra, st);
+    case kLayoutTN: return dispatch_layout<SCHED, kLayoutTN>(bn, ta, tb, p, grid, extra, st);
+    case kLayoutTT: return dispatch_layout<SCHED, kLayoutTT>(bn, ta, tb, p, grid, extra, st);
+    default: return DG_ERR_INVALID_ARG;
+  }
+}
+
 template <int SCHED>
 int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
              int grid, int extra, cudaStream_t st) {
@@ -1257,6 +1338,8 @@ int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmPar
   if constexpr (is_ue8m0(SCHED)) {
     return launch_instance<kUECandidate.bn, kUECandidate.stages, kUECandidate.nbuf, SCHED>(
         ta, tb, p, grid, extra, st, false);
+  } else if constexpr (SCHED == kDenseQuant) {
+    return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st, false);
   } else {
     switch (bn) {
       case 256: return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st, coop);
@@ -1287,6 +1370,26 @@ int make_tmap(CUtensorMap *m, const void *ptr, int64_t k, int64_t rows, int64_t 
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
+
+// 3-D tensor map over an E4M3 tensor stored [dim2][K][rows] (K outermost
+// within a slab: an MN-major operand) with a box of [1][128][128] (128 K rows
+// of 128 values) and the 128-byte swizzle.  rows % 16 == 0 (the row stride of
+// a TMA tensor is a multiple of 16 bytes).
+int make_tmap_mn(CUtensorMap *m, const void *ptr, int64_t rows, int64_t k, int64_t slabs) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return DG_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(k),
+                              static_cast<cuuint64_t>(slabs)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(rows),
+                                 static_cast<cuuint64_t>(rows * k)};
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(BK), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
 
 // Cycles one CTA spends per 128-K block of a unit, measured on B200.  The
 // tensor cores take ~540 cycles per block for any N up to 256 (one
@@ -1341,7 +1444,8 @@ double estimate_tail(int64_t waves, int64_t k, int bn, int s) {
 // (`ws_bytes`).  Tile forms whose shared memory (with `extra` bytes of
 // masked prefix tables) exceeds `max_smem` are skipped.
 Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, int num_sms,
-                     size_t ws_bytes, int extra = 0, int max_smem = 232448) {
+                     size_t ws_bytes, int extra = 0, int max_smem = 232448,
+                     int layout = kLayoutNT) {
   const int64_t m_blocks = (rows + BM - 1) / BM;
   const int64_t k_blocks = k / BK;
   const int64_t m_blocks_eff =
@@ -1350,6 +1454,8 @@ Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, 
   double best = 1e300;
   for (const Candidate &cand : kCandidates) {
     if (config_smem(cand.bn, extra, sched) > max_smem) continue;
+    // transposed layouts: whole 128-value MN-major columns of B
+    if (layout != kLayoutNT && cand.bn % 128 != 0) continue;
     const int64_t tiles = m_blocks * ((n + cand.bn - 1) / cand.bn);
     for (int s = 1; s <= 16; ++s) {
       if (s > 1 && (sched != kDense || m_blocks > 2)) break;
@@ -1383,10 +1489,17 @@ Choice choose_config(int sched, int64_t rows, int64_t n, int64_t k, int groups, 
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int num_sms) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   // the split the heuristic picks when the workspace is not a constraint
-  const Choice c = choose_config(kDense, M, N, K, 1, num_sms, ~static_cast<size_t>(0));
-  if (c.splits <= 1) return 0;
-  const int64_t tiles = ((M + BM - 1) / BM) * ((N + c.bn - 1) / c.bn) - c.full_tiles;
-  return (split_ws_bytes(tiles, c.splits, c.bn) + 255) & ~static_cast<size_t>(255);
+  // the larger of the splits the NT layout and the transposed layouts (tiles
+  // of 128 or 256 only) prefer
+  size_t need = 0;
+  for (int layout : {kLayoutNT, kLayoutTN}) {
+    const Choice c = choose_config(kDense, M, N, K, 1, num_sms, ~static_cast<size_t>(0), 0,
+                                   232448, layout);
+    if (c.splits <= 1) continue;
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + c.bn - 1) / c.bn) - c.full_tiles;
+    need = std::max(need, split_ws_bytes(tiles, c.splits, c.bn));
+  }
+  return need == 0 ? 0 : (need + 255) & ~static_cast<size_t>(255);
 }
 
 // Test knobs of the abort path (both unset in normal use):
@@ -1423,22 +1536,28 @@ static int set_test_knobs(const TestKnobs &k, cudaStream_t stream) {
 }
 
 static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
-                         cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws);
+                                cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws,
+                                int layout);
 
 int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
-                    cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws) {
+                    cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws, int layout) {
   const TestKnobs knobs = test_knobs();
-  if (!knobs.on) return launch_fp8_gemm_impl(sched, A, B, p, stream, num_sms, ws_bytes, ws);
+  if (!knobs.on)
+    return launch_fp8_gemm_impl(sched, A, B, p, stream, num_sms, ws_bytes, ws, layout);
   int rc = set_test_knobs(knobs, stream);
   if (rc) return rc;
-  rc = launch_fp8_gemm_impl(sched, A, B, p, stream, num_sms, ws_bytes, ws);
+  rc = launch_fp8_gemm_impl(sched, A, B, p, stream, num_sms, ws_bytes, ws, layout);
   const int rc2 = set_test_knobs(TestKnobs{}, stream);
   return rc ? rc : rc2;
 }
 
 static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
-                         cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws) {
+                                cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws,
+                                int layout) {
   const int64_t rows = p.rows, n = p.n, k = p.k;
+  // transposed layouts: the plain dense GEMM (no C) and the k-grouped GEMM
+  if (layout != kLayoutNT && !(sched == kKGrouped || (sched == kDense && p.c == nullptr)))
+    return DG_ERR_INVALID_ARG;
   p.num_k_blocks = static_cast<int>(k / BK);
   if (ws == nullptr) ws_bytes = 0;
 
@@ -1474,8 +1593,27 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
     return masked ? dispatch<kMaskedUE8M0>(bn, ta, tb, p, grid, extra, stream)
                   : dispatch<kDenseUE8M0>(bn, ta, tb, p, grid, extra, stream);
   }
+  if (sched == kDenseQuant) {
+    // whole 128-column groups per thread: 256-wide tiles, K never split (a
+    // split tile's reduction spreads a row's group over several threads)
+    const int bn = 256;
+    p.num_m_blocks = static_cast<int>((rows + BM - 1) / BM);
+    p.num_n_blocks = static_cast<int>((n + bn - 1) / bn);
+    p.splits = 1;
+    p.full_tiles = 0;
+    p.ws = nullptr;
+    p.a_box_rows = rows <= BM / 2 ? BM / 2 : BM;
+    CUtensorMap ta, tb;
+    int rc = make_tmap(&ta, A, k, rows, 1, p.a_box_rows);
+    if (rc) return rc;
+    rc = make_tmap(&tb, B, k, n, 1, bn);
+    if (rc) return rc;
+    const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
+    return dispatch<kDenseQuant>(bn, ta, tb, p, grid, extra, stream);
+  }
   const Choice choice =
-      choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes, extra, max_smem);
+      choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes, extra, max_smem, layout);
   int bn = choice.bn, splits = choice.splits;
   int64_t full_tiles = choice.full_tiles;
   bool splits_forced = false;  // DG_SPLITS: exactly this many, or none
@@ -1489,7 +1627,7 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
   if (const char *e = getenv("DG_BLOCK_N")) {
     const int v = atoi(e);
     for (const Candidate &c : kCandidates)
-      if (c.bn == v && v != bn) {
+      if (c.bn == v && v != bn && (layout == kLayoutNT || v % 128 == 0)) {
         bn = v;
         splits = 1;  // the split chosen for another width does not carry over
         full_tiles = 0;
@@ -1558,10 +1696,14 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
 
   // ------------------------------------------------ tensor maps
   CUtensorMap ta, tb;
-  p.a_box_rows = (sched == kDense && rows <= BM / 2) ? BM / 2 : BM;
-  int rc = make_tmap(&ta, A, k, rows, sched == kMasked ? p.groups : 1, p.a_box_rows);
+  p.a_box_rows = (sched == kDense && rows <= BM / 2 && !a_mn_major(layout)) ? BM / 2 : BM;
+  int rc = a_mn_major(layout)
+               ? make_tmap_mn(&ta, A, rows, k, 1)
+               : make_tmap(&ta, A, k, rows, sched == kMasked ? p.groups : 1, p.a_box_rows);
   if (rc) return rc;
-  rc = make_tmap(&tb, B, k, n, (sched == kDense || sched == kKGrouped) ? 1 : p.groups, bn);
+  rc = b_mn_major(layout)
+           ? make_tmap_mn(&tb, B, n, k, 1)
+           : make_tmap(&tb, B, k, n, (sched == kDense || sched == kKGrouped) ? 1 : p.groups, bn);
   if (rc) return rc;
 
   // ------------------------------------------------ grid
@@ -1586,7 +1728,9 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
       if (sc < chosen && all_tiles * sc * 5 < static_cast<int64_t>(num_sms) * 3) break;
       p.splits = sc;
       grid = static_cast<int>(all_tiles * sc);
-      rc = dispatch<kDenseCluster>(bn, ta, tb, p, grid, extra, stream);
+      rc = layout == kLayoutNT
+               ? dispatch<kDenseCluster>(bn, ta, tb, p, grid, extra, stream)
+               : dispatch_any_layout<kDenseCluster>(layout, bn, ta, tb, p, grid, extra, stream);
     }
     if (rc == kClusterNoFit) {
       p.splits = chosen;
@@ -1614,11 +1758,19 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
   }
   switch (sched) {
     case kDense:
+      if (layout != kLayoutNT)
+        return dispatch_any_layout<kDense>(layout, bn, ta, tb, p, grid, extra, stream);
       return acc ? dispatch<kDenseAcc>(bn, ta, tb, p, grid, extra, stream)
                  : dispatch<kDense>(bn, ta, tb, p, grid, extra, stream);
     case kContiguous: return dispatch<kContiguous>(bn, ta, tb, p, grid, extra, stream);
     case kMasked: return dispatch<kMasked>(bn, ta, tb, p, grid, extra, stream);
-    case kKGrouped: return dispatch<kKGrouped>(bn, ta, tb, p, grid, extra, stream);
+    case kKGrouped:
+      // the k-grouped form's transposed variant is TN (both operands stored
+      // with the token axis K outermost)
+      if (layout == kLayoutTN)
+        return dispatch_layout<kKGrouped, kLayoutTN>(bn, ta, tb, p, grid, extra, stream);
+      if (layout != kLayoutNT) return DG_ERR_INVALID_ARG;
+      return dispatch<kKGrouped>(bn, ta, tb, p, grid, extra, stream);
     default: return DG_ERR_INVALID_ARG;
   }
 }

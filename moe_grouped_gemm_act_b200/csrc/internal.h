@@ -16,6 +16,10 @@ int launch_quantize_1x128(const void *x, int x_dtype, int64_t batch, int64_t M,
                           float *sf, int64_t ld_sf, int flags,
                           cudaStream_t stream, int num_sms);
 
+int launch_quantize_128x1(const void *x, int x_dtype, int64_t K, int64_t M, int64_t ld_x,
+                          uint8_t *q, int64_t ld_q, float *sf, int64_t ld_sf, int flags,
+                          cudaStream_t stream);
+
 int launch_quantize_128x128(const float *w, int64_t G, int64_t N, int64_t K,
                             uint8_t *q, float *sf, int flags,
                             cudaStream_t stream);
@@ -42,14 +46,32 @@ inline cudaLaunchAttribute pdl_attribute() {
 // scales given as packed UE8M0 codes, applied by the tensor cores
 // (block-scaled MMA): the tile accumulates in TMEM over all of K and the
 // promotion warps only drain it for the epilogue.
+// kDenseQuant: dense tiles whose epilogue quantizes D: each row's 128-column
+// groups go out as E4M3 codes with one FP32 scale, as the 1x128 quantizer
+// would write them from the BF16 result.
 enum Sched : int {
   kDense = 0, kContiguous = 1, kMasked = 2, kDenseCluster = 3, kDenseAcc = 4, kKGrouped = 5,
-  kDenseUE8M0 = 6, kMaskedUE8M0 = 7
+  kDenseUE8M0 = 6, kMaskedUE8M0 = 7, kDenseQuant = 8
 };
+
+// Operand layouts of D = A * B^T ("DeepGEMM architecture deep dive",
+// section 3: sm_100 supports NT, TN, NN and TT).  The letters say how A and B
+// are used: N as stored, T transposed.  NT: A [M][K], B [N][K] (both
+// K-major); NN: B stored [K][N]; TN: A [K][M] and B [K][N]; TT: A [K][M].
+// An operand stored with K outermost is MN-major in shared memory.
+enum Layout : int { kLayoutNT = 0, kLayoutNN = 1, kLayoutTN = 2, kLayoutTT = 3 };
+__host__ __device__ constexpr bool a_mn_major(int layout) {
+  return layout == kLayoutTN || layout == kLayoutTT;
+}
+__host__ __device__ constexpr bool b_mn_major(int layout) {
+  return layout == kLayoutNN || layout == kLayoutTN;
+}
 
 // The tile schedule (work list, row validity, epilogue) a schedule follows.
 __host__ __device__ constexpr int base_sched(int sched) {
-  return sched == kDenseUE8M0 ? kDense : sched == kMaskedUE8M0 ? kMasked : sched;
+  return (sched == kDenseUE8M0 || sched == kDenseQuant) ? kDense
+         : sched == kMaskedUE8M0                        ? kMasked
+                                                        : sched;
 }
 __host__ __device__ constexpr bool is_ue8m0(int sched) {
   return sched == kDenseUE8M0 || sched == kMaskedUE8M0;
@@ -71,9 +93,13 @@ struct GemmParams {
   union {
     uint16_t *d;         // BF16 output [slab][rows][N]
     float *d_f32;        // k-grouped: FP32 output [group][rows][N]
+    uint8_t *dq;         // quantizing epilogue: E4M3 codes [rows][N]
   };
-  const float *c;        // dense D = C + A B^T: FP32 C [rows][N]; k-grouped:
+  union {
+    const float *c;      // dense D = C + A B^T: FP32 C [rows][N]; k-grouped:
                          // [group][rows][N] (nullptr: none)
+    float *sfd;          // quantizing epilogue: MN-major scales [N/128][ld_sfd]
+  };
   const int32_t *m_indices;  // contiguous: expert per row (-1 = padding)
   union {
     const int32_t *masked_m;  // masked: valid rows per expert
@@ -84,6 +110,7 @@ struct GemmParams {
   union {
     uint32_t *ws_ticket;  // split-K arrival counters, one per output tile
     int64_t ld_sfb;       // k-grouped and UE8M0: row stride of the B scales
+    int64_t ld_sfd;       // quantizing epilogue: row stride of D's scales
   };
   int rows;              // dense: M; contiguous: M_total; masked: M_max
   int n, k;
@@ -95,6 +122,7 @@ struct GemmParams {
   int full_tiles;        // dense: tiles (in raster order) computed whole before
                          // the remaining ones, each split `splits` ways
   int a_box_rows;        // rows of A per TMA load: 128, or 64 when M <= 64
+  int q_flags;           // quantizing epilogue: DG_SCALE_FP32 or DG_SCALE_POW2
 };
 
 struct GemmConfig {
@@ -106,9 +134,11 @@ struct GemmConfig {
 };
 
 // Host entry of the GEMM: picks a config, encodes tensor maps, launches.
+// `layout` (kLayoutNT .. kLayoutTT) selects how A and B are stored; layouts
+// other than NT serve the dense and k-grouped schedules.
 int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B,
                     GemmParams p, cudaStream_t stream, int num_sms,
-                    size_t ws_bytes, void *ws);
+                    size_t ws_bytes, void *ws, int layout = kLayoutNT);
 
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int num_sms);
 

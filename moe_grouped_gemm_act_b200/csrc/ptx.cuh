@@ -406,6 +406,23 @@ __device__ __forceinline__ uint64_t smem_desc_k128_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile written by TMA
+// with the 128-byte swizzle: each K row holds 128 bytes (128 FP8 values) of
+// M or N, 8 consecutive K rows form a 1024-byte swizzle atom (stride byte
+// offset 1024 between atoms along K), and a tile wider than 128 values is
+// several such 128-wide columns `lbo` bytes apart (leading byte offset).
+// Advancing along K by 32 rows adds 4096 bytes to the start address.  The
+// tile base must be 1024-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);      // start address
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;   // leading byte offset
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;             // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                     // version
+  d |= static_cast<uint64_t>(2) << 61;                     // 128-byte swizzle
+  return d;
+}
+
 // Shared-memory descriptor of a no-swizzle K-major source whose rows are 16
 // bytes, stored contiguously (8-row core matrices of 128 bytes, one after
 // the other): the source of tcgen05.cp's 32x128b shape.  Stride byte offset
@@ -427,6 +444,12 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {
          (0u << 7) | (0u << 10) |                   // A, B: E4M3
          (static_cast<uint32_t>(n >> 3) << 17) |    // N / 8
          (static_cast<uint32_t>(m >> 4) << 24);     // M / 16
+}
+
+// The same with the operands' majorness: bit 15 set when A is MN-major (its
+// shared-memory tile holds K rows of M values), bit 16 when B is.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32_major(int m, int n, bool a_mn, bool b_mn) {
+  return idesc_e4m3_f32(m, n) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
 }
 
 // Instruction descriptor of the block-scaled kind::mxf8f6f4: A and B E4M3

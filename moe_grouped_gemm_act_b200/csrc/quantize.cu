@@ -30,65 +30,11 @@
 #include "dg.h"
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_math.cuh"
 
 namespace dg {
 
 namespace {
-
-constexpr float kE4M3Max = 448.0f;
-constexpr float kFastDivMin = 7.8886090522101181e-31f;  // 2^-100
-
-// Smallest power of two >= a (a >= 0, finite), from the FP32 bits.
-__device__ __forceinline__ float pow2_round_up(float a) {
-  const uint32_t b = __float_as_uint(a);
-  const uint32_t e = (b >> 23) & 0xFFu, m = b & 0x7FFFFFu;
-  if (m == 0) return a;  // zero or already a power of two
-  if (e != 0) return __uint_as_float((e + 1u) << 23);
-  // subnormal: next power of two of the mantissa field (may reach 2^-126)
-  return __uint_as_float(1u << (32 - __clz(m - 1u)));
-}
-
-__device__ __forceinline__ float group_scale(float amax, int flags) {
-  float s = __fdiv_rn(amax, kE4M3Max);
-  if (flags & DG_SCALE_POW2) s = pow2_round_up(s);
-  return s;
-}
-
-// RN(x / s) from y = RN(1/s); valid for s >= 2^-100 (see the file comment).
-__device__ __forceinline__ float div_by_scale(float x, float s, float y) {
-  const float q0 = x * y;
-  const float q1 = fmaf(fmaf(-s, q0, x), y, q0);
-  return fmaf(fmaf(-s, q1, x), y, q1);
-}
-
-// Four E4M3 codes of the quotients q[0..3], little-endian in 32 bits.  The
-// sign of each code is taken from the dividend v (the scale is positive), so
-// values that round to zero, -0.0 included, keep their sign.
-__device__ __forceinline__ uint32_t pack_codes(const float q[4], const float v[4]) {
-  const uint32_t lo =
-      __nv_cvt_float2_to_fp8x2(make_float2(q[0], q[1]), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t hi =
-      __nv_cvt_float2_to_fp8x2(make_float2(q[2], q[3]), __NV_SATFINITE, __NV_E4M3);
-  // top byte of each dividend (sign + 7 exponent bits), masked to the sign
-  const uint32_t t01 = __byte_perm(__float_as_uint(v[0]), __float_as_uint(v[1]), 0x73);
-  const uint32_t t23 = __byte_perm(__float_as_uint(v[2]), __float_as_uint(v[3]), 0x73);
-  const uint32_t signs = __byte_perm(t01, t23, 0x5410) & 0x80808080u;
-  return (lo | (hi << 16)) | signs;
-}
-
-// Codes of v[0..3] divided by the group scale.
-__device__ __forceinline__ uint32_t encode4(const float v[4], float s, float y, bool fast) {
-  if (s == 0.0f) return 0u;  // all-zero group
-  float q[4];
-  if (fast) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = div_by_scale(v[i], s, y);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = __fdiv_rn(v[i], s);
-  }
-  return pack_codes(q, v);
-}
 
 template <typename T>
 __device__ __forceinline__ void load4(const T *p, float v[4]);
@@ -159,6 +105,50 @@ quantize_1x128_kernel(const T *__restrict__ x, int64_t batch, int64_t M, int64_t
       sf[(b * Kg + g) * ld_sf + r] = s;
     }
   }
+}
+
+// Groups of 128 rows of one column: x stored [K][M] (M contiguous), the group
+// of column m and K group g is x[128 g .. 128 g + 127][m] -- the 1 x 128
+// groups along K of an operand stored with K outermost.  Each thread owns one
+// column of one group: it loads the group's 128 values into registers (a warp
+// reads 32 consecutive columns of a row: one 128-byte line for FP32), takes
+// their amax, and writes the codes back row by row and the scale to
+// sf[g][m] (MN-major).
+template <typename T>
+__global__ void __launch_bounds__(128)
+quantize_128x1_kernel(const T *__restrict__ x, int64_t M, int64_t ld_x, uint8_t *__restrict__ q,
+                      int64_t ld_q, float *__restrict__ sf, int64_t ld_sf, int flags) {
+  grid_launch_dependents();
+  grid_dependency_wait();
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t g = blockIdx.y;
+  if (m >= M) return;
+  const T *src = x + g * 128 * ld_x + m;
+  float v[128];
+  float a = 0.0f;
+#pragma unroll
+  for (int r = 0; r < 128; ++r) {
+    if constexpr (sizeof(T) == 4) {
+      v[r] = __ldcs(reinterpret_cast<const float *>(src) + r * ld_x);
+    } else {
+      v[r] = __uint_as_float(static_cast<uint32_t>(
+                 __ldcs(reinterpret_cast<const unsigned short *>(src) + r * ld_x)) << 16);
+    }
+    a = fmaxf(a, fabsf(v[r]));
+  }
+  const float s = group_scale(a, flags);
+  const bool fast = s >= kFastDivMin;
+  const float y = fast ? __frcp_rn(s) : 0.0f;
+  uint8_t *dst = q + g * 128 * ld_q + m;
+#pragma unroll
+  for (int r = 0; r < 128; r += 4) {
+    const uint32_t w = encode4(v + r, s, y, fast);
+    dst[(r + 0) * ld_q] = static_cast<uint8_t>(w);
+    dst[(r + 1) * ld_q] = static_cast<uint8_t>(w >> 8);
+    dst[(r + 2) * ld_q] = static_cast<uint8_t>(w >> 16);
+    dst[(r + 3) * ld_q] = static_cast<uint8_t>(w >> 24);
+  }
+  sf[g * ld_sf + m] = s;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -240,6 +230,30 @@ int launch_quantize_1x128(const void *x, int x_dtype, int64_t batch, int64_t M, 
     e = cudaLaunchKernelEx(&cfg, quantize_1x128_kernel<__nv_bfloat16>,
                            static_cast<const __nv_bfloat16 *>(x), batch, M, Kg, ld_x, q, ld_q, sf,
                            ld_sf, flags);
+  }
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
+int launch_quantize_128x1(const void *x, int x_dtype, int64_t K, int64_t M, int64_t ld_x,
+                          uint8_t *q, int64_t ld_q, float *sf, int64_t ld_sf, int flags,
+                          cudaStream_t stream) {
+  const int64_t blocks_x = (M + 127) / 128;
+  if (blocks_x > 0x7FFFFFFF || K / 128 > 65535) return DG_ERR_INVALID_ARG;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks_x), static_cast<unsigned>(K / 128));
+  cfg.blockDim = dim3(128);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (x_dtype == DG_DTYPE_F32) {
+    e = cudaLaunchKernelEx(&cfg, quantize_128x1_kernel<float>, static_cast<const float *>(x), M,
+                           ld_x, q, ld_q, sf, ld_sf, flags);
+  } else {
+    e = cudaLaunchKernelEx(&cfg, quantize_128x1_kernel<__nv_bfloat16>,
+                           static_cast<const __nv_bfloat16 *>(x), M, ld_x, q, ld_q, sf, ld_sf,
+                           flags);
   }
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
