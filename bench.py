@@ -157,6 +157,27 @@ def workload_spec(name: str) -> dict:
                     desc="m-grouped masked, G=32, M_max=256, N=7168 K=2048, "
                          "masked_m ~ U{0..256}, every scale rounded up to a power of two "
                          "(UE8M0-representable)")
+    if name == "masked_ue8m0":
+        return dict(name=name, kind="masked", bound="hbm", pow2=True, ue8m0=True,
+                    **inputs.MASKED,
+                    desc="m-grouped masked, G=32, M_max=256, N=7168 K=2048, "
+                         "masked_m ~ U{0..256}, power-of-two scales as packed UE8M0 words "
+                         "applied by the tensor cores (block-scaled MMA)")
+    if name == "prefill_quant":
+        # the prefill shapes whose N is a whole number of 128-wide groups (an
+        # output quantized 1x128 is the next GEMM's A, whose K must be)
+        return dict(name=name, kind="dense", m=inputs.PREFILL_M,
+                    nk=[nk for nk in inputs.PREFILL_NK if nk[0] % 128 == 0],
+                    seeds=inputs.PREFILL_SEEDS, bound="tensor", quant_out=True,
+                    desc="dense NT prefill with the output quantized 1x128 in the epilogue "
+                         "(E4M3 codes + FP32 scales), M=4096, (N,K) in "
+                         "{(7168,16384),(4096,7168),(24576,1536)}; A, B and scales as prefill")
+    if name == "kgrouped_tn":
+        return dict(name=name, kind="kgrouped", bound="tensor", tn=True, **inputs.K_GROUPED,
+                    desc="k-grouped contiguous TN (MoE weight gradient, operands stored "
+                         "token-major: A [K, M], B [K, N]), G=8, M=4096 N=7168, 32768 "
+                         "tokens multinomial over experts along K, segments padded to 128; "
+                         "1x128-along-K FP32 scales on both, FP32 D[g] out")
     if name == "kgrouped":
         return dict(name=name, kind="kgrouped", bound="tensor", **inputs.K_GROUPED,
                     desc="k-grouped contiguous (MoE weight gradient), G=8, M=4096 N=7168, "
@@ -257,6 +278,7 @@ class DenseData:
         m = spec["m"]
         self.m = m
         self.acc = bool(spec.get("acc"))
+        self.quant_out = bool(spec.get("quant_out"))
         self.shapes = []
         gen = torch.Generator(device=device)
         for n, k in spec["nk"]:
@@ -267,7 +289,11 @@ class DenseData:
             ld = dg.dg_get_tma_aligned_size(m, 4)
             qa = torch.empty((m, k), dtype=torch.uint8, device=device)
             sfa = torch.empty((k // 128, ld), dtype=torch.float32, device=device)
-            d = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+            if self.quant_out:   # E4M3 codes and MN-major 1x128 scales of D
+                d = (torch.empty((m, n), dtype=torch.uint8, device=device),
+                     torch.empty((n // 128, ld), dtype=torch.float32, device=device))
+            else:
+                d = torch.empty((m, n), dtype=torch.bfloat16, device=device)
             wsb = dg.dg_fp8_gemm_nt_workspace_size(m, n, k)
             ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=device) if wsb else None
             c = None
@@ -285,8 +311,10 @@ class DenseData:
         """Algorithmic bytes of one shape's GEMM launch (A, alpha, B, beta, D,
         and C when accumulating)."""
         n, k = s["n"], s["k"]
+        out = (self.m * n + 4 * self.m * (n // 128)) if getattr(self, "quant_out", False) \
+            else 2 * self.m * n
         tot = self.m * k + 4 * self.m * (k // 128) + n * k + \
-            4 * (-(-n // 128)) * (k // 128) + 2 * self.m * n
+            4 * (-(-n // 128)) * (k // 128) + out
         if self.acc:
             tot += 4 * self.m * n  # C
         return tot
@@ -296,7 +324,10 @@ class DenseData:
         return sum(self.shape_bytes(s) for s in self.shapes)
 
     def gemm(self, s):
-        if self.acc:
+        if self.quant_out:
+            self.dg.dg_fp8_gemm_nt_quantize(s["qa"], s["sfa"], s["qb"], s["sfb"], dq=s["d"][0],
+                                            sfd=s["d"][1])
+        elif self.acc:
             self.dg.dg_fp8_gemm_nt_accumulate(s["qa"], s["sfa"], s["qb"], s["sfb"], s["c"], s["d"],
                                               workspace=s["ws"])
         else:
@@ -350,10 +381,13 @@ class DenseData:
                 a=torch.from_numpy(s["x_host"]).pin_memory(),
                 qb=s["qb"].cpu().pin_memory(), sfb=s["sfb"].cpu().pin_memory(),
                 c=None if s["c"] is None else s["c"].cpu().pin_memory(),
-                d=torch.empty(s["d"].shape, dtype=torch.bfloat16).pin_memory()))
+                d=tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in s["d"])
+                if self.quant_out else
+                torch.empty(s["d"].shape, dtype=torch.bfloat16).pin_memory()))
         self.h2d = sum(h["a"].numel() * 4 + h["qb"].numel() + h["sfb"].numel() * 4 +
                        (0 if h["c"] is None else h["c"].numel() * 4) for h in self.host)
-        self.d2h = sum(h["d"].numel() * 2 for h in self.host)
+        self.d2h = sum((sum(t.numel() * t.element_size() for t in h["d"]) if self.quant_out
+                        else h["d"].numel() * 2) for h in self.host)
 
     def e2e_step(self, device):
         dg = self.dg
@@ -362,6 +396,11 @@ class DenseData:
             qb = h["qb"].to(device, non_blocking=True)
             sfb = h["sfb"].to(device, non_blocking=True)
             qa, sfa = dg.dg_quantize_1x128(a)
+            if self.quant_out:
+                dg.dg_fp8_gemm_nt_quantize(qa, sfa, qb, sfb, dq=s["d"][0], sfd=s["d"][1])
+                for dst, src in zip(h["d"], s["d"]):
+                    dst.copy_(src, non_blocking=True)
+                continue
             if h["c"] is not None:
                 c = h["c"].to(device, non_blocking=True)
                 dg.dg_fp8_gemm_nt_accumulate(qa, sfa, qb, sfb, c, s["d"], workspace=s["ws"])
@@ -409,6 +448,11 @@ class GroupedData(DenseData):
         self.sample_src = GroupedOracleSample.source(spec, x, w, index.cpu().numpy())
         del w
         qa, sfa = dg.dg_quantize_1x128(a32, pow2=self.pow2)
+        # UE8M0: B's block scales packed once (weights); A's are packed
+        # every step after the quantizer
+        self.ue8m0 = bool(spec.get("ue8m0"))
+        self.pb = dg.dg_pack_ue8m0_128x128(sfb, n) if self.ue8m0 else None
+        self.pa = dg.dg_pack_ue8m0(sfa, qa.shape[-2]) if self.ue8m0 else None
         d = torch.empty(d_shape, dtype=torch.bfloat16, device=device)
         self.m = rows_valid
         self.active = active
@@ -423,11 +467,19 @@ class GroupedData(DenseData):
     def gemm_bytes(self) -> float:
         s = self.shapes[0]
         n, k, v = s["n"], s["k"], self.m
+        if getattr(self, "ue8m0", False):
+            # packed words: 4 K groups per int32, per row of A and of B
+            words = -(-(k // 128) // 4)
+            return (v * k + 4 * v * words + self.active * (n * k + 4 * n * words)
+                    + 2 * v * n + 4 * s["index"].numel())
         return (v * k + 4 * v * (k // 128) + self.active * (n * k + 4 * (-(-n // 128)) * (k // 128))
                 + 2 * v * n + 4 * s["index"].numel())
 
     def gemm(self, s):
-        if self.kind == "masked":
+        if self.ue8m0:
+            self.dg.dg_m_grouped_fp8_gemm_nt_masked_ue8m0(s["qa"], self.pa, s["qb"], self.pb,
+                                                          s["d"], s["index"])
+        elif self.kind == "masked":
             self.dg.dg_m_grouped_fp8_gemm_nt_masked(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"],
                                                     s["index"])
         else:
@@ -435,10 +487,16 @@ class GroupedData(DenseData):
                                                         s["d"], s["index"])
 
     def step(self):
-        """One pass of the hot path: quantize the activations, then GEMM."""
+        """One pass of the hot path: quantize the activations (and, for the
+        UE8M0 form, pack their scales), then GEMM."""
         s = self.shapes[0]
         self.dg.dg_quantize_1x128(s["a32"], pow2=self.pow2, q=s["qa"], sf=s["sfa"])
+        if self.ue8m0:
+            self.dg.dg_pack_ue8m0(s["sfa"], s["qa"].shape[-2], packed=self.pa)
         self.gemm(s)
+
+    def launches_per_step(self) -> int:
+        return 3 if self.ue8m0 else 2
 
     def make_host(self):
         s = self.shapes[0]
@@ -457,6 +515,12 @@ class GroupedData(DenseData):
         sfb = h["sfb"].to(device, non_blocking=True)
         index = h["index"].to(device, non_blocking=True)
         qa, sfa = self.dg.dg_quantize_1x128(a, pow2=self.pow2)
+        if self.ue8m0:
+            pa = self.dg.dg_pack_ue8m0(sfa, qa.shape[-2])
+            pb = self.dg.dg_pack_ue8m0_128x128(sfb, qb.shape[-2])
+            self.dg.dg_m_grouped_fp8_gemm_nt_masked_ue8m0(qa, pa, qb, pb, s["d"], index)
+            h["d"].copy_(s["d"], non_blocking=True)
+            return
         if self.kind == "masked":
             self.dg.dg_m_grouped_fp8_gemm_nt_masked(qa, sfa, qb, sfb, s["d"], index)
         else:
@@ -468,7 +532,9 @@ class KGroupedData(DenseData):
     """The MoE weight gradient: one step quantizes the activation gradient A
     [M, K] and the activations B [N, K] (1x128 along the token axis K), then
     runs the k-grouped GEMM into FP32 D [G, M, N].  FLOPs count the valid
-    tokens (not the padding of the segments)."""
+    tokens (not the padding of the segments).  The TN form stores both
+    operands token-major (A [K, M], B [K, N]), quantizes them with the
+    K-outermost quantizer and runs the TN k-grouped GEMM."""
 
     def __init__(self, spec, device):
         import torch
@@ -477,12 +543,17 @@ class KGroupedData(DenseData):
         a, b, lay = KGroupedOracleSample.generate(spec)
         self.sample_src = KGroupedOracleSample.source(a, b)
         G, m, n, k = spec["groups"], spec["m"], spec["n"], lay.k_total
-        a32 = torch.from_numpy(a).to(device)
-        b32 = torch.from_numpy(b).to(device)
-        qa = torch.empty((m, k), dtype=torch.uint8, device=device)
+        self.tn = bool(spec.get("tn"))
+        if self.tn:   # token-major storage (set-up, untimed)
+            a32 = torch.from_numpy(np.ascontiguousarray(a.T)).to(device)
+            b32 = torch.from_numpy(np.ascontiguousarray(b.T)).to(device)
+        else:
+            a32 = torch.from_numpy(a).to(device)
+            b32 = torch.from_numpy(b).to(device)
+        qa = torch.empty(tuple(a32.shape), dtype=torch.uint8, device=device)
         sfa = torch.empty((k // 128, dg.dg_get_tma_aligned_size(m, 4)), dtype=torch.float32,
                           device=device)
-        qb = torch.empty((n, k), dtype=torch.uint8, device=device)
+        qb = torch.empty(tuple(b32.shape), dtype=torch.uint8, device=device)
         sfb = torch.empty((k // 128, dg.dg_get_tma_aligned_size(n, 4)), dtype=torch.float32,
                           device=device)
         d = torch.empty((G, m, n), dtype=torch.float32, device=device)
@@ -492,7 +563,8 @@ class KGroupedData(DenseData):
         self.k_total = k
         tokens = int(lay.counts.sum())
         self.shapes = [dict(n=n, k=tokens, a32=a32, b32=b32, qa=qa, sfa=sfa, qb=qb, sfb=sfb,
-                            d=d, k_sizes=ks, x_host=a, b_host=b, ws=None)]
+                            d=d, k_sizes=ks, x_host=a.T if self.tn else a,
+                            b_host=b.T if self.tn else b, ws=None)]
         torch.cuda.synchronize()
 
     def shape_bytes(self, s) -> float:
@@ -504,13 +576,19 @@ class KGroupedData(DenseData):
         return (m + n) * k + 4 * (m + n) * (k // 128) + 4 * self.groups * m * n + 4 * self.groups
 
     def gemm(self, s):
-        self.dg.dg_k_grouped_fp8_gemm_nt_contiguous(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"],
-                                                    s["k_sizes"])
+        f = (self.dg.dg_k_grouped_fp8_gemm_tn_contiguous if self.tn
+             else self.dg.dg_k_grouped_fp8_gemm_nt_contiguous)
+        f(s["qa"], s["sfa"], s["qb"], s["sfb"], s["d"], s["k_sizes"])
+
+    def quantize(self, x, q=None, sf=None):
+        if self.tn:
+            return self.dg.dg_quantize_128x1(x, q=q, sf=sf)
+        return self.dg.dg_quantize_1x128(x, q=q, sf=sf)
 
     def step(self):
         s = self.shapes[0]
-        self.dg.dg_quantize_1x128(s["a32"], q=s["qa"], sf=s["sfa"])
-        self.dg.dg_quantize_1x128(s["b32"], q=s["qb"], sf=s["sfb"])
+        self.quantize(s["a32"], q=s["qa"], sf=s["sfa"])
+        self.quantize(s["b32"], q=s["qb"], sf=s["sfb"])
         self.gemm(s)
 
     def launches_per_step(self) -> int:
@@ -534,9 +612,11 @@ class KGroupedData(DenseData):
         a = h["a"].to(device, non_blocking=True)
         b = h["b"].to(device, non_blocking=True)
         ks = h["k_sizes"].to(device, non_blocking=True)
-        qa, sfa = self.dg.dg_quantize_1x128(a)
-        qb, sfb = self.dg.dg_quantize_1x128(b)
-        self.dg.dg_k_grouped_fp8_gemm_nt_contiguous(qa, sfa, qb, sfb, s["d"], ks)
+        qa, sfa = self.quantize(a)
+        qb, sfb = self.quantize(b)
+        f = (self.dg.dg_k_grouped_fp8_gemm_tn_contiguous if self.tn
+             else self.dg.dg_k_grouped_fp8_gemm_nt_contiguous)
+        f(qa, sfa, qb, sfb, s["d"], ks)
         h["d"].copy_(s["d"], non_blocking=True)
 
 
@@ -579,6 +659,7 @@ class OracleSample:
         from oracle import quant as oq
         self.prepared = []
         self.acc = bool(spec.get("acc"))
+        self.quant_out = bool(spec.get("quant_out"))
         g = np.random.default_rng(spec["seeds"]["seed_a"])
         for n, k in spec["nk"]:
             x = inputs.activations(spec["m"], k, seed=spec["seeds"]["seed_a"] + k,
@@ -589,7 +670,8 @@ class OracleSample:
             cs = (g.standard_normal((rows, c)) * 4).astype(np.float32) if self.acc else None
             self.prepared.append((x[:rows].copy(), qb, beta, c, k, cs))
         self.desc = (f"{rows} rows of A x first {cols} columns of D per (N,K) pair, "
-                     f"full K" + (", D = C + A B^T" if self.acc else ""))
+                     f"full K" + (", D = C + A B^T" if self.acc else "") +
+                     (", D quantized 1x128" if self.quant_out else ""))
 
     def run(self) -> tuple[float, float]:
         """Returns (seconds, FLOPs) of one pass."""
@@ -598,7 +680,11 @@ class OracleSample:
         flops = 0.0
         for xs, qb, beta, c, k, cs in self.prepared:
             qa, alpha = oq.quantize_1x128(xs)
-            if cs is None:
+            if self.quant_out:
+                from oracle import bf16 as ob
+                d = ob.from_bits(og.fp8_gemm_nt(qa, alpha, qb, beta)).astype(np.float32)
+                oq.quantize_1x128(d)
+            elif cs is None:
                 og.fp8_gemm_nt(qa, alpha, qb, beta)
             else:
                 og.fp8_gemm_nt_accumulate(qa, alpha, qb, beta, cs)
@@ -807,7 +893,7 @@ def job_throughput(work_per_step: float, steps: int, world: int, ms: float) -> f
 
 
 ALL_WORKLOADS = ["prefill", "decode64", "decode128", "contiguous", "masked", "masked_pow2",
-                 "kgrouped", "prefill_acc"]
+                 "masked_ue8m0", "kgrouped", "kgrouped_tn", "prefill_acc", "prefill_quant"]
 
 
 def measure_workload(name: str, args, rank: int, world: int, device, cpu_secs: float) -> dict:

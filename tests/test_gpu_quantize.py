@@ -156,3 +156,21 @@ def test_quantize_rejects_bad_args():
     x = torch.zeros(4, 100, device="cuda")
     with pytest.raises(dg.DGError):
         dg.dg_quantize_1x128(x)          # K % 128 != 0
+
+
+# ------------------------------------------------ operands stored K outermost
+@pytest.mark.parametrize("pow2", [False, True])
+@pytest.mark.parametrize("k,m,dtype", [(256, 300, torch.float32), (1024, 64, torch.float32),
+                                       (384, 136, torch.bfloat16)])
+def test_128x1_is_the_1x128_quantizer_of_the_transpose(k, m, dtype, pow2):
+    # groups of 128 consecutive K elements of each column of x [K][M] -- the
+    # oracle's 1x128 quantizer on the logical [M][K] operand, bit for bit
+    x = inputs.activations(m, k, seed=k + m, outliers=True)
+    x[3, :128] = 0.0                       # an all-zero group
+    xd = torch.from_numpy(np.ascontiguousarray(x.T)).cuda().to(dtype)
+    xs = xd.float().cpu().numpy().T       # the values the device sees, [M][K]
+    q, sf = dg.dg_quantize_128x1(xd, pow2=pow2)
+    torch.cuda.synchronize()
+    q0, a0 = quant.quantize_1x128(np.ascontiguousarray(xs), pow2=pow2)
+    assert np.array_equal(q.cpu().numpy(), q0.T)
+    assert np.array_equal(sf.cpu().numpy()[:, :m], a0.T)
