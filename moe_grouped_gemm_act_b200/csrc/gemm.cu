@@ -131,9 +131,11 @@ constexpr uint32_t kSfStageBytes = kSfABytes + 1024;
 // (A) + 8 (B) columns, 16 apart.
 constexpr uint32_t kSfSlotCols = 16;
 
-template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false, bool UE = false>
+template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false, bool UE = false,
+          bool PAIR = false>
 struct Layout {
-  static constexpr uint32_t kBBytes = BN * BK;
+  // the 2-CTA form keeps half of the B tile (BN / 2 rows) in each CTA
+  static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   // With STAGED, staging of the output for coalesced stores: 128 rows x
   // kOutCols BF16 (kind 1: a 256-wide tile goes out in two column halves) or
@@ -145,8 +147,9 @@ struct Layout {
   static constexpr uint32_t kOutOff = STAGES * kStageBytes;
   static constexpr uint32_t kRowOkOff = kOutOff + (STAGED ? BM * kOutCols * kOutElem : 0);
   static constexpr uint32_t kBarOff = kRowOkOff + (STAGED ? BM : 0);
-  // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain epi
-  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
+  // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain epi, then (2-CTA form)
+  // pfull[S]: the peer's stage has landed
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2 + (PAIR ? STAGES : 0);
   static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
   static constexpr uint32_t kPrefixOff = kMiscOff + 16;
   // k-grouped: a ring of per-column B scale slices, one per K block in
@@ -301,10 +304,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // the quantizing epilogue writes each thread's row group itself
   constexpr bool kQ = SCHED == kDenseQuant;
   constexpr int kStaged = instance_staging(SCHED);
-  constexpr bool kDenseLike = (S == kDense || S == kDenseAcc) && !kUE && !kQ;
+  constexpr bool kDenseLike =
+      (S == kDense || S == kDenseAcc) && !kUE && !kQ && SCHED != kDensePair;
   static_assert(!kQ || BN == 256, "the quantizing epilogue needs whole 128-column groups");
   constexpr bool kKG = S == kKGrouped;
-  using L = Layout<BN, STAGES, NBUF, kStaged, kKG, kUE>;
+  // 2-CTA form: the cluster's two CTAs compute one 256-row tile
+  constexpr bool kPair = SCHED == kDensePair;
+  constexpr int TM = kPair ? 2 * BM : BM;   // rows per tile
+  static_assert(!kPair || (BN == 256 && LAYOUT == kLayoutNT), "the 2-CTA form: NT, 256 wide");
+  using L = Layout<BN, STAGES, NBUF, kStaged, kKG, kUE, kPair>;
   constexpr int W = BN / 2;                 // columns per promotion thread
   // BN = 256 runs with the warpgroup register split (promo_regs per promotion
   // thread), the narrower tiles fit the launch allocation as they are.  The
@@ -330,10 +338,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
   auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bars + 8u * (2 * STAGES + NBUF + b); };
-  const uint32_t drain_bar = bars + 8u * (L::kNumBars - 2);
+  const uint32_t drain_bar = bars + 8u * (2 * STAGES + 2 * NBUF);
   // synchronises the promotion threads in the epilogue (bounded, unlike a
   // named barrier, so that an aborting warp cannot strand the others)
-  const uint32_t epi_bar = bars + 8u * (L::kNumBars - 1);
+  const uint32_t epi_bar = drain_bar + 8u;
+  // 2-CTA form, rank 0: the peer's copy of stage s has landed
+  auto pfull_bar = [&](int s) { return epi_bar + 8u * (1 + s); };
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *s_flag = reinterpret_cast<int *>(smem + L::kMiscOff + 8);
@@ -342,8 +352,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int u_first = static_cast<int>(blockIdx.x);
-  const int u_stride = static_cast<int>(gridDim.x);
+  // 2-CTA form: rank 0 issues the pair's MMAs; units are per cluster
+  const uint32_t rank = kPair ? cluster_ctarank() : 0;
+  const int u_first = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int u_stride = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   // ---------------------------------------------------------------- setup
   // the next kernel of the stream may begin its own set-up as our CTAs leave
@@ -359,17 +371,26 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), kPromoWarps);
+      // 2-CTA form: the promotion warps of both CTAs hand rank 0's MMA warp
+      // the buffer
+      mbar_init(tempty_bar(b), kPair ? 2 * kPromoWarps : kPromoWarps);
     }
     mbar_init(drain_bar, 1);
     mbar_init(epi_bar, kPromoThreads);
+    if constexpr (kPair)
+      for (int s = 0; s < STAGES; ++s) mbar_init(pfull_bar(s), 1);
     *s_abort = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(s_tmem), L::kTmemCols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_u32(s_tmem), L::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(s_tmem), L::kTmemCols);
+      tmem_relinquish();
+    }
   }
   // nothing above touched global memory; from here on the previous kernel's
   // results (A, the scales, the index arrays) are visible
@@ -437,6 +458,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int units = num_units(p, S, s_prefix);
@@ -460,8 +482,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         t.group = block_expert(p, t.m_blk, true);
         if (t.group < 0) continue;
       }
-      const int a_row = t.m_blk * BM;
-      const int b_row = t.n_blk * BN;
+      const int a_row = t.m_blk * TM + static_cast<int>(rank) * BM;
+      const int b_row = t.n_blk * BN + (kPair ? static_cast<int>(rank) * (BN / 2) : 0);
       // D = C + A B^T: the epilogue's C rows are asked into L2 kCAhead K
       // blocks before the tile's last one -- late enough that the operand
       // stream of a long K does not evict them first, early enough to cover
@@ -546,7 +568,69 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     for (int i = max(0, it - STAGES); i < it; ++i)
       if (i != starve_it) mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &never, p.status);
   } else if (warp == 1) {
-   if constexpr (kUE) {
+   if constexpr (kPair) {
+    if (rank == 1) {
+      // ====================================== 2-CTA form, rank 1: forwarder
+      // This CTA's stages land on its own `full` barriers (so that its own
+      // producer can wait for them before the CTA exits); pass each stage's
+      // arrival on to rank 0's `pfull`, with release at cluster scope so
+      // that rank 0's MMAs read the landed data.
+      const uint32_t peer_pfull0 = mapa_shared(pfull_bar(0), 0);
+      int it = 0;
+      bool alive = true;
+      for (int u = u_first; u < units && alive; u += u_stride) {
+        const Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
+        for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(full_bar(s), (it / STAGES) & 1, s_abort, p.status)) {
+            alive = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive_release_cluster(peer_pfull0 + 8u * s);
+          __syncwarp();
+        }
+      }
+    } else {
+      // ========================================= 2-CTA form, rank 0: MMAs
+      // One cta_group::2 MMA of 256 x BN x 32 covers both CTAs' rows; its
+      // completion frees both CTAs' stages and publishes both CTAs' TMEM
+      // buffers (multicast commits).
+      constexpr uint32_t idesc = idesc_e4m3_f32(2 * BM, BN);
+      int it = 0, acc_it = 0;
+      bool alive = true;
+      for (int u = u_first; u < units && alive; u += u_stride) {
+        const Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
+        for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it, ++acc_it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          const int buf = acc_it % NBUF;
+          const uint32_t bph = (acc_it / NBUF) & 1;
+          if (!mbar_wait(tempty_bar(buf), bph ^ 1, s_abort, p.status)) { alive = false; break; }
+          if (!mbar_wait(full_bar(s), ph, s_abort, p.status)) { alive = false; break; }
+          if (!mbar_wait_cluster(pfull_bar(s), ph, s_abort, p.status)) { alive = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sa = base + s * L::kStageBytes;
+            const uint64_t adesc = smem_desc_k128_sw128(sa);
+            const uint64_t bdesc = smem_desc_k128_sw128(sa + kABytes);
+            const uint32_t d = tmem_base + buf * BN;
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k)
+              umma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+            umma_commit_pair_both(tfull_bar(buf));
+            umma_commit_pair_both(empty_bar(s));
+          }
+          __syncwarp();
+        }
+      }
+      // every MMA issued above must complete before either CTA frees TMEM or
+      // leaves (bounded, and not cut short by the abort flag)
+      if (lane == 0) umma_commit_pair_own(drain_bar);
+      __syncwarp();
+      volatile int never = 0;
+      mbar_wait(drain_bar, 0, &never, p.status);
+    }
+   } else if constexpr (kUE) {
     // ================================================ MMA issuer, UE8M0 scales
     // The tensor cores apply the scales: each K block's 4 MMAs (kind::mxf8f6f4
     // with block scaling) accumulate into the tile's single TMEM accumulator,
@@ -637,9 +721,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       }
     }
    }
-    {
+    if constexpr (!kPair) {
       // every MMA issued above must complete before TMEM is freed (bounded,
-      // and not cut short by the abort flag)
+      // and not cut short by the abort flag).  (The 2-CTA form drains in its
+      // own branch: a kernel's tcgen05 operations all use one CTA group.)
       if (lane == 0) umma_commit(drain_bar);
       __syncwarp();
       volatile int never = 0;
@@ -668,7 +753,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     };
     for (int u = u_first; u < units && alive; u += u_stride) {
       Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
-      const int row = t.m_blk * BM + row_in_tile;
+      const int row = t.m_blk * TM + static_cast<int>(rank) * BM + row_in_tile;
       bool row_ok;
       if constexpr (S == kContiguous) {
         t.group = block_expert(p, t.m_blk, false);
@@ -787,9 +872,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           } else {
             if (c0 + LW == W) {
               // all of this buffer has been read: hand it back to the MMA warp
+              // (2-CTA form: rank 0's, on its barrier)
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(tempty_bar(buf));
+              if (lane == 0) {
+                if constexpr (kPair) {
+                  mbar_arrive_cluster(mapa_shared(tempty_bar(buf), 0));
+                } else {
+                  mbar_arrive(tempty_bar(buf));
+                }
+              }
             }
 #pragma unroll
             for (int c = 0; c < LW; c += 2)
@@ -1055,7 +1147,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const uint32_t s_out = base + L::kOutOff;
         uint8_t *s_rowok = smem + L::kRowOkOff;
         const int ptid = threadIdx.x - kControlWarps * 32;
-        const int64_t slab_row0 = static_cast<int64_t>(t.slab) * p.rows + t.m_blk * BM;
+        const int64_t slab_row0 = static_cast<int64_t>(t.slab) * p.rows + t.m_blk * TM +
+                                  static_cast<int>(rank) * BM;
         if (half == 0) s_rowok[row_in_tile] = row_ok ? 1 : 0;
 #pragma unroll
         for (int ph = 0; ph < kPhases; ++ph) {
@@ -1144,8 +1237,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
+  // 2-CTA form: neither CTA leaves or frees TMEM while rank 0's MMAs may
+  // still read its shared memory or write its TMEM (rank 0 drained them)
+  if constexpr (kPair) cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, L::kTmemCols);
+  if (warp == 1) {
+    if constexpr (kPair) {
+      tmem_dealloc_pair(tmem_base, L::kTmemCols);
+    } else {
+      tmem_dealloc(tmem_base, L::kTmemCols);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -1157,14 +1259,19 @@ struct Candidate {
 constexpr Candidate kCandidates[] = {
     {256, 4, 2}, {128, 6, 4}, {64, 8, 8}, {32, 8, 8}, {16, 8, 8}};
 
+// Whether dense NT launches of two or more M blocks take the 2-CTA form
+// unless DG_PAIR says otherwise.
+constexpr bool kPairByDefault = false;
+
 // The UE8M0 schedules' one tile form: 256 wide, one accumulator (the tile
 // sums all of K in TMEM), three stages (the fourth does not fit beside the
 // per-stage scale-factor areas and the output staging).
 constexpr Candidate kUECandidate = {256, 3, 1};
 
-template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false, bool UE = false>
+template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false, bool UE = false,
+          bool PAIR = false>
 constexpr int smem_bytes_for(int extra) {
-  return 1024 + Layout<BN, STAGES, NBUF, STAGED, KG, UE>::kTableOff + extra;
+  return 1024 + Layout<BN, STAGES, NBUF, STAGED, KG, UE, PAIR>::kTableOff + extra;
 }
 
 bool print_configs() {
@@ -1176,7 +1283,8 @@ template <int BN, int STAGES, int NBUF, int SCHED, int LAYOUT = kLayoutNT>
 int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                     int grid, int extra_smem, cudaStream_t stream, bool coop) {
   const int smem = smem_bytes_for<BN, STAGES, NBUF, instance_staging(SCHED),
-                                  SCHED == kKGrouped, is_ue8m0(SCHED)>(extra_smem);
+                                  SCHED == kKGrouped, is_ue8m0(SCHED), SCHED == kDensePair>(
+      extra_smem);
   auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED, LAYOUT>;
   static int configured_smem[64] = {0};  // per device; grows only
   int dev = 0;
@@ -1199,8 +1307,8 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
       return DG_ERR_CUDA;
     configured_smem[dev] = smem;
   }
-  // clusters: the `splits` CTAs of a tile
-  const int cluster = SCHED == kDenseCluster ? p.splits : 1;
+  // clusters: the `splits` CTAs of a tile, or the CTA pair
+  const int cluster = SCHED == kDenseCluster ? p.splits : SCHED == kDensePair ? 2 : 1;
   if constexpr (SCHED == kDenseCluster) {
     // every cluster must be resident at once (one wave): ask the occupancy
     // calculator how many clusters of this size fit (cached per device)
@@ -1231,6 +1339,36 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
     }
     if (grid / cluster > fit[dev][cluster] - 1) return kClusterNoFit;
   }
+  int launch_grid = grid;
+  if constexpr (SCHED == kDensePair) {
+    // a persistent grid of pairs: never more pairs than fit at once (clusters
+    // of two need two free SMs of one GPC; a pair that is not resident would
+    // only start once another has finished all its tiles)
+    static int pairs_fit[64] = {};  // max active clusters + 1; 0 = not asked yet
+    if (pairs_fit[dev] == 0) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(grid);
+      q.blockDim = dim3(kThreads);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = 2;
+      a[0].val.clusterDim.y = 1;
+      a[0].val.clusterDim.z = 1;
+      q.attrs = a;
+      q.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      if (print_configs()) fprintf(stderr, "[dg] 2-CTA form: at most %d pairs resident\n", n);
+      pairs_fit[dev] = n + 1;
+    }
+    const int fit = pairs_fit[dev] - 1;
+    if (fit < 1) return DG_ERR_CUDA;
+    launch_grid = 2 * std::min(grid / 2, fit);
+  }
   if (coop) {
     // the splits of a tile wait for each other: all CTAs must be resident
     cudaLaunchConfig_t cfg = {};
@@ -1248,7 +1386,7 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
     // programmatic dependent launch: the kernel's set-up overlaps the tail of
     // the previous kernel (it waits for that grid before touching memory)
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
+    cfg.gridDim = dim3(launch_grid);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -1340,6 +1478,9 @@ int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmPar
         ta, tb, p, grid, extra, st, false);
   } else if constexpr (SCHED == kDenseQuant) {
     return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st, false);
+  } else if constexpr (SCHED == kDensePair) {
+    // 32 KB stages (A 16 KB + half of B 16 KB): six fit beside the staging
+    return launch_instance<256, 6, 2, SCHED>(ta, tb, p, grid, extra, st, false);
   } else {
     switch (bn) {
       case 256: return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st, coop);
@@ -1611,6 +1752,38 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
     const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
     const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
     return dispatch<kDenseQuant>(bn, ta, tb, p, grid, extra, stream);
+  }
+  // The 2-CTA form for dense NT shapes of at least two M blocks: each SM
+  // loads its 128 rows of A and half of the 256-wide B tile, two thirds of
+  // the single-CTA form's operand bytes per K block.  DG_PAIR=1 / 0 forces
+  // it on / off.
+  bool pair = false;
+  if (sched == kDense && p.c == nullptr && layout == kLayoutNT && rows > BM && n >= 256 &&
+      num_sms >= 2) {
+    pair = kPairByDefault;
+    if (const char *e = getenv("DG_PAIR")) pair = *e == '1';
+  }
+  if (pair) {
+    const int bn = 256;
+    p.num_m_blocks = static_cast<int>((rows + 2 * BM - 1) / (2 * BM));
+    p.num_n_blocks = static_cast<int>((n + bn - 1) / bn);
+    p.splits = 1;
+    p.full_tiles = 0;
+    p.ws = nullptr;
+    p.a_box_rows = BM;
+    CUtensorMap ta, tb;
+    int rc = make_tmap(&ta, A, k, rows, 1, BM);
+    if (rc) return rc;
+    rc = make_tmap(&tb, B, k, n, 1, bn / 2);
+    if (rc) return rc;
+    const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
+    const int grid =
+        2 * static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms / 2)));
+    if (print_configs())
+      fprintf(stderr, "[dg] gemm sched=dense rows=%lld n=%lld k=%lld: 2-CTA BN=256 grid=%d\n",
+              static_cast<long long>(rows), static_cast<long long>(n),
+              static_cast<long long>(k), grid);
+    return dispatch<kDensePair>(bn, ta, tb, p, grid, extra, stream);
   }
   const Choice choice =
       choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes, extra, max_smem, layout);

@@ -49,9 +49,12 @@ inline cudaLaunchAttribute pdl_attribute() {
 // kDenseQuant: dense tiles whose epilogue quantizes D: each row's 128-column
 // groups go out as E4M3 codes with one FP32 scale, as the 1x128 quantizer
 // would write them from the BF16 result.
+// kDensePair: dense 256-row tiles computed by the two CTAs of a cluster with
+// cta_group::2 MMAs (each CTA loads its 128 rows of A and half of the B tile,
+// so each SM moves two thirds of the single-CTA form's operand bytes).
 enum Sched : int {
   kDense = 0, kContiguous = 1, kMasked = 2, kDenseCluster = 3, kDenseAcc = 4, kKGrouped = 5,
-  kDenseUE8M0 = 6, kMaskedUE8M0 = 7, kDenseQuant = 8
+  kDenseUE8M0 = 6, kMaskedUE8M0 = 7, kDenseQuant = 8, kDensePair = 9
 };
 
 // Operand layouts of D = A * B^T ("DeepGEMM architecture deep dive",
@@ -69,7 +72,7 @@ __host__ __device__ constexpr bool b_mn_major(int layout) {
 
 // The tile schedule (work list, row validity, epilogue) a schedule follows.
 __host__ __device__ constexpr int base_sched(int sched) {
-  return (sched == kDenseUE8M0 || sched == kDenseQuant) ? kDense
+  return (sched == kDenseUE8M0 || sched == kDenseQuant || sched == kDensePair) ? kDense
          : sched == kMaskedUE8M0                        ? kMasked
                                                         : sched;
 }

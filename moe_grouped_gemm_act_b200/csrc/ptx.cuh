@@ -389,6 +389,111 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr) {
   return v;
 }
 
+// ------------------------------------------------------------------ CTA pairs
+// The 2-CTA form: the two CTAs of a cluster (ranks 0 and 1) compute a
+// 256-row tile with cta_group::2 MMAs issued by rank 0; each CTA holds its
+// own 128 rows of A and half of the B tile, and its own 128 accumulator rows
+// in TMEM.
+
+// Arrive on the mbarrier at a cluster-window address (the peer's) with
+// release semantics at cluster scope: the peer's acquire then sees what this
+// thread saw (the stage's data, which landed on this CTA's own barrier).
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   cluster_addr)
+               : "memory");
+}
+
+// Arrive on an mbarrier given by its cluster-window address (possibly in the
+// peer CTA), default semantics: the arrive follows this thread's completed
+// TMEM reads, which tcgen05.wait::ld and tcgen05.fence::before_thread_sync
+// order.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_acquire_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait with acquire semantics at cluster scope (for a barrier the peer
+// CTA arrives on with mbar_arrive_release_cluster); bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  volatile int *abort, int *status) {
+  if (mbar_try_wait_acquire_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait_acquire_cluster(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > g_wait_limit_ns) {
+      record_status(status, DG_ERR_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
+  asm volatile(
+      "tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+      "r"(ncols)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A * B^T with M = 256: rows 0-127 of A and D in
+// rank 0, rows 128-255 in rank 1; B split along N between the two CTAs'
+// shared memory at the same offsets.  Issued by one thread of rank 0.
+__device__ __forceinline__ void umma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, "
+      "%8, %9, %10, %11, %12}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z),
+      "r"(z), "r"(z), "r"(z), "r"(z)
+      : "memory");
+}
+
+// Arrives once on this CTA's mbarrier `bar` when all tcgen05 operations issued
+// so far by this thread (pair MMAs included) have completed.
+__device__ __forceinline__ void umma_commit_pair_own(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+// Arrives once on the mbarrier at offset `bar` in both CTAs of the pair when
+// all tcgen05 operations issued so far by this thread have completed.
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster."
+      "b64 [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+
 // ------------------------------------------------------------------ UMMA descriptors
 // Shared-memory matrix descriptor for a K-major operand tile whose rows are
 // 128 bytes (one 128-wide FP8 K block), written by TMA with the 128-byte

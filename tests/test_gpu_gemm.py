@@ -61,6 +61,50 @@ def test_dense_ragged_every_block_n(bn, m, n, k):
     check_gemm(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"{m}x{n}x{k} BN={bn}")
 
 
+@pytest.mark.parametrize("pair", [0, 1])
+@pytest.mark.parametrize("m,n,k", [(300, 392, 1024), (1000, 2112, 384), (513, 256, 256),
+                                   (256, 4096, 2048), (2048, 7168, 1536)])
+def test_dense_pair_and_single_cta_forms(pair, m, n, k):
+    # the 2-CTA form (cta_group::2, 256 x 256 tiles, each CTA loading half of
+    # B) and the single-CTA form
+    qa, alpha, qb, beta = dense_case(m, n, k, seed=m + 7 * n + k)
+    with env(DG_PAIR=pair):
+        got = run_dense(qa, alpha, qb, beta)
+    check_gemm(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"{m}x{n}x{k} pair={pair}")
+
+
+def test_dense_pair_exact_integers_bit_exact_and_deterministic():
+    g = np.random.default_rng(2)
+    m, n, k = 640, 768, 4096
+    a = g.integers(-4, 5, size=(m, k)).astype(np.float32)
+    b = g.integers(-4, 5, size=(n, k)).astype(np.float32)
+    qa, qb = e4m3.encode_rne(a), e4m3.encode_rne(b)
+    ones_a, ones_b = np.ones((m, k // 128), np.float32), np.ones((n // 128, k // 128), np.float32)
+    with env(DG_PAIR=1):
+        got = run_dense(qa, ones_a, qb, ones_b)
+        again = run_dense(qa, ones_a, qb, ones_b)
+    exact = a.astype(np.int64) @ b.astype(np.int64).T
+    assert np.array_equal(got, bf16.to_bits(exact.astype(np.float64)))
+    assert np.array_equal(got, again)
+
+
+def test_dense_pair_starved_wait_runs_out_and_the_next_call_is_clean():
+    # the abort path of the 2-CTA form: rank 0 of the first pair leaves out
+    # one stage; its MMA warp's wait runs out, rank 1's producer then runs
+    # out waiting for the stage to be freed, both CTAs wait for their own
+    # copies and leave; the next call is correct
+    qa, alpha, qb, beta = dense_case(512, 512, 2048, seed=12)
+    d = torch.zeros((512, 512), dtype=torch.bfloat16, device="cuda")
+    dg.dg_get_device_status()
+    with env(DG_PAIR=1, DG_TEST_STARVE_LOAD=2, DG_TEST_WAIT_LIMIT_US=20000):
+        dg.dg_fp8_gemm_nt(dev(qa), sfa_to_device(alpha), dev(qb), dev(beta), d)
+        torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == dg.DG_ERR_TIMEOUT
+    with env(DG_PAIR=1):
+        got = run_dense(qa, alpha, qb, beta)
+    check_gemm(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), "pair, after the timeout")
+
+
 @pytest.mark.parametrize("splits", [2, 3, 8])
 @pytest.mark.parametrize("bn", [32, 128, 256])
 def test_dense_split_k(splits, bn):
