@@ -96,17 +96,20 @@ static_assert(ctrl_regs(kDense) * 32 * kControlWarps + promo_regs(kDense) * kPro
 static_assert(ctrl_regs(kMasked) * 32 * kControlWarps + promo_regs(kMasked) * kPromoThreads <=
                   kLaunchRegs * kThreads,
               "register split exceeds the launch allocation");
+// Whether an instance runs with the warpgroup register split: the 256-wide
+// tiles (except contiguous: with the split, ptxas spills in its promotion
+// loop, measured 40 % slower) and the wider non-power-of-two tiles of the
+// cluster split.
+__host__ __device__ constexpr int gcd_c(int a, int b) { return b == 0 ? a : gcd_c(b, a % b); }
+__host__ __device__ constexpr bool uses_reg_split(int bn, int sched) {
+  return (bn == 256 && sched != kContiguous) || (bn > 128 && sched == kDenseCluster);
+}
 constexpr int kRasterGroupM = 16;       // M blocks per raster group (dense)
 constexpr int kCAhead = 8;              // K blocks between the C prefetch and the tile's end
 constexpr uint32_t kABytes = BM * BK;   // 16 KB per stage
 constexpr int kClusterNoFit = 1;        // launch_instance: clusters do not fit one wave
-
-// Test hook: the K-block iteration whose loads CTA 0's producer leaves out
-// (-1: none).  Nothing then completes that stage's `full` barrier, so the MMA
-// warp's bounded wait on it runs out: the way the tests exercise the abort
-// path without faulting anything.  Set from the host only while the
-// DG_TEST_STARVE_LOAD variable is present.
-static __device__ int g_starve_load_it = -1;
+constexpr int kMaxClusterSplits = 8;    // K splits reduced inside one (portable) cluster
+constexpr uint32_t kStoreBoxCols = 64;  // BF16 columns per TMA store box (128 bytes)
 
 // How a schedule's epilogue stages the output tile in shared memory: 0 not
 // at all, 1 the BF16 tile, 2 the FP32 tile (D = C + A B^T adds C as it
@@ -147,9 +150,8 @@ struct Layout {
   static constexpr uint32_t kOutOff = STAGES * kStageBytes;
   static constexpr uint32_t kRowOkOff = kOutOff + (STAGED ? BM * kOutCols * kOutElem : 0);
   static constexpr uint32_t kBarOff = kRowOkOff + (STAGED ? BM : 0);
-  // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain epi, then (2-CTA form)
-  // pfull[S]: the peer's stage has landed
-  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2 + (PAIR ? STAGES : 0);
+  // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain epi
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
   static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
   static constexpr uint32_t kPrefixOff = kMiscOff + 16;
   // k-grouped: a ring of per-column B scale slices, one per K block in
@@ -164,8 +166,11 @@ struct Layout {
   static constexpr uint32_t kSfBytes = UE ? STAGES * kSfStageBytes : 0u;
   static constexpr uint32_t kTableOff = kSfOff + kSfBytes;
   static_assert(!UE || BN == 256, "the UE8M0 scale-factor layout is laid out for 256-wide tiles");
-  // accumulator buffers, then (UE8M0) the scale-factor slots
-  static constexpr uint32_t kCols = BN * NBUF + (UE ? 2 * kSfSlotCols : 0);
+  // accumulator buffers (a non-power-of-two width starts each buffer on a
+  // power-of-two column), then (UE8M0) the scale-factor slots
+  static constexpr uint32_t kBufCols =
+      (BN & (BN - 1)) == 0 ? BN : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+  static constexpr uint32_t kCols = kBufCols * NBUF + (UE ? 2 * kSfSlotCols : 0);
   static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64
                                       : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
   static_assert(kCols <= 512, "TMEM holds 512 columns");
@@ -286,6 +291,7 @@ template <int BN, int STAGES, int NBUF, int SCHED, int LAYOUT = kLayoutNT>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
+                const __grid_constant__ CUtensorMap tmap_d,
                 const GemmParams p) {
   // dense and masked tiles leave through shared memory (coalesced row
   // stores); contiguous tiles store each thread's row segment directly
@@ -311,19 +317,37 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // 2-CTA form: the cluster's two CTAs compute one 256-row tile
   constexpr bool kPair = SCHED == kDensePair;
   constexpr int TM = kPair ? 2 * BM : BM;   // rows per tile
+  // dense tile schedules: B's first stages can be asked into L2 at entry
+  constexpr bool kPrefetchB = S == kDense || S == kDenseCluster || S == kDenseAcc;
+  // 128- and 256-wide BF16 tiles leave by TMA stores of the staged tile:
+  // dense tiles always (rows and columns past D are clipped by the tensor
+  // map), UE8M0 masked tiles whose 128 rows are all valid.  (The FP32-scale
+  // masked instance keeps its row stores: with both paths in it, ptxas
+  // spills and it ran 25 % slower.)
+  constexpr bool kTmaStore = (S == kDense || (S == kMasked && kUE)) && kStaged == 1 && BN >= 128;
   static_assert(!kPair || (BN == 256 && LAYOUT == kLayoutNT), "the 2-CTA form: NT, 256 wide");
   using L = Layout<BN, STAGES, NBUF, kStaged, kKG, kUE, kPair>;
   constexpr int W = BN / 2;                 // columns per promotion thread
-  // BN = 256 runs with the warpgroup register split (promo_regs per promotion
-  // thread), the narrower tiles fit the launch allocation as they are.  The
-  // contiguous schedule keeps the launch allocation: with the split, ptxas
-  // spills in its promotion loop (measured 40 % slower).
-  constexpr bool kRegSplit = BN == 256 && S != kContiguous;
+  // the wide tiles run with the warpgroup register split (promo_regs per
+  // promotion thread), the others fit the launch allocation as they are
+  constexpr bool kRegSplit = uses_reg_split(BN, S);
   // columns per TMEM load chunk: the whole slice up to 64 (one wait per
   // chunk; the buffer is handed back after the last chunk's wait, so the
   // fewer chunks, the sooner the MMA warp can reuse it); 16 for a 256-wide
-  // tile without the register split (128 accumulators under 168 registers)
-  constexpr int LW = W <= 64 ? W : kRegSplit ? 64 : 16;
+  // tile without the register split (128 accumulators under 168 registers).
+  // Non-power-of-two tiles: the largest of 64 / 32 / 16 dividing the slice
+  // under the split, else 16.  A thread's first column is a multiple of W, so
+  // the 128-column boundaries of B's scale blocks fall on multiples of
+  // gcd(W, 128) within its slice, and a chunk never straddles one.
+  constexpr bool kPow2 = (BN & (BN - 1)) == 0;
+  constexpr int LW = kPow2 ? (W <= 64 ? W : kRegSplit ? 64 : 16)
+                           : kRegSplit ? (W % 64 == 0 ? 64 : W % 32 == 0 ? 32 : 16) : 16;
+  // a thread's W columns may span two 128-column blocks of B's scales
+  // (non-power-of-two tiles only)
+  constexpr bool kStraddle = !kPow2;
+  static_assert(kPow2 || (S == kDenseCluster && BN % 32 == 0 && !kUE && LAYOUT == kLayoutNT),
+                "non-power-of-two tiles serve the NT cluster split, 32-column multiples");
+  static_assert(kPow2 || gcd_c(W, 128) % LW == 0, "a TMEM chunk within one scale block");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(W % LW == 0 && (LW == 8 || LW == 16 || LW == 32 || LW == 64), "TMEM chunk");
 
@@ -342,8 +366,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // synchronises the promotion threads in the epilogue (bounded, unlike a
   // named barrier, so that an aborting warp cannot strand the others)
   const uint32_t epi_bar = drain_bar + 8u;
-  // 2-CTA form, rank 0: the peer's copy of stage s has landed
-  auto pfull_bar = [&](int s) { return epi_bar + 8u * (1 + s); };
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *s_flag = reinterpret_cast<int *>(smem + L::kMiscOff + 8);
@@ -360,6 +382,28 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // ---------------------------------------------------------------- setup
   // the next kernel of the stream may begin its own set-up as our CTAs leave
   grid_launch_dependents();
+  if constexpr (kPrefetchB) {
+    // B's boxes of this CTA's first stages are asked into L2 before the
+    // set-up, so that HBM is busy while the barriers and TMEM are prepared
+    // (a decode-sized launch otherwise spends microseconds before its first
+    // bytes).  Same coordinates as the producer's loads.  A prefetch only
+    // fills L2, which the previous kernel's writes also go through, so it
+    // may precede the dependency wait; dense tiles only (their schedule
+    // needs no device data).
+    if (warp == 3 && lane < STAGES && u_first < num_units(p, S, nullptr)) {
+      const Tile t = unit_to_tile(p, S, u_first, nullptr, nullptr);
+      const int kb = t.k_begin + lane;
+      const int b_row = t.n_blk * BN + (kPair ? static_cast<int>(rank) * (BN / 2) : 0);
+      if (kb < t.k_end) {
+        if constexpr (kBmn) {
+#pragma unroll
+          for (int j = 0; j < BN / 128; ++j) tma_prefetch_3d(&tmap_b, b_row + 128 * j, kb * BK, 0);
+        } else {
+          tma_prefetch_3d(&tmap_b, kb * BK, b_row, 0);
+        }
+      }
+    }
+  }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
@@ -376,9 +420,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       mbar_init(tempty_bar(b), kPair ? 2 * kPromoWarps : kPromoWarps);
     }
     mbar_init(drain_bar, 1);
-    mbar_init(epi_bar, kPromoThreads);
-    if constexpr (kPair)
-      for (int s = 0; s < STAGES; ++s) mbar_init(pfull_bar(s), 1);
+    mbar_init(epi_bar, kPromoWarps);
     *s_abort = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -473,7 +515,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     // reads stale rows 64-127, which only reach output rows that are never
     // stored) and the B box
     const uint32_t stage_tx = static_cast<uint32_t>(p.a_box_rows) * BK + L::kBBytes;
-    const int starve_it = blockIdx.x == 0 ? g_starve_load_it : -1;
+    // test hook (GemmParams::starve_it): nothing completes the left-out
+    // stage's `full` barrier, so the MMA warp's bounded wait on it runs out,
+    // which exercises the abort path without faulting anything
+    const int starve_it = blockIdx.x == 0 ? p.starve_it : -1;
     int it = 0;
     bool alive = true;
     for (int u = u_first; u < units && alive; u += u_stride) {
@@ -508,7 +553,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!mbar_wait(empty_bar(s), ph ^ 1, s_abort, p.status)) { alive = false; break; }
-        if (lane == 0 && it != starve_it) {
+        if (kPair && lane == 0 && it != starve_it) {
+          // 2-CTA form: both CTAs' boxes complete on rank 0's `full`
+          // barrier, which rank 0 arms for the pair's bytes
+          const uint32_t sa = base + s * L::kStageBytes;
+          const uint32_t fb = mapa_shared(full_bar(s), 0);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2 * stage_tx);
+          tma_load_3d_pair(sa, &tmap_a, fb, kb * BK, a_row, t.slab);
+          tma_load_3d_pair(sa + kABytes, &tmap_b, fb, kb * BK, b_row, t.group);
+        } else if (lane == 0 && it != starve_it) {
           const uint32_t sa = base + s * L::kStageBytes;
           // (the k-grouped form's B is one [N][K] tensor for all groups)
           const int b_slab = kKG ? 0 : t.group;
@@ -564,33 +617,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     // wait (bounded, and not cut short by the abort flag) for the `full`
     // barrier of each of the last STAGES iterations armed above.  Earlier
     // iterations were consumed by the MMA warp, so their copies landed.
+    // (2-CTA form: rank 0's barriers count both CTAs' bytes, and rank 1
+    // leaves only after rank 0 at the teardown's cluster barrier.)
     volatile int never = 0;
-    for (int i = max(0, it - STAGES); i < it; ++i)
-      if (i != starve_it) mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &never, p.status);
+    if (!kPair || rank == 0)
+      for (int i = max(0, it - STAGES); i < it; ++i)
+        if (i != starve_it) mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &never, p.status);
   } else if (warp == 1) {
    if constexpr (kPair) {
-    if (rank == 1) {
-      // ====================================== 2-CTA form, rank 1: forwarder
-      // This CTA's stages land on its own `full` barriers (so that its own
-      // producer can wait for them before the CTA exits); pass each stage's
-      // arrival on to rank 0's `pfull`, with release at cluster scope so
-      // that rank 0's MMAs read the landed data.
-      const uint32_t peer_pfull0 = mapa_shared(pfull_bar(0), 0);
-      int it = 0;
-      bool alive = true;
-      for (int u = u_first; u < units && alive; u += u_stride) {
-        const Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
-        for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(full_bar(s), (it / STAGES) & 1, s_abort, p.status)) {
-            alive = false;
-            break;
-          }
-          if (lane == 0) mbar_arrive_release_cluster(peer_pfull0 + 8u * s);
-          __syncwarp();
-        }
-      }
-    } else {
+    // (2-CTA form: rank 1's MMA warp has no loop; rank 0 issues the
+    // pair's MMAs)
+    if (rank == 0) {
       // ========================================= 2-CTA form, rank 0: MMAs
       // One cta_group::2 MMA of 256 x BN x 32 covers both CTAs' rows; its
       // completion frees both CTAs' stages and publishes both CTAs' TMEM
@@ -607,13 +644,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           const uint32_t bph = (acc_it / NBUF) & 1;
           if (!mbar_wait(tempty_bar(buf), bph ^ 1, s_abort, p.status)) { alive = false; break; }
           if (!mbar_wait(full_bar(s), ph, s_abort, p.status)) { alive = false; break; }
-          if (!mbar_wait_cluster(pfull_bar(s), ph, s_abort, p.status)) { alive = false; break; }
           tc_fence_after();
           if (lane == 0) {
             const uint32_t sa = base + s * L::kStageBytes;
             const uint64_t adesc = smem_desc_k128_sw128(sa);
             const uint64_t bdesc = smem_desc_k128_sw128(sa + kABytes);
-            const uint32_t d = tmem_base + buf * BN;
+            const uint32_t d = tmem_base + buf * L::kBufCols;
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k)
               umma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
@@ -640,7 +676,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     // MMAs from this thread execute in order.
     constexpr uint32_t idesc0 = idesc_mxf8_ue8m0(BM, BN);
     const uint32_t acc_t = tmem_base;
-    const uint32_t sf_t = tmem_base + static_cast<uint32_t>(BN * NBUF);
+    const uint32_t sf_t = tmem_base + static_cast<uint32_t>(L::kBufCols * NBUF);
     int it = 0, tile_i = 0;
     bool alive = true;
     for (int u = u_first; u < units && alive; u += u_stride, ++tile_i) {
@@ -708,7 +744,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                                       : smem_desc_k128_sw128(sa);
           const uint64_t bdesc = kBmn ? smem_desc_mn_sw128(sa + kABytes, BK * 128)
                                       : smem_desc_k128_sw128(sa + kABytes);
-          const uint32_t d = tmem_base + buf * BN;
+          const uint32_t d = tmem_base + buf * L::kBufCols;
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)
             umma_f8(d, adesc + kAStep * k, bdesc + kBStep * k, idesc, k > 0 ? 1u : 0u);
@@ -743,13 +779,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     int it = 0;
     int tile_i = 0;  // UE8M0: tiles drained so far (the accumulator's phase)
     bool alive = true;
-    // every promotion thread arrives, then waits for the phase (bounded)
+    // every promotion warp arrives once (its lanes' shared-memory writes
+    // ordered before lane 0's release by the warp barrier), then all wait for
+    // the phase (bounded); the warp agrees on the outcome so that it stays
+    // converged for the next sync
     uint32_t epi_phase = 0;
     auto epi_sync = [&]() -> bool {
-      mbar_arrive(epi_bar);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_bar);
       const bool ok = mbar_wait(epi_bar, epi_phase & 1, s_abort, p.status);
       ++epi_phase;
-      return ok;
+      return __all_sync(0xffffffffu, ok);
     };
     for (int u = u_first; u < units && alive; u += u_stride) {
       Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
@@ -793,10 +833,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty_bar(0));
       } else {
-      // a thread's W columns (W divides 128 or equals 128) lie in one beta block
+      // a thread's W columns lie in one beta block when W divides 128 or
+      // equals it; a non-power-of-two tile's columns from col0 + cb on take
+      // the next block's beta (sfb_ptr1)
       const int nb = min(col0, p.n - 1) / 128;
       const float *sfb_ptr =
           p.sfb + (static_cast<int64_t>(t.group) * nb_total + nb) * kg_total;
+      const int cb = kStraddle ? (nb + 1) * 128 - col0 : W;
+      const float *sfb_ptr1 =
+          kStraddle ? p.sfb + (static_cast<int64_t>(t.group) * nb_total +
+                               min(nb + 1, nb_total - 1)) * kg_total
+                    : sfb_ptr;
 
       // This thread's row scale alpha is loaded two K blocks ahead into
       // registers (one coalesced 128-byte load per warp and block); rows past
@@ -818,14 +865,24 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       float b_batch_next =
           !kKG && t.k_begin + 32 + lane < t.k_end ? __ldg(sfb_ptr + t.k_begin + 32 + lane)
                                                    : 0.0f;
+      float b1_batch =
+          kStraddle && t.k_begin + lane < t.k_end ? __ldg(sfb_ptr1 + t.k_begin + lane) : 0.0f;
+      float b1_batch_next = kStraddle && t.k_begin + 32 + lane < t.k_end
+                                ? __ldg(sfb_ptr1 + t.k_begin + 32 + lane)
+                                : 0.0f;
       for (int kb = t.k_begin; kb < t.k_end; ++kb, ++it) {
-        float sc = a_cur;
+        float sc = a_cur, sc1 = a_cur;
         if constexpr (!kKG) {
           const int j = (kb - t.k_begin) & 31;
           sc = a_cur * __shfl_sync(0xffffffffu, b_batch, j);
+          if constexpr (kStraddle) sc1 = a_cur * __shfl_sync(0xffffffffu, b1_batch, j);
           if (j == 31) {
             b_batch = b_batch_next;
             b_batch_next = kb + 33 + lane < t.k_end ? __ldg(sfb_ptr + kb + 33 + lane) : 0.0f;
+            if constexpr (kStraddle) {
+              b1_batch = b1_batch_next;
+              b1_batch_next = kb + 33 + lane < t.k_end ? __ldg(sfb_ptr1 + kb + 33 + lane) : 0.0f;
+            }
           }
         }
         a_cur = a_next;
@@ -846,7 +903,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
         for (int c0 = 0; c0 < W; c0 += LW) {
           uint32_t r[LW];
-          tmem_ld<LW>(tmem_base + t_lane + buf * BN + half * W + c0, r);
+          tmem_ld<LW>(tmem_base + t_lane + buf * L::kBufCols + half * W + c0, r);
           tmem_wait_ld();
           reg_barrier<LW>(r);
           if constexpr (kKG) {
@@ -865,6 +922,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
               ffma2(acc[c0 + c + 2], acc[c0 + c + 3], y2, y3, sc);
             }
             if (c0 + LW == W) {
+              // the scale slot is refilled by a bulk copy (async proxy) once
+              // the buffer is back: order this thread's generic reads of it
+              // before that write (without the fence, repeated runs differed
+              // in the last scale reads' columns)
+              fence_proxy_async_smem();
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(tempty_bar(buf));
@@ -883,10 +945,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
               }
             }
+            const float s_chunk = !kStraddle || c0 < cb ? sc : sc1;
 #pragma unroll
             for (int c = 0; c < LW; c += 2)
               ffma2(acc[c0 + c], acc[c0 + c + 1], __uint_as_float(r[c]), __uint_as_float(r[c + 1]),
-                    sc);
+                    s_chunk);
           }
         }
       }
@@ -1133,23 +1196,33 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           }
         }
       } else {
-        // The tile leaves through shared memory so that each warp store
-        // writes whole row segments (16-byte chunks of consecutive columns of
-        // a row in consecutive lanes).  Staging layout: [128 rows][kOutCols]
-        // BF16 with 16-byte chunk c of row r at chunk c ^ (r mod kSw), which
-        // keeps both the row-per-lane writes and the row-major reads free of
-        // bank conflicts.  A 256-wide tile goes out in two column halves,
-        // each written by the warps that own it.
+        // The tile leaves through shared memory.  Staging layout: [128 rows]
+        // x kOutCols BF16; a 128-column half is two boxes of [128 rows][64
+        // columns], 128 bytes a row, 16-byte chunk c of row r at c ^ (r mod 8)
+        // -- the 128-byte swizzle of the TMA store's tensor map, and free of
+        // bank conflicts both for the row-per-lane writes and for row-major
+        // reads.  A 256-wide tile goes out in two column halves, each written
+        // by the warps that own it.  Dense tiles leave by TMA stores issued
+        // by one thread, and so do UE8M0 masked tiles whose rows are all
+        // valid; other masked tiles (rows past an expert's count stay
+        // untouched) leave by warp stores of whole row segments, valid rows
+        // only.
         constexpr int kChunks = L::kOutCols / 8;        // 16-byte chunks per staged row
         constexpr int kSw = kChunks < 8 ? kChunks : 8;  // swizzle span, in chunks
         constexpr int kPhases = BN > 128 ? 2 : 1;
-        constexpr int kRowBytes = L::kOutCols * 2;
+        constexpr int kRowBytes = kChunks < 8 ? L::kOutCols * 2 : 128;
+        auto staged_off = [&](int r, int c) -> uint32_t {
+          return static_cast<uint32_t>((c / kSw) * (BM * kRowBytes) + r * kRowBytes +
+                                       ((c % kSw) ^ (r % kSw)) * 16);
+        };
         const uint32_t s_out = base + L::kOutOff;
         uint8_t *s_rowok = smem + L::kRowOkOff;
         const int ptid = threadIdx.x - kControlWarps * 32;
         const int64_t slab_row0 = static_cast<int64_t>(t.slab) * p.rows + t.m_blk * TM +
                                   static_cast<int>(rank) * BM;
-        if (half == 0) s_rowok[row_in_tile] = row_ok ? 1 : 0;
+        const bool tma_tile =
+            kTmaStore && (S == kDense || (t.m_blk + 1) * BM <= masked_rows(p, t.slab));
+        if (!tma_tile && half == 0) s_rowok[row_in_tile] = row_ok ? 1 : 0;
 #pragma unroll
         for (int ph = 0; ph < kPhases; ++ph) {
           if (kPhases == 1 || half == ph) {
@@ -1162,23 +1235,36 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __nv_bfloat162 h = __floats2bfloat162_rn(acc[c + 2 * j], acc[c + 2 * j + 1]);
                 w[j] = *reinterpret_cast<const uint32_t *>(&h);
               }
-              const int chunk = (scol0 + c) / 8;
-              st_shared_v4(s_out + row_in_tile * kRowBytes + ((chunk ^ (row_in_tile % kSw)) * 16),
-                           w[0], w[1], w[2], w[3]);
+              st_shared_v4(s_out + staged_off(row_in_tile, (scol0 + c) / 8), w[0], w[1], w[2],
+                           w[3]);
             }
+            // the TMA store reads the tile through the async proxy
+            if constexpr (kTmaStore) fence_proxy_async_smem();
           }
           if (!epi_sync()) {
             alive = false;
             break;
           }
           const int col_base = t.n_blk * BN + ph * 128;
+          if (tma_tile) {
+            if (ptid == 0) {
+#pragma unroll
+              for (int j = 0; j < kChunks / 8; ++j)
+                if (col_base + j * static_cast<int>(kStoreBoxCols) < p.n)
+                  tma_store_3d(&tmap_d, s_out + j * (BM * 128u), col_base + j * kStoreBoxCols,
+                               t.m_blk * TM + static_cast<int>(rank) * BM, t.slab);
+              bulk_commit_group();
+              bulk_wait_group_read_all();  // the staging tile may be written again
+            }
+          } else {
 #pragma unroll 1
-          for (int f = ptid; f < BM * kChunks; f += kPromoThreads) {
-            const int r = f / kChunks, ch = f - r * kChunks;
-            const int col = col_base + ch * 8;
-            if (s_rowok[r] && col < p.n) {
-              const uint4 v = ld_shared_v4(s_out + r * kRowBytes + ((ch ^ (r % kSw)) * 16));
-              *reinterpret_cast<uint4 *>(p.d + (slab_row0 + r) * p.n + col) = v;
+            for (int f = ptid; f < BM * kChunks; f += kPromoThreads) {
+              const int r = f / kChunks, ch = f - r * kChunks;
+              const int col = col_base + ch * 8;
+              if (s_rowok[r] && col < p.n) {
+                const uint4 v = ld_shared_v4(s_out + staged_off(r, ch));
+                *reinterpret_cast<uint4 *>(p.d + (slab_row0 + r) * p.n + col) = v;
+              }
             }
           }
           if (!epi_sync()) {
@@ -1188,6 +1274,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
       }
       if (!alive) break;
+    }
+    // the TMA stores of D have completed before the CTA exits
+    if constexpr (kTmaStore) {
+      if (threadIdx.x == kControlWarps * 32) bulk_wait_group_all();
     }
   }
 
@@ -1212,13 +1302,21 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       for (int f = split * share + ptid; f < f_end; f += kPromoThreads) {
         const int r = f / kChunksF, c = f - r * kChunksF;
         const uint32_t off = base + 16u * (r * kChunksF + (c ^ (r % kSwF)));
-        float4 sum = ld_shared_cluster_v4(mapa_shared(off, 0));
-        for (int q = 1; q < p.splits; ++q) {  // split order: deterministic
-          const float4 v = ld_shared_cluster_v4(mapa_shared(off, static_cast<uint32_t>(q)));
-          sum.x += v.x;
-          sum.y += v.y;
-          sum.z += v.z;
-          sum.w += v.w;
+        // every split's chunk in flight at once, then summed in split order
+        // (deterministic); a cluster has at most kMaxClusterSplits CTAs
+        float4 v[kMaxClusterSplits];
+#pragma unroll
+        for (int q = 0; q < kMaxClusterSplits; ++q)
+          if (q < p.splits) v[q] = ld_shared_cluster_v4(mapa_shared(off, static_cast<uint32_t>(q)));
+        float4 sum = v[0];
+#pragma unroll
+        for (int q = 1; q < kMaxClusterSplits; ++q) {
+          if (q < p.splits) {
+            sum.x += v[q].x;
+            sum.y += v[q].y;
+            sum.z += v[q].z;
+            sum.w += v[q].w;
+          }
         }
         const int col = t.n_blk * BN + 4 * c;
         if (col < p.n) {
@@ -1259,6 +1357,14 @@ struct Candidate {
 constexpr Candidate kCandidates[] = {
     {256, 4, 2}, {128, 6, 4}, {64, 8, 8}, {32, 8, 8}, {16, 8, 8}};
 
+// Tile forms of the cluster split (decode-sized dense NT shapes): the
+// power-of-two forms above and non-power-of-two widths, which let more of
+// the SMs stream B when the power-of-two tiling leaves clusters that do not
+// fit one wave.  Stages: as many as fit the shared memory (more blocks in
+// flight per SM).
+constexpr Candidate kClusterForms[] = {{256, 4, 2}, {224, 5, 2}, {192, 5, 2}, {160, 6, 2},
+                                       {128, 6, 4}, {96, 7, 4},  {64, 8, 8}};
+
 // Whether dense NT launches of two or more M blocks take the 2-CTA form
 // unless DG_PAIR says otherwise.
 constexpr bool kPairByDefault = false;
@@ -1279,17 +1385,79 @@ bool print_configs() {
   return e && *e && *e != '0';
 }
 
+// Sets the instance's dynamic shared memory limit (once per device, grows
+// only); false on a CUDA error.
+template <int BN, int STAGES, int NBUF, int SCHED, int LAYOUT>
+bool configure_smem(int smem) {
+  static int configured_smem[64] = {0};  // per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (smem > configured_smem[dev]) {
+    if (cudaFuncSetAttribute(fp8_gemm_kernel<BN, STAGES, NBUF, SCHED, LAYOUT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return false;
+    configured_smem[dev] = smem;
+  }
+  return true;
+}
+
+template <int BN, int STAGES, int NBUF, int SCHED>
+constexpr int instance_smem(int extra) {
+  return smem_bytes_for<BN, STAGES, NBUF, instance_staging(SCHED), SCHED == kKGrouped,
+                        is_ue8m0(SCHED), SCHED == kDensePair>(extra);
+}
+
+// How many thread-block clusters of `cluster` CTAs of this instance can be
+// resident at once (the occupancy calculator, cached per device; 0 when the
+// size is unsupported or the query fails).
+template <int BN, int STAGES, int NBUF, int SCHED, int LAYOUT>
+int clusters_fit(int cluster) {
+  static int fit[64][kMaxClusterSplits + 1] = {};  // max active clusters + 1; 0 = not asked
+  int dev = 0;
+  if (cluster < 2 || cluster > kMaxClusterSplits || cudaGetDevice(&dev) != cudaSuccess ||
+      dev < 0 || dev >= 64)
+    return 0;
+  if (fit[dev][cluster] == 0) {
+    const int smem = instance_smem<BN, STAGES, NBUF, SCHED>(0);
+    int n = 0;
+    if (configure_smem<BN, STAGES, NBUF, SCHED, LAYOUT>(smem)) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(cluster);
+      q.blockDim = dim3(kThreads);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = cluster;
+      a[0].val.clusterDim.y = 1;
+      a[0].val.clusterDim.z = 1;
+      q.attrs = a;
+      q.numAttrs = 1;
+      const cudaError_t e =
+          cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<BN, STAGES, NBUF, SCHED, LAYOUT>, &q);
+      if (e != cudaSuccess) {
+        cudaGetLastError();  // clear: the caller takes another form
+        n = 0;
+      }
+      if (print_configs())
+        fprintf(stderr, "[dg] BN=%d clusters of %d: at most %d resident (%s)\n", BN, cluster, n,
+                cudaGetErrorString(e));
+    } else {
+      cudaGetLastError();
+    }
+    fit[dev][cluster] = n + 1;
+  }
+  return fit[dev][cluster] - 1;
+}
+
 template <int BN, int STAGES, int NBUF, int SCHED, int LAYOUT = kLayoutNT>
-int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb,
+                    const CUtensorMap &td, const GemmParams &p,
                     int grid, int extra_smem, cudaStream_t stream, bool coop) {
-  const int smem = smem_bytes_for<BN, STAGES, NBUF, instance_staging(SCHED),
-                                  SCHED == kKGrouped, is_ue8m0(SCHED), SCHED == kDensePair>(
-      extra_smem);
+  const int smem = instance_smem<BN, STAGES, NBUF, SCHED>(extra_smem);
   auto kern = fp8_gemm_kernel<BN, STAGES, NBUF, SCHED, LAYOUT>;
-  static int configured_smem[64] = {0};  // per device; grows only
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DG_ERR_CUDA;
-  if constexpr (BN == 256) {
+  if constexpr (uses_reg_split(BN, base_sched(SCHED))) {
     // the warpgroup register split needs the full launch allocation: never
     // launch an instance compiled to fewer registers (its promotion warps
     // would wait for registers that never come)
@@ -1301,43 +1469,12 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
     }
     if (regs_checked < 0) return DG_ERR_CUDA;
   }
-  if (smem > configured_smem[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return DG_ERR_CUDA;
-    configured_smem[dev] = smem;
-  }
+  if (!configure_smem<BN, STAGES, NBUF, SCHED, LAYOUT>(smem)) return DG_ERR_CUDA;
   // clusters: the `splits` CTAs of a tile, or the CTA pair
   const int cluster = SCHED == kDenseCluster ? p.splits : SCHED == kDensePair ? 2 : 1;
   if constexpr (SCHED == kDenseCluster) {
-    // every cluster must be resident at once (one wave): ask the occupancy
-    // calculator how many clusters of this size fit (cached per device)
-    static int fit[64][9] = {};  // max active clusters + 1; 0 = not asked yet
-    if (cluster < 2 || cluster > 8) return kClusterNoFit;
-    if (fit[dev][cluster] == 0) {
-      cudaLaunchConfig_t q = {};
-      q.gridDim = dim3(grid);
-      q.blockDim = dim3(kThreads);
-      q.dynamicSmemBytes = smem;
-      cudaLaunchAttribute a[1];
-      a[0].id = cudaLaunchAttributeClusterDimension;
-      a[0].val.clusterDim.x = cluster;
-      a[0].val.clusterDim.y = 1;
-      a[0].val.clusterDim.z = 1;
-      q.attrs = a;
-      q.numAttrs = 1;
-      int n = 0;
-      const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &q);
-      if (e != cudaSuccess) {
-        cudaGetLastError();  // clear: the caller falls back to the other path
-        n = 0;
-      }
-      if (print_configs())
-        fprintf(stderr, "[dg] BN=%d clusters of %d: at most %d resident (%s)\n", BN, cluster, n,
-                cudaGetErrorString(e));
-      fit[dev][cluster] = n + 1;
-    }
-    if (grid / cluster > fit[dev][cluster] - 1) return kClusterNoFit;
+    // every cluster must be resident at once (one wave)
+    if (grid / cluster > clusters_fit<BN, STAGES, NBUF, SCHED, LAYOUT>(cluster)) return kClusterNoFit;
   }
   int launch_grid = grid;
   if constexpr (SCHED == kDensePair) {
@@ -1381,7 +1518,7 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return DG_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, td, p) != cudaSuccess) return DG_ERR_CUDA;
   } else {
     // programmatic dependent launch: the kernel's set-up overlaps the tail of
     // the previous kernel (it waits for that grid before touching memory)
@@ -1401,9 +1538,24 @@ int launch_instance(const CUtensorMap &ta, const CUtensorMap &tb, const GemmPara
       attr[1].val.clusterDim.z = 1;
       cfg.numAttrs = 2;
     }
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return DG_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, td, p) != cudaSuccess) return DG_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
+// Clusters of `cluster` CTAs of the cluster-split instance of width `bn`
+// that fit at once (0 for a width without an instance).
+int cluster_split_fit(int bn, int cluster) {
+  switch (bn) {
+    case 256: return clusters_fit<256, 4, 2, kDenseCluster, kLayoutNT>(cluster);
+    case 224: return clusters_fit<224, 5, 2, kDenseCluster, kLayoutNT>(cluster);
+    case 192: return clusters_fit<192, 5, 2, kDenseCluster, kLayoutNT>(cluster);
+    case 160: return clusters_fit<160, 6, 2, kDenseCluster, kLayoutNT>(cluster);
+    case 128: return clusters_fit<128, 6, 4, kDenseCluster, kLayoutNT>(cluster);
+    case 96: return clusters_fit<96, 7, 4, kDenseCluster, kLayoutNT>(cluster);
+    case 64: return clusters_fit<64, 8, 8, kDenseCluster, kLayoutNT>(cluster);
+    default: return 0;
+  }
 }
 
 // Dynamic shared memory of a single-CTA tile form for a schedule (extra =
@@ -1430,6 +1582,14 @@ int config_smem(int bn, int extra, int sched) {
     case 64: return single_smem<64, 8, 8>(sched, extra);
     case 32: return single_smem<32, 8, 8>(sched, extra);
     case 16: return single_smem<16, 8, 8>(sched, extra);
+    default: break;
+  }
+  if (sched != kDenseCluster) return 1 << 30;
+  switch (bn) {  // the cluster split's non-power-of-two widths
+    case 224: return single_smem<224, 5, 2>(sched, extra);
+    case 192: return single_smem<192, 5, 2>(sched, extra);
+    case 160: return single_smem<160, 6, 2>(sched, extra);
+    case 96: return single_smem<96, 7, 4>(sched, extra);
     default: return 1 << 30;
   }
 }
@@ -1446,48 +1606,61 @@ int max_smem_per_block() {
 // The transposed layouts: tiles 256 or 128 wide (a whole number of
 // 128-value MN-major columns of B).
 template <int SCHED, int LAYOUT>
-int dispatch_layout(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+int dispatch_layout(int bn, const CUtensorMap &ta, const CUtensorMap &tb,
+                    const CUtensorMap &td, const GemmParams &p,
                     int grid, int extra, cudaStream_t st) {
   const bool coop = p.splits > 1 && SCHED != kDenseCluster;
   switch (bn) {
-    case 256: return launch_instance<256, 4, 2, SCHED, LAYOUT>(ta, tb, p, grid, extra, st, coop);
-    case 128: return launch_instance<128, 6, 4, SCHED, LAYOUT>(ta, tb, p, grid, extra, st, coop);
+    case 256: return launch_instance<256, 4, 2, SCHED, LAYOUT>(ta, tb, td, p, grid, extra, st, coop);
+    case 128: return launch_instance<128, 6, 4, SCHED, LAYOUT>(ta, tb, td, p, grid, extra, st, coop);
     default: return DG_ERR_INVALID_ARG;
   }
 }
 
 template <int SCHED>
 int dispatch_any_layout(int layout, int bn, const CUtensorMap &ta, const CUtensorMap &tb,
+                    const CUtensorMap &td,
                         const GemmParams &p, int grid, int extra, cudaStream_t st) {
   switch (layout) {
-    case kLayoutNN: return dispatch_layout<SCHED, kLayoutNN>(bn, ta, tb, p, grid, extra, st);
-    case kLayoutTN: return dispatch_layout<SCHED, kLayoutTN>(bn, ta, tb, p, grid, extra, st);
-    case kLayoutTT: return dispatch_layout<SCHED, kLayoutTT>(bn, ta, tb, p, grid, extra, st);
+    case kLayoutNN: return dispatch_layout<SCHED, kLayoutNN>(bn, ta, tb, td, p, grid, extra, st);
+    case kLayoutTN: return dispatch_layout<SCHED, kLayoutTN>(bn, ta, tb, td, p, grid, extra, st);
+    case kLayoutTT: return dispatch_layout<SCHED, kLayoutTT>(bn, ta, tb, td, p, grid, extra, st);
     default: return DG_ERR_INVALID_ARG;
   }
 }
 
 template <int SCHED>
-int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+int dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb,
+                    const CUtensorMap &td, const GemmParams &p,
              int grid, int extra, cudaStream_t st) {
+  if constexpr (SCHED == kDenseCluster) {
+    // the non-power-of-two widths (cluster split, NT only)
+    switch (bn) {
+      case 224: return launch_instance<224, 5, 2, SCHED>(ta, tb, td, p, grid, extra, st, false);
+      case 192: return launch_instance<192, 5, 2, SCHED>(ta, tb, td, p, grid, extra, st, false);
+      case 160: return launch_instance<160, 6, 2, SCHED>(ta, tb, td, p, grid, extra, st, false);
+      case 96: return launch_instance<96, 7, 4, SCHED>(ta, tb, td, p, grid, extra, st, false);
+      default: break;
+    }
+  }
   // splits that wait for each other through global memory need all CTAs
   // resident; a cluster's splits are co-scheduled by construction
   const bool coop = p.splits > 1 && SCHED != kDenseCluster;
   if constexpr (is_ue8m0(SCHED)) {
     return launch_instance<kUECandidate.bn, kUECandidate.stages, kUECandidate.nbuf, SCHED>(
-        ta, tb, p, grid, extra, st, false);
+        ta, tb, td, p, grid, extra, st, false);
   } else if constexpr (SCHED == kDenseQuant) {
-    return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st, false);
+    return launch_instance<256, 4, 2, SCHED>(ta, tb, td, p, grid, extra, st, false);
   } else if constexpr (SCHED == kDensePair) {
     // 32 KB stages (A 16 KB + half of B 16 KB): six fit beside the staging
-    return launch_instance<256, 6, 2, SCHED>(ta, tb, p, grid, extra, st, false);
+    return launch_instance<256, 6, 2, SCHED>(ta, tb, td, p, grid, extra, st, false);
   } else {
     switch (bn) {
-      case 256: return launch_instance<256, 4, 2, SCHED>(ta, tb, p, grid, extra, st, coop);
-      case 128: return launch_instance<128, 6, 4, SCHED>(ta, tb, p, grid, extra, st, coop);
-      case 64: return launch_instance<64, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
-      case 32: return launch_instance<32, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
-      case 16: return launch_instance<16, 8, 8, SCHED>(ta, tb, p, grid, extra, st, coop);
+      case 256: return launch_instance<256, 4, 2, SCHED>(ta, tb, td, p, grid, extra, st, coop);
+      case 128: return launch_instance<128, 6, 4, SCHED>(ta, tb, td, p, grid, extra, st, coop);
+      case 64: return launch_instance<64, 8, 8, SCHED>(ta, tb, td, p, grid, extra, st, coop);
+      case 32: return launch_instance<32, 8, 8, SCHED>(ta, tb, td, p, grid, extra, st, coop);
+      case 16: return launch_instance<16, 8, 8, SCHED>(ta, tb, td, p, grid, extra, st, coop);
       default: return DG_ERR_INVALID_ARG;
     }
   }
@@ -1532,6 +1705,25 @@ int make_tmap_mn(CUtensorMap *m, const void *ptr, int64_t rows, int64_t k, int64
   return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
+// 3-D tensor map over the BF16 output D [slabs][rows][n] for the epilogue's
+// TMA stores: a box of [1][128 rows][64 columns] (128 bytes, the staging
+// tile's 128-byte swizzle).  n % 8 == 0 and D 16-byte aligned (checked by
+// the entry points), so the row stride is a multiple of 16 bytes.
+int make_tmap_d(CUtensorMap *m, void *d, int64_t rows, int64_t n, int64_t slabs) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return DG_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(slabs)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(n * 2),
+                                 static_cast<cuuint64_t>(n * rows * 2)};
+  const cuuint32_t box[3] = {kStoreBoxCols, BM, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, d, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
 // Cycles one CTA spends per 128-K block of a unit, measured on B200.  The
 // tensor cores take ~540 cycles per block for any N up to 256 (one
 // 128 x N x 32 MMA per ~135 cycles), so narrow tiles waste them; the
@@ -1539,7 +1731,11 @@ int make_tmap_mn(CUtensorMap *m, const void *ptr, int64_t rows, int64_t k, int64
 double kb_cycles(int bn) {
   switch (bn) {
     case 256: return 1240.0;
+    case 224: return 1160.0;  // (non-power-of-two widths: interpolated)
+    case 192: return 1070.0;
+    case 160: return 990.0;
     case 128: return 900.0;
+    case 96: return 830.0;
     case 64: return 770.0;
     default: return 750.0;
   }
@@ -1558,6 +1754,49 @@ double estimate(int64_t m_blocks, int64_t n, int64_t k, int bn, int splits, int 
   const double t = waves * per_unit;
   const double bytes = static_cast<double>(n) * k + m_blocks * 128.0 * k;
   return std::max(t, bytes / (23.0 * sms));
+}
+
+// The cluster split of a decode-sized shape streams B through every CTA's
+// stage ring: a CTA completes about one K block per kLoadLatency / STAGES
+// cycles (each block's copy takes a loaded-memory round trip; STAGES are in
+// flight; measured ~2.9 us per round trip with the 4-stage 256-wide form on
+// B200), never faster than its tensor work, and the launch never moves its
+// bytes faster than HBM (~3,400 bytes per SM cycle).
+constexpr double kLoadLatency = 5600.0;
+constexpr double kHbmBytesPerCycle = 3400.0;
+
+double estimate_cluster(int64_t m_blocks, int64_t n, int64_t k, const Candidate &f, int s) {
+  const int64_t kb = (k / BK + s - 1) / s;
+  const double per_kb = std::max(kb_cycles(f.bn), kLoadLatency / f.stages);
+  const double t = kb * per_kb + 2500.0 + 1500.0 + 300.0 * s;
+  const double bytes = static_cast<double>(n) * k + m_blocks * 128.0 * k;
+  return std::max(t, bytes / kHbmBytesPerCycle);
+}
+
+// The cluster split's form for a decode-sized dense NT shape: the width and
+// split of the fastest estimate among the forms whose clusters all fit one
+// wave (occupancy calculator) within `sms` CTAs.  {0, 0} when none does.
+struct ClusterPick {
+  int bn, splits;
+};
+ClusterPick pick_cluster_form(int64_t rows, int64_t n, int64_t k, int sms, int max_smem) {
+  const int64_t m_blocks = (rows + BM - 1) / BM;
+  ClusterPick best{0, 0};
+  double best_t = 1e300;
+  for (const Candidate &f : kClusterForms) {
+    if (config_smem(f.bn, 0, kDenseCluster) > max_smem) continue;
+    const int64_t tiles = m_blocks * ((n + f.bn - 1) / f.bn);
+    for (int s = 2; s <= kMaxClusterSplits; ++s) {
+      if (tiles * s > sms || s > k / BK) break;
+      if (cluster_split_fit(f.bn, s) < tiles) continue;
+      const double e = estimate_cluster(m_blocks, n, k, f, s);
+      if (e < best_t * 0.99) {
+        best_t = e;
+        best = {f.bn, s};
+      }
+    }
+  }
+  return best;
 }
 
 size_t split_ws_bytes(int64_t tiles, int splits, int bn) {
@@ -1645,35 +1884,27 @@ size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int num_sms) {
 
 // Test knobs of the abort path (both unset in normal use):
 // DG_TEST_STARVE_LOAD=i makes CTA 0's producer leave out the loads of its
-// iteration i, DG_TEST_WAIT_LIMIT_US=t lowers every wait's limit to t
-// microseconds.  They are written to the device before this call's kernel and
-// put back after it, in stream order.
+// iteration i (a kernel parameter); DG_TEST_WAIT_LIMIT_US=t lowers every
+// wait's limit to t microseconds (at least kWaitCheckNs), written to the
+// device before this call's kernel and put back after it, in stream order.
 struct TestKnobs {
-  bool on = false;
   int starve = -1;
   unsigned long long limit_ns = kWaitLimitNs;
 };
 
 static TestKnobs test_knobs() {
   TestKnobs k;
-  if (const char *e = getenv("DG_TEST_STARVE_LOAD")) {
-    k.on = true;
-    k.starve = atoi(e);
-  }
-  if (const char *e = getenv("DG_TEST_WAIT_LIMIT_US")) {
-    k.on = true;
+  if (const char *e = getenv("DG_TEST_STARVE_LOAD")) k.starve = atoi(e);
+  if (const char *e = getenv("DG_TEST_WAIT_LIMIT_US"))
     k.limit_ns = strtoull(e, nullptr, 10) * 1000ull;
-  }
   return k;
 }
 
-static int set_test_knobs(const TestKnobs &k, cudaStream_t stream) {
-  if (cudaMemcpyToSymbolAsync(g_starve_load_it, &k.starve, sizeof(int), 0,
-                              cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyToSymbolAsync(g_wait_limit_ns, &k.limit_ns, sizeof(k.limit_ns), 0,
-                              cudaMemcpyHostToDevice, stream) != cudaSuccess)
-    return DG_ERR_CUDA;
-  return DG_OK;
+static int set_wait_limit(unsigned long long limit_ns, cudaStream_t stream) {
+  return cudaMemcpyToSymbolAsync(g_wait_limit_ns, &limit_ns, sizeof(limit_ns), 0,
+                                 cudaMemcpyHostToDevice, stream) == cudaSuccess
+             ? DG_OK
+             : DG_ERR_CUDA;
 }
 
 static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
@@ -1683,12 +1914,13 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
 int launch_fp8_gemm(int sched, const uint8_t *A, const uint8_t *B, GemmParams p,
                     cudaStream_t stream, int num_sms, size_t ws_bytes, void *ws, int layout) {
   const TestKnobs knobs = test_knobs();
-  if (!knobs.on)
+  p.starve_it = knobs.starve;
+  if (knobs.limit_ns == kWaitLimitNs)
     return launch_fp8_gemm_impl(sched, A, B, p, stream, num_sms, ws_bytes, ws, layout);
-  int rc = set_test_knobs(knobs, stream);
+  int rc = set_wait_limit(knobs.limit_ns, stream);
   if (rc) return rc;
   rc = launch_fp8_gemm_impl(sched, A, B, p, stream, num_sms, ws_bytes, ws, layout);
-  const int rc2 = set_test_knobs(TestKnobs{}, stream);
+  const int rc2 = set_wait_limit(kWaitLimitNs, stream);
   return rc ? rc : rc2;
 }
 
@@ -1718,12 +1950,13 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
     p.full_tiles = 0;
     p.ws = nullptr;
     p.a_box_rows = BM;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, td = {};
     const bool masked = base_sched(sched) == kMasked;
     int rc = make_tmap(&ta, A, k, rows, masked ? p.groups : 1, BM);
     if (rc) return rc;
     rc = make_tmap(&tb, B, k, n, masked ? p.groups : 1, bn);
     if (rc) return rc;
+    if ((rc = make_tmap_d(&td, p.d, rows, n, masked ? p.groups : 1))) return rc;
     const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks *
                           (masked ? p.groups : 1);
     const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
@@ -1731,8 +1964,8 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
       fprintf(stderr, "[dg] gemm sched=%d (UE8M0) rows=%lld n=%lld k=%lld groups=%d grid=%d\n",
               sched, static_cast<long long>(rows), static_cast<long long>(n),
               static_cast<long long>(k), p.groups, grid);
-    return masked ? dispatch<kMaskedUE8M0>(bn, ta, tb, p, grid, extra, stream)
-                  : dispatch<kDenseUE8M0>(bn, ta, tb, p, grid, extra, stream);
+    return masked ? dispatch<kMaskedUE8M0>(bn, ta, tb, td, p, grid, extra, stream)
+                  : dispatch<kDenseUE8M0>(bn, ta, tb, td, p, grid, extra, stream);
   }
   if (sched == kDenseQuant) {
     // whole 128-column groups per thread: 256-wide tiles, K never split (a
@@ -1744,14 +1977,14 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
     p.full_tiles = 0;
     p.ws = nullptr;
     p.a_box_rows = rows <= BM / 2 ? BM / 2 : BM;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, td = {};
     int rc = make_tmap(&ta, A, k, rows, 1, p.a_box_rows);
     if (rc) return rc;
     rc = make_tmap(&tb, B, k, n, 1, bn);
     if (rc) return rc;
     const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
     const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
-    return dispatch<kDenseQuant>(bn, ta, tb, p, grid, extra, stream);
+    return dispatch<kDenseQuant>(bn, ta, tb, td, p, grid, extra, stream);
   }
   // The 2-CTA form for dense NT shapes of at least two M blocks: each SM
   // loads its 128 rows of A and half of the 256-wide B tile, two thirds of
@@ -1771,11 +2004,12 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
     p.full_tiles = 0;
     p.ws = nullptr;
     p.a_box_rows = BM;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, td = {};
     int rc = make_tmap(&ta, A, k, rows, 1, BM);
     if (rc) return rc;
     rc = make_tmap(&tb, B, k, n, 1, bn / 2);
     if (rc) return rc;
+    if ((rc = make_tmap_d(&td, p.d, rows, n, 1))) return rc;
     const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
     const int grid =
         2 * static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms / 2)));
@@ -1783,13 +2017,14 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
       fprintf(stderr, "[dg] gemm sched=dense rows=%lld n=%lld k=%lld: 2-CTA BN=256 grid=%d\n",
               static_cast<long long>(rows), static_cast<long long>(n),
               static_cast<long long>(k), grid);
-    return dispatch<kDensePair>(bn, ta, tb, p, grid, extra, stream);
+    return dispatch<kDensePair>(bn, ta, tb, td, p, grid, extra, stream);
   }
   const Choice choice =
       choose_config(sched, rows, n, k, p.groups, num_sms, ws_bytes, extra, max_smem, layout);
   int bn = choice.bn, splits = choice.splits;
   int64_t full_tiles = choice.full_tiles;
   bool splits_forced = false;  // DG_SPLITS: exactly this many, or none
+  bool bn_forced = false;      // DG_BLOCK_N
   // D = C + A B^T (dense only): single-CTA tiles, splits through the
   // workspace (the FP32 tile is staged in the 32 KB the BF16 tile uses, so
   // every tile form still fits)
@@ -1798,13 +2033,20 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
   // every tile's K, DG_TAIL_SPLITS only the last partial wave's tiles (dense;
   // both need enough workspace).
   if (const char *e = getenv("DG_BLOCK_N")) {
+    // (a non-power-of-two width serves the cluster split only: NT, with
+    // DG_SPLITS of at least 2)
     const int v = atoi(e);
-    for (const Candidate &c : kCandidates)
-      if (c.bn == v && v != bn && (layout == kLayoutNT || v % 128 == 0)) {
+    bool known = false;
+    for (const Candidate &c : kCandidates) known = known || c.bn == v;
+    for (const Candidate &c : kClusterForms) known = known || (c.bn == v && layout == kLayoutNT);
+    if (known && (layout == kLayoutNT || v % 128 == 0)) {
+      if (v != bn) {
         bn = v;
         splits = 1;  // the split chosen for another width does not carry over
         full_tiles = 0;
       }
+      bn_forced = true;
+    }
   }
   if (const char *e = getenv("DG_SPLITS")) {
     // every tile split v ways (v = 1: no split)
@@ -1833,23 +2075,41 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
       full_tiles = waves * num_sms;
     }
   }
-  if (config_smem(bn, extra, sched == kDense && acc ? kDenseAcc : sched) > max_smem)
-    return DG_ERR_INVALID_ARG;  // too many experts
+  // (a non-power-of-two width exists only as the cluster split's form)
+  const int smem_sched = (bn & (bn - 1)) != 0 ? kDenseCluster
+                         : sched == kDense && acc ? kDenseAcc
+                                                  : sched;
+  if (config_smem(bn, extra, smem_sched) > max_smem) return DG_ERR_INVALID_ARG;  // too many experts
   p.num_m_blocks = static_cast<int>((rows + BM - 1) / BM);
   p.num_n_blocks = static_cast<int>((n + bn - 1) / bn);
   p.splits = splits;
   p.full_tiles = splits > 1 ? static_cast<int>(full_tiles) : 0;
-  const int64_t all_tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
+  int64_t all_tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
   p.ws = nullptr;
   if (sched != kKGrouped) p.ws_ticket = nullptr;  // (k-grouped: ld_sfb shares it)
   // Every tile split (decode-sized shapes, one wave): the splits of a tile
   // form a cluster and reduce through distributed shared memory, needing no
   // workspace or arrival counters, when all clusters fit in one wave
   // (DG_CLUSTER_SPLIT=0 forces the workspace path).
-  bool try_cluster = sched == kDense && !acc && splits > 1 && splits <= 8 &&
+  bool try_cluster = sched == kDense && !acc && splits > 1 && splits <= kMaxClusterSplits &&
                      p.full_tiles == 0 && all_tiles * splits <= num_sms;
   if (const char *e = getenv("DG_CLUSTER_SPLIT"))
     if (*e == '0') try_cluster = false;
+  // ... with the width and split the bandwidth model prefers among the
+  // cluster forms that fit one wave, non-power-of-two widths included
+  // (unless DG_BLOCK_N / DG_SPLITS force them)
+  bool picked = false;
+  if (try_cluster && layout == kLayoutNT && !bn_forced && !splits_forced) {
+    const ClusterPick cp = pick_cluster_form(rows, n, k, num_sms, max_smem);
+    if (cp.bn > 0) {
+      bn = cp.bn;
+      splits = cp.splits;
+      p.splits = splits;
+      p.num_n_blocks = static_cast<int>((n + bn - 1) / bn);
+      all_tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
+      picked = true;
+    }
+  }
   // the workspace path: FP32 partials and one arrival counter per split tile
   auto setup_workspace = [&]() -> int {
     const int64_t split_tiles = all_tiles - p.full_tiles;
@@ -1868,7 +2128,7 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
   }
 
   // ------------------------------------------------ tensor maps
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, td = {};
   p.a_box_rows = (sched == kDense && rows <= BM / 2 && !a_mn_major(layout)) ? BM / 2 : BM;
   int rc = a_mn_major(layout)
                ? make_tmap_mn(&ta, A, rows, k, 1)
@@ -1878,6 +2138,8 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
            ? make_tmap_mn(&tb, B, n, k, 1)
            : make_tmap(&tb, B, k, n, (sched == kDense || sched == kKGrouped) ? 1 : p.groups, bn);
   if (rc) return rc;
+  // the plain dense tiles store D with TMA
+  if (sched == kDense && !acc && (rc = make_tmap_d(&td, p.d, rows, n, 1))) return rc;
 
   // ------------------------------------------------ grid
   int64_t units;
@@ -1896,15 +2158,18 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
     // still keeps 3/5 of the SMs busy
     int rc = kClusterNoFit;
     const int chosen = p.splits;
-    const int lowest = splits_forced ? chosen : 2;
+    // (a picked form fits by construction: the launch asks the same cached
+    // occupancy query)
+    const int lowest = splits_forced || picked ? chosen : 2;
     for (int sc = chosen; sc >= lowest && rc == kClusterNoFit; --sc) {
       if (sc < chosen && all_tiles * sc * 5 < static_cast<int64_t>(num_sms) * 3) break;
       p.splits = sc;
       grid = static_cast<int>(all_tiles * sc);
       rc = layout == kLayoutNT
-               ? dispatch<kDenseCluster>(bn, ta, tb, p, grid, extra, stream)
-               : dispatch_any_layout<kDenseCluster>(layout, bn, ta, tb, p, grid, extra, stream);
+               ? dispatch<kDenseCluster>(bn, ta, tb, td, p, grid, extra, stream)
+               : dispatch_any_layout<kDenseCluster>(layout, bn, ta, tb, td, p, grid, extra, stream);
     }
+    if (rc == kClusterNoFit && picked) return DG_ERR_CUDA;  // (the query disagreed with itself)
     if (rc == kClusterNoFit) {
       p.splits = chosen;
       grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms)));
@@ -1932,18 +2197,18 @@ static int launch_fp8_gemm_impl(int sched, const uint8_t *A, const uint8_t *B, G
   switch (sched) {
     case kDense:
       if (layout != kLayoutNT)
-        return dispatch_any_layout<kDense>(layout, bn, ta, tb, p, grid, extra, stream);
-      return acc ? dispatch<kDenseAcc>(bn, ta, tb, p, grid, extra, stream)
-                 : dispatch<kDense>(bn, ta, tb, p, grid, extra, stream);
-    case kContiguous: return dispatch<kContiguous>(bn, ta, tb, p, grid, extra, stream);
-    case kMasked: return dispatch<kMasked>(bn, ta, tb, p, grid, extra, stream);
+        return dispatch_any_layout<kDense>(layout, bn, ta, tb, td, p, grid, extra, stream);
+      return acc ? dispatch<kDenseAcc>(bn, ta, tb, td, p, grid, extra, stream)
+                 : dispatch<kDense>(bn, ta, tb, td, p, grid, extra, stream);
+    case kContiguous: return dispatch<kContiguous>(bn, ta, tb, td, p, grid, extra, stream);
+    case kMasked: return dispatch<kMasked>(bn, ta, tb, td, p, grid, extra, stream);
     case kKGrouped:
       // the k-grouped form's transposed variant is TN (both operands stored
       // with the token axis K outermost)
       if (layout == kLayoutTN)
-        return dispatch_layout<kKGrouped, kLayoutTN>(bn, ta, tb, p, grid, extra, stream);
+        return dispatch_layout<kKGrouped, kLayoutTN>(bn, ta, tb, td, p, grid, extra, stream);
       if (layout != kLayoutNT) return DG_ERR_INVALID_ARG;
-      return dispatch<kKGrouped>(bn, ta, tb, p, grid, extra, stream);
+      return dispatch<kKGrouped>(bn, ta, tb, td, p, grid, extra, stream);
     default: return DG_ERR_INVALID_ARG;
   }
 }

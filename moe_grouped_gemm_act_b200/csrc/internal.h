@@ -126,6 +126,8 @@ struct GemmParams {
                          // the remaining ones, each split `splits` ways
   int a_box_rows;        // rows of A per TMA load: 128, or 64 when M <= 64
   int q_flags;           // quantizing epilogue: DG_SCALE_FP32 or DG_SCALE_POW2
+  int starve_it;         // test hook: the K-block iteration whose loads CTA 0's
+                         // producer leaves out (-1: none; set by launch_fp8_gemm)
 };
 
 struct GemmConfig {

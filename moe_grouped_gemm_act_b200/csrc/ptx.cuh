@@ -26,6 +26,16 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // test that starves a wait on purpose, so that the wait runs out quickly.
 static __device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 
+// Waits shorter than this never read g_wait_limit_ns, so that the limit's
+// global load (cold in every cache at a kernel's start) stays off the path of
+// ordinary waits; a lowered limit is therefore never below it.
+constexpr uint64_t kWaitCheckNs = 1000000ull;
+
+// Whether a wait that has run for `elapsed` ns is past the limit.
+__device__ __forceinline__ bool wait_expired(uint64_t elapsed) {
+  return elapsed > kWaitCheckNs && elapsed > g_wait_limit_ns;
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -94,7 +104,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > g_wait_limit_ns) {
+    if (wait_expired(globaltimer() - t0)) {
       record_status(status, DG_ERR_TIMEOUT);
       *abort = 1;
       return false;
@@ -116,7 +126,7 @@ __device__ __forceinline__ bool wait_counter(const uint32_t *counter, uint32_t t
   const uint64_t t0 = globaltimer();
   while (ld_acquire_gpu(counter) < target) {
     __nanosleep(64);
-    if (globaltimer() - t0 > g_wait_limit_ns) {
+    if (wait_expired(globaltimer() - t0)) {
       record_status(status, DG_ERR_TIMEOUT);
       return false;
     }
@@ -139,6 +149,47 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap,
       "bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+// tma_load_3d for the CTA pair of a cta_group::2 MMA: the box lands in this
+// CTA's shared memory and its bytes complete on the mbarrier at the
+// cluster-window address `bar` (the even CTA's, which counts both CTAs'
+// bytes).  No multicast.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void *tmap, uint32_t bar,
+                                                 int32_t c0, int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::"
+      "bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// 3-D tiled TMA store of a shared-memory box to global memory (the box's
+// part outside the tensor is not written), tracked by this thread's bulk
+// async-group.  Coordinates as for tma_load_3d; none negative.
+__device__ __forceinline__ void tma_store_3d(const void *tmap, uint32_t src, int32_t c0,
+                                             int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          tmap),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Closes this thread's current bulk async-group.
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until every committed bulk group of this thread has finished reading
+// its shared-memory source (the source may then be overwritten).
+__device__ __forceinline__ void bulk_wait_group_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Waits until every committed bulk group of this thread has completed.
+__device__ __forceinline__ void bulk_wait_group_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // 1-D bulk copy global -> shared, completing on mbarrier `bar`.  Both
@@ -166,6 +217,15 @@ __device__ __forceinline__ void grid_dependency_wait() {
 
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Asks for the box of a 3-D tensor map at the given coordinates (as for
+// tma_load_3d) to be brought into L2: no destination, nothing to wait for.
+__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int32_t c0, int32_t c1,
+                                                int32_t c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tmap),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 // Asks for `bytes` of global memory at `src` to be brought into L2 (no
@@ -436,7 +496,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait_acquire_cluster(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > g_wait_limit_ns) {
+    if (wait_expired(globaltimer() - t0)) {
       record_status(status, DG_ERR_TIMEOUT);
       *abort = 1;
       return false;

@@ -96,7 +96,7 @@ def test_per_shape_report_fractions():
     rows = bench.per_shape_report(data, [0.5, 2.0], "tensor", 1000.0)
     assert rows[0]["tflops"] == pytest.approx(2 * 128 * 256 * 1024 / 0.5e-3 / 1e12)
     assert rows[1]["frac"] == pytest.approx(rows[1]["tflops"] / 1000.0)
-    assert rows[0]["gemm_us"] == pytest.approx(500.0)
+    assert rows[0]["gemm_us_alone"] == pytest.approx(500.0)
     hb = bench.per_shape_report(data, [0.5, 2.0], "hbm", 6000.0)
     want = 128 * 1024 + 4 * 128 * 8 + 256 * 1024 + 4 * 2 * 8 + 2 * 128 * 256
     assert hb[0]["gbs"] == pytest.approx(want / 0.5e-3 / 1e9)

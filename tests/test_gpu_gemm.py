@@ -61,6 +61,27 @@ def test_dense_ragged_every_block_n(bn, m, n, k):
     check_gemm(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"{m}x{n}x{k} BN={bn}")
 
 
+@pytest.mark.parametrize("bn,pair", [(256, 0), (128, 0), (256, 1)])
+@pytest.mark.parametrize("m,n", [(200, 400), (130, 136), (1, 520), (64, 7168), (385, 2112)])
+def test_dense_stores_stay_inside_d(m, n, bn, pair):
+    # D sits inside a larger buffer of sentinels: the epilogue's TMA stores
+    # (boxes of 128 rows x 64 columns, clipped at D's last row and column)
+    # must leave every element around it as it was, and D must be right
+    k = 512
+    qa, alpha, qb, beta = dense_case(m, n, k, seed=3 * m + n)
+    pad = 4096  # elements on each side (keeps D 16-byte aligned)
+    buf = torch.full((pad + m * n + pad,), SENTINEL, dtype=torch.int16, device="cuda")
+    d = buf[pad:pad + m * n].view(m, n).view(torch.bfloat16)
+    with env(DG_BLOCK_N=bn, DG_PAIR=pair, DG_SPLITS=1):
+        dg.dg_fp8_gemm_nt(dev(qa), sfa_to_device(alpha), dev(qb), dev(beta), d)
+        torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    host = buf.cpu().numpy()
+    assert np.all(host[:pad] == SENTINEL) and np.all(host[pad + m * n:] == SENTINEL)
+    got = host[pad:pad + m * n].reshape(m, n).view(np.uint16)
+    check_gemm(got, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"{m}x{n} BN={bn} pair={pair}")
+
+
 @pytest.mark.parametrize("pair", [0, 1])
 @pytest.mark.parametrize("m,n,k", [(300, 392, 1024), (1000, 2112, 384), (513, 256, 256),
                                    (256, 4096, 2048), (2048, 7168, 1536)])
@@ -121,6 +142,22 @@ def test_dense_split_k(splits, bn):
     check_gemm(a, want, f"split {splits}")
     assert np.array_equal(a, b), "split-K result not deterministic"
     assert np.array_equal(a, c), "cluster and workspace reductions differ"
+
+
+@pytest.mark.parametrize("bn", [224, 192, 160, 96])
+@pytest.mark.parametrize("m,n,k,splits", [(64, 2112, 2048, 4), (128, 1000, 1536, 3),
+                                          (1, 736, 1024, 2), (200, 2048, 2048, 2)])
+def test_cluster_split_non_power_of_two_widths(bn, m, n, k, splits):
+    # tiles whose width is not a power of two (the cluster split of decode
+    # shapes): a promotion thread's columns may span two 128-column blocks of
+    # B's scales, each with its own beta; ragged N and M, every split summed
+    # in order (deterministic)
+    qa, alpha, qb, beta = dense_case(m, n, k, seed=bn + m + n)
+    with env(DG_BLOCK_N=bn, DG_SPLITS=splits, DG_CLUSTER_SPLIT=1):
+        a = run_dense(qa, alpha, qb, beta, workspace=True)
+        b = run_dense(qa, alpha, qb, beta, workspace=True)
+    check_gemm(a, gemm.fp8_gemm_nt_f64(qa, alpha, qb, beta), f"{m}x{n}x{k} BN={bn} S={splits}")
+    assert np.array_equal(a, b), "cluster split not deterministic"
 
 
 def test_dense_split_k_cluster_ragged_rows():
