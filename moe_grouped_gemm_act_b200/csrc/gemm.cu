@@ -82,14 +82,15 @@ constexpr int kThreads = 32 * (kControlWarps + kPromoWarps);
 // gives up most of them so that each promotion thread can hold its 128
 // accumulators and a 64-column TMEM chunk.  Either split uses exactly the
 // launch allocation (40 x 128 + 232 x 256 = 56 x 128 + 224 x 256 = 168 x 384);
-// per schedule, the one with which ptxas spills least.
+// per schedule, the one with which ptxas spills least (the 2-CTA form:
+// 80 / 124 bytes of spill stores / loads with 40 / 232, 20 / 48 with 56 / 224,
+// 96 / 128 with fewer promotion registers; 28 % faster with 56 / 224).
 constexpr int kLaunchRegs = 168;
-__host__ __device__ constexpr int ctrl_regs(int sched) {
-  return (sched == kMasked || sched == kDenseCluster || is_ue8m0(sched)) ? 56 : 40;
+__host__ __device__ constexpr bool wide_control(int sched) {
+  return sched == kMasked || sched == kDenseCluster || is_ue8m0(sched) || sched == kDensePair;
 }
-__host__ __device__ constexpr int promo_regs(int sched) {
-  return (sched == kMasked || sched == kDenseCluster || is_ue8m0(sched)) ? 224 : 232;
-}
+__host__ __device__ constexpr int ctrl_regs(int sched) { return wide_control(sched) ? 56 : 40; }
+__host__ __device__ constexpr int promo_regs(int sched) { return wide_control(sched) ? 224 : 232; }
 static_assert(ctrl_regs(kDense) * 32 * kControlWarps + promo_regs(kDense) * kPromoThreads <=
                   kLaunchRegs * kThreads,
               "register split exceeds the launch allocation");
