@@ -64,12 +64,17 @@ FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 # the GEMM code it was taken on (gemm_source_hash, stored beside it); on a
 # mismatch the bench reports null.
 GEMM_TRAFFIC = {
-    "prefill": ("3e97d80689d725cc", 210.8e6),
-    "prefill_acc": ("05d65bb9d3528fd6", 405.3e6),
-    "decode64": ("05d65bb9d3528fd6", 51.3e6),
-    "decode128": ("05d65bb9d3528fd6", 52.0e6),
-    "masked": ("05d65bb9d3528fd6", 533.6e6),
-    "contiguous": ("05d65bb9d3528fd6", 978.3e6),
+    "prefill": ("201f9c6ffc869866", 210.4e6),
+    "decode64": ("201f9c6ffc869866", 50.5e6),
+    "decode128": ("201f9c6ffc869866", 51.1e6),
+    "contiguous": ("201f9c6ffc869866", 971.0e6),
+    "masked": ("201f9c6ffc869866", 531.5e6),
+    "masked_pow2": ("201f9c6ffc869866", 531.5e6),
+    "masked_ue8m0": ("201f9c6ffc869866", 535.0e6),
+    "kgrouped": ("201f9c6ffc869866", 1431.5e6),
+    "kgrouped_tn": ("201f9c6ffc869866", 1413.9e6),
+    "prefill_acc": ("201f9c6ffc869866", 403.2e6),
+    "prefill_quant": ("201f9c6ffc869866", 220.4e6),
 }
 
 
