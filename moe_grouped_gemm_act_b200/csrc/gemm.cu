@@ -151,8 +151,8 @@ struct Layout {
   static constexpr uint32_t kOutOff = STAGES * kStageBytes;
   static constexpr uint32_t kRowOkOff = kOutOff + (STAGED ? BM * kOutCols * kOutElem : 0);
   static constexpr uint32_t kBarOff = kRowOkOff + (STAGED ? BM : 0);
-  // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain epi
-  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 2;
+  // full[S] empty[S] tfull[NBUF] tempty[NBUF] drain epi staged free
+  static constexpr uint32_t kNumBars = 2 * STAGES + 2 * NBUF + 4;
   static constexpr uint32_t kMiscOff = kBarOff + 8 * kNumBars;
   static constexpr uint32_t kPrefixOff = kMiscOff + 16;
   // k-grouped: a ring of per-column B scale slices, one per K block in
@@ -326,6 +326,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // masked instance keeps its row stores: with both paths in it, ptxas
   // spills and it ran 25 % slower.)
   constexpr bool kTmaStore = (S == kDense || (S == kMasked && kUE)) && kStaged == 1 && BN >= 128;
+  // dense TMA-stored tiles hand the stores to warp 2: the promotion warps
+  // write their columns into the staging tile and go on to the next tile;
+  // warp 2 issues each staging use's TMA store and frees the tile once the
+  // store has read it.  Warps writing one staging use: the half that owns it
+  // (256 wide: two uses per tile) or both halves (128 wide: one use).
+  constexpr bool kStoreWarp = kTmaStore && S == kDense && !kUE && !kPair;
+  constexpr int kStoreUses = BN > 128 ? 2 : 1;
+  constexpr int kStoreWriters = kStoreUses == 2 ? kPromoWarps / 2 : kPromoWarps;
   static_assert(!kPair || (BN == 256 && LAYOUT == kLayoutNT), "the 2-CTA form: NT, 256 wide");
   using L = Layout<BN, STAGES, NBUF, kStaged, kKG, kUE, kPair>;
   constexpr int W = BN / 2;                 // columns per promotion thread
@@ -367,6 +375,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // synchronises the promotion threads in the epilogue (bounded, unlike a
   // named barrier, so that an aborting warp cannot strand the others)
   const uint32_t epi_bar = drain_bar + 8u;
+  // TMA-stored tiles: a staging use has been written (by its writer warps),
+  // and a use's TMA store has finished reading the staging tile
+  const uint32_t staged_bar = epi_bar + 8u;
+  const uint32_t free_bar = epi_bar + 16u;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   int *s_flag = reinterpret_cast<int *>(smem + L::kMiscOff + 8);
@@ -422,6 +434,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     mbar_init(drain_bar, 1);
     mbar_init(epi_bar, kPromoWarps);
+    mbar_init(staged_bar, kStoreWriters);
+    mbar_init(free_bar, 1);
     *s_abort = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -767,6 +781,40 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       volatile int never = 0;
       mbar_wait(drain_bar, 0, &never, p.status);
     }
+  } else if (kStoreWarp && warp == 2) {
+    // ============================================================ D stores
+    // For each staging use (in the promotion warps' order: the whole tiles,
+    // then their column halves), wait until its writers have staged it,
+    // store it by TMA, and free the staging tile once the store has read it.
+    // Split tiles (reduced through the workspace) stage nothing.
+    uint32_t use = 0;
+    bool alive = true;
+    for (int u = u_first; u < units && alive; u += u_stride) {
+      const Tile t = unit_to_tile(p, S, u, s_prefix, s_mblocks);
+      if (t.nsplit > 1) continue;
+      for (int ph = 0; ph < kStoreUses; ++ph, ++use) {
+        if (!mbar_wait(staged_bar, use & 1, s_abort, p.status)) {
+          alive = false;
+          break;
+        }
+        if (lane == 0) {
+          const int col_base = t.n_blk * BN + ph * 128;
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            if (col_base + j * static_cast<int>(kStoreBoxCols) < p.n)
+              tma_store_3d(&tmap_d, base + L::kOutOff + j * (BM * 128u),
+                           col_base + j * kStoreBoxCols,
+                           t.m_blk * TM + static_cast<int>(rank) * BM, t.slab);
+          bulk_commit_group();
+          bulk_wait_group_read_all();  // the staging tile may be written again
+          mbar_arrive(free_bar);
+        }
+        __syncwarp();
+      }
+    }
+    // the stores of D have completed before the CTA exits
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
   } else {
     if constexpr (kRegSplit) setmaxnreg_inc<promo_regs(SCHED)>();
@@ -785,6 +833,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     // the phase (bounded); the warp agrees on the outcome so that it stays
     // converged for the next sync
     uint32_t epi_phase = 0;
+    uint32_t store_use = 0;  // staging uses so far (tiles stored by warp 2)
     auto epi_sync = [&]() -> bool {
       __syncwarp();
       if (lane == 0) mbar_arrive(epi_bar);
@@ -1221,6 +1270,41 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int ptid = threadIdx.x - kControlWarps * 32;
         const int64_t slab_row0 = static_cast<int64_t>(t.slab) * p.rows + t.m_blk * TM +
                                   static_cast<int>(rank) * BM;
+        if constexpr (kStoreWarp) {
+          // This warp's staging use: wait until the previous use's TMA
+          // store has read the staging tile, write the columns, make them
+          // visible to the async proxy and hand the use to warp 2.
+#pragma unroll
+          for (int ph = 0; ph < kStoreUses; ++ph) {
+            if (kStoreUses == 1 || half == ph) {
+              const uint32_t use = store_use + static_cast<uint32_t>(ph);
+              bool ok = use == 0 || mbar_wait(free_bar, (use - 1) & 1, s_abort, p.status);
+              if (!__all_sync(0xffffffffu, ok)) {
+                alive = false;
+                break;
+              }
+              const int scol0 = kStoreUses == 1 ? half * W : 0;  // staged column of acc[0]
+#pragma unroll
+              for (int c = 0; c < W; c += 8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const __nv_bfloat162 h =
+                      __floats2bfloat162_rn(acc[c + 2 * j], acc[c + 2 * j + 1]);
+                  w[j] = *reinterpret_cast<const uint32_t *>(&h);
+                }
+                st_shared_v4(s_out + staged_off(row_in_tile, (scol0 + c) / 8), w[0], w[1], w[2],
+                             w[3]);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(staged_bar);
+            }
+          }
+          store_use += kStoreUses;
+          if (!alive) break;
+          continue;
+        }
         const bool tma_tile =
             kTmaStore && (S == kDense || (t.m_blk + 1) * BM <= masked_rows(p, t.slab));
         if (!tma_tile && half == 0) s_rowok[row_in_tile] = row_ok ? 1 : 0;
