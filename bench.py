@@ -75,6 +75,7 @@ GEMM_TRAFFIC = {
     "kgrouped_tn": ("87efc2d0418d62a9", 1418.4e6),
     "prefill_acc": ("87efc2d0418d62a9", 403.6e6),
     "prefill_quant": ("87efc2d0418d62a9", 220.4e6),
+    "prefill_ue8m0": ("87efc2d0418d62a9", 218.9e6),
 }
 
 
@@ -168,6 +169,12 @@ def workload_spec(name: str) -> dict:
                     desc="m-grouped masked, G=32, M_max=256, N=7168 K=2048, "
                          "masked_m ~ U{0..256}, power-of-two scales as packed UE8M0 words "
                          "applied by the tensor cores (block-scaled MMA)")
+    if name == "prefill_ue8m0":
+        return dict(name=name, kind="dense", m=inputs.PREFILL_M, nk=inputs.PREFILL_NK,
+                    seeds=inputs.PREFILL_SEEDS, bound="tensor", pow2=True, ue8m0=True,
+                    desc="dense NT prefill with power-of-two scales as packed UE8M0 words "
+                         "applied by the tensor cores (block-scaled MMA), M=4096, (N,K) in "
+                         "{(7168,16384),(4096,7168),(24576,1536),(2112,7168)}; A, B as prefill")
     if name == "prefill_quant":
         # the prefill shapes whose N is a whole number of 128-wide groups (an
         # output quantized 1x128 is the next GEMM's A, whose K must be)
@@ -284,13 +291,17 @@ class DenseData:
         self.m = m
         self.acc = bool(spec.get("acc"))
         self.quant_out = bool(spec.get("quant_out"))
+        # UE8M0: power-of-two scales packed for the block-scaled MMA (B's once,
+        # A's every step after the quantizer)
+        self.ue8m0 = bool(spec.get("ue8m0"))
+        self.pow2 = bool(spec.get("pow2"))
         self.shapes = []
         gen = torch.Generator(device=device)
         for n, k in spec["nk"]:
             x = inputs.activations(m, k, seed=spec["seeds"]["seed_a"] + k, outliers=True)
             w = inputs.weights((n, k), seed=spec["seeds"]["seed_b"] + n + k)
             a32 = torch.from_numpy(x).to(device)
-            qb, sfb = dg.dg_quantize_128x128(torch.from_numpy(w).to(device))
+            qb, sfb = dg.dg_quantize_128x128(torch.from_numpy(w).to(device), pow2=self.pow2)
             ld = dg.dg_get_tma_aligned_size(m, 4)
             qa = torch.empty((m, k), dtype=torch.uint8, device=device)
             sfa = torch.empty((k // 128, ld), dtype=torch.float32, device=device)
@@ -305,8 +316,10 @@ class DenseData:
             if self.acc:  # D = C + A B^T: a seeded FP32 C per shape
                 gen.manual_seed(spec["seeds"]["seed_a"] + 7 * k + n)
                 c = torch.randn((m, n), generator=gen, device=device, dtype=torch.float32) * 4
+            pb = dg.dg_pack_ue8m0_128x128(sfb, n) if self.ue8m0 else None
+            pa = dg.dg_pack_ue8m0(sfa.zero_(), m) if self.ue8m0 else None
             self.shapes.append(dict(n=n, k=k, a32=a32, qb=qb, sfb=sfb, qa=qa, sfa=sfa, d=d,
-                                    ws=ws, x_host=x, w_host=w, c=c))
+                                    ws=ws, x_host=x, w_host=w, c=c, pa=pa, pb=pb))
         torch.cuda.synchronize()
 
     def flops(self) -> float:
@@ -318,6 +331,10 @@ class DenseData:
         n, k = s["n"], s["k"]
         out = (self.m * n + 4 * self.m * (n // 128)) if getattr(self, "quant_out", False) \
             else 2 * self.m * n
+        if getattr(self, "ue8m0", False):
+            # packed words: 4 K groups per int32, per row of A and of B
+            words = -(-(k // 128) // 4)
+            return self.m * k + 4 * self.m * words + n * k + 4 * n * words + out
         tot = self.m * k + 4 * self.m * (k // 128) + n * k + \
             4 * (-(-n // 128)) * (k // 128) + out
         if self.acc:
@@ -329,7 +346,9 @@ class DenseData:
         return sum(self.shape_bytes(s) for s in self.shapes)
 
     def gemm(self, s):
-        if self.quant_out:
+        if self.ue8m0:
+            self.dg.dg_fp8_gemm_nt_ue8m0(s["qa"], s["pa"], s["qb"], s["pb"], s["d"])
+        elif self.quant_out:
             self.dg.dg_fp8_gemm_nt_quantize(s["qa"], s["sfa"], s["qb"], s["sfb"], dq=s["d"][0],
                                             sfd=s["d"][1])
         elif self.acc:
@@ -342,7 +361,9 @@ class DenseData:
     def step(self):
         """One pass of the hot path: for every shape, quantize A, then GEMM."""
         for s in self.shapes:
-            self.dg.dg_quantize_1x128(s["a32"], q=s["qa"], sf=s["sfa"])
+            self.dg.dg_quantize_1x128(s["a32"], pow2=self.pow2, q=s["qa"], sf=s["sfa"])
+            if self.ue8m0:
+                self.dg.dg_pack_ue8m0(s["sfa"], self.m, packed=s["pa"])
             self.gemm(s)
 
     def capture(self):
@@ -375,8 +396,9 @@ class DenseData:
 
     def launches_per_step(self) -> int:
         # this library's kernels per step: one quantizer and one GEMM per
-        # shape (a split-K call also enqueues a runtime memset, not counted)
-        return 2 * len(self.shapes)
+        # shape, plus the UE8M0 form's scale packing (a split-K call also
+        # enqueues a runtime memset, not counted)
+        return (3 if self.ue8m0 else 2) * len(self.shapes)
 
     def input_bytes(self) -> float:
         """Bytes of inputs a step streams (FP32 activations and FP8 B)."""
@@ -405,7 +427,13 @@ class DenseData:
             a = h["a"].to(device, non_blocking=True)
             qb = h["qb"].to(device, non_blocking=True)
             sfb = h["sfb"].to(device, non_blocking=True)
-            qa, sfa = dg.dg_quantize_1x128(a)
+            qa, sfa = dg.dg_quantize_1x128(a, pow2=self.pow2)
+            if self.ue8m0:
+                pa = dg.dg_pack_ue8m0(sfa, qa.shape[0])
+                pb = dg.dg_pack_ue8m0_128x128(sfb, qb.shape[0])
+                dg.dg_fp8_gemm_nt_ue8m0(qa, pa, qb, pb, s["d"])
+                h["d"].copy_(s["d"], non_blocking=True)
+                continue
             if self.quant_out:
                 dg.dg_fp8_gemm_nt_quantize(qa, sfa, qb, sfb, dq=s["d"][0], sfd=s["d"][1])
                 for dst, src in zip(h["d"], s["d"]):
@@ -671,18 +699,20 @@ class OracleSample:
         self.prepared = []
         self.acc = bool(spec.get("acc"))
         self.quant_out = bool(spec.get("quant_out"))
+        self.pow2 = bool(spec.get("pow2"))
         g = np.random.default_rng(spec["seeds"]["seed_a"])
         for n, k in spec["nk"]:
             x = inputs.activations(spec["m"], k, seed=spec["seeds"]["seed_a"] + k,
                                    outliers=True)
             w = inputs.weights((n, k), seed=spec["seeds"]["seed_b"] + n + k)
             c = min(n, cols)
-            qb, beta = oq.quantize_128x128(w[:c])
+            qb, beta = oq.quantize_128x128(w[:c], pow2=self.pow2)
             cs = (g.standard_normal((rows, c)) * 4).astype(np.float32) if self.acc else None
             self.prepared.append((x[:rows].copy(), qb, beta, c, k, cs))
         self.desc = (f"{rows} rows of A x first {cols} columns of D per (N,K) pair, "
                      f"full K" + (", D = C + A B^T" if self.acc else "") +
-                     (", D quantized 1x128" if self.quant_out else ""))
+                     (", D quantized 1x128" if self.quant_out else "") +
+                     (", power-of-two scales" if self.pow2 else ""))
 
     def run(self) -> tuple[float, float]:
         """Returns (seconds, FLOPs) of one pass."""
@@ -690,7 +720,7 @@ class OracleSample:
         t0 = time.perf_counter()
         flops = 0.0
         for xs, qb, beta, c, k, cs in self.prepared:
-            qa, alpha = oq.quantize_1x128(xs)
+            qa, alpha = oq.quantize_1x128(xs, pow2=self.pow2)
             if self.quant_out:
                 from oracle import bf16 as ob
                 d = ob.from_bits(og.fp8_gemm_nt(qa, alpha, qb, beta)).astype(np.float32)
@@ -904,7 +934,8 @@ def job_throughput(work_per_step: float, steps: int, world: int, ms: float) -> f
 
 
 ALL_WORKLOADS = ["prefill", "decode64", "decode128", "contiguous", "masked", "masked_pow2",
-                 "masked_ue8m0", "kgrouped", "kgrouped_tn", "prefill_acc", "prefill_quant"]
+                 "masked_ue8m0", "kgrouped", "kgrouped_tn", "prefill_acc", "prefill_quant",
+                 "prefill_ue8m0"]
 
 
 def measure_workload(name: str, args, rank: int, world: int, device, cpu_secs: float) -> dict:
