@@ -120,9 +120,11 @@ __host__ __device__ constexpr int staged_epilogue(int sched) {
 }
 
 // The staging kind an instance uses (every schedule, including the UE8M0
-// and quantizing forms).
+// and quantizing forms): the UE8M0 forms stage the BF16 tile 64 columns at a
+// time (kind 3), which leaves room for a fourth stage beside their per-stage
+// scale-factor areas.
 __host__ __device__ constexpr int instance_staging(int sched) {
-  return sched == kDenseQuant ? 0 : staged_epilogue(base_sched(sched));
+  return sched == kDenseQuant ? 0 : is_ue8m0(sched) ? 3 : staged_epilogue(base_sched(sched));
 }
 
 // Scale-factor bytes per stage of the UE8M0 schedules: the K block's packed
@@ -146,7 +148,7 @@ struct Layout {
   // FP32 (kind 2: 64-column phases), then one byte per row saying whether it
   // is stored
   static constexpr uint32_t kOutCols =
-      STAGED == 2 ? (BN < 64 ? BN : 64) : (BN < 128 ? BN : 128);
+      STAGED >= 2 ? (BN < 64 ? BN : 64) : (BN < 128 ? BN : 128);
   static constexpr uint32_t kOutElem = STAGED == 2 ? 4 : 2;
   static constexpr uint32_t kOutOff = STAGES * kStageBytes;
   static constexpr uint32_t kRowOkOff = kOutOff + (STAGED ? BM * kOutCols * kOutElem : 0);
@@ -325,7 +327,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   // map), UE8M0 masked tiles whose 128 rows are all valid.  (The FP32-scale
   // masked instance keeps its row stores: with both paths in it, ptxas
   // spills and it ran 25 % slower.)
-  constexpr bool kTmaStore = (S == kDense || (S == kMasked && kUE)) && kStaged == 1 && BN >= 128;
+  constexpr bool kTmaStore =
+      (S == kDense || (S == kMasked && kUE)) && (kStaged == 1 || kStaged == 3) && BN >= 128;
   // dense TMA-stored tiles hand the stores to warp 2: the promotion warps
   // write their columns into the staging tile and go on to the next tile;
   // warp 2 issues each staging use's TMA store and frees the tile once the
@@ -1259,7 +1262,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         // only.
         constexpr int kChunks = L::kOutCols / 8;        // 16-byte chunks per staged row
         constexpr int kSw = kChunks < 8 ? kChunks : 8;  // swizzle span, in chunks
-        constexpr int kPhases = BN > 128 ? 2 : 1;
+        // phases of kOutCols columns: one (a 128-wide or narrower tile), one
+        // per column half (256 wide, 128-column staging), or two per half
+        // (256 wide, 64-column staging: the UE8M0 forms)
+        constexpr int kPhases = BN > static_cast<int>(L::kOutCols) ? BN / L::kOutCols : 1;
+        constexpr int kPhasesPerHalf = kPhases > 1 ? kPhases / 2 : 1;
         constexpr int kRowBytes = kChunks < 8 ? L::kOutCols * 2 : 128;
         auto staged_off = [&](int r, int c) -> uint32_t {
           return static_cast<uint32_t>((c / kSw) * (BM * kRowBytes) + r * kRowBytes +
@@ -1310,18 +1317,23 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (!tma_tile && half == 0) s_rowok[row_in_tile] = row_ok ? 1 : 0;
 #pragma unroll
         for (int ph = 0; ph < kPhases; ++ph) {
-          if (kPhases == 1 || half == ph) {
-            const int scol0 = kPhases == 1 ? half * W : 0;  // staged column of acc[0]
+          // the phase's columns belong to half ph / kPhasesPerHalf, slice
+          // ph % kPhasesPerHalf of each of its threads' W columns
+          if (kPhases == 1 || half == ph / kPhasesPerHalf) {
+            const int sub = kPhases == 1 ? 0 : ph % kPhasesPerHalf;
 #pragma unroll
             for (int c = 0; c < W; c += 8) {
+              if (kPhases > 1 && c / static_cast<int>(L::kOutCols) != sub) continue;
               uint32_t w[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const __nv_bfloat162 h = __floats2bfloat162_rn(acc[c + 2 * j], acc[c + 2 * j + 1]);
                 w[j] = *reinterpret_cast<const uint32_t *>(&h);
               }
-              st_shared_v4(s_out + staged_off(row_in_tile, (scol0 + c) / 8), w[0], w[1], w[2],
-                           w[3]);
+              // staged column of acc[c]: the thread's own (one phase) or its
+              // place in the phase's kOutCols
+              const int scol = kPhases == 1 ? half * W + c : c % static_cast<int>(L::kOutCols);
+              st_shared_v4(s_out + staged_off(row_in_tile, scol / 8), w[0], w[1], w[2], w[3]);
             }
             // the TMA store reads the tile through the async proxy
             if constexpr (kTmaStore) fence_proxy_async_smem();
@@ -1330,11 +1342,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             alive = false;
             break;
           }
-          const int col_base = t.n_blk * BN + ph * 128;
+          const int col_base = t.n_blk * BN + ph * static_cast<int>(L::kOutCols);
           if (tma_tile) {
             if (ptid == 0) {
 #pragma unroll
-              for (int j = 0; j < kChunks / 8; ++j)
+              for (int j = 0; j < (kChunks + 7) / 8; ++j)
                 if (col_base + j * static_cast<int>(kStoreBoxCols) < p.n)
                   tma_store_3d(&tmap_d, s_out + j * (BM * 128u), col_base + j * kStoreBoxCols,
                                t.m_blk * TM + static_cast<int>(rank) * BM, t.slab);
@@ -1455,9 +1467,9 @@ constexpr Candidate kClusterForms[] = {{256, 4, 2}, {224, 5, 2}, {192, 5, 2}, {1
 constexpr bool kPairByDefault = false;
 
 // The UE8M0 schedules' one tile form: 256 wide, one accumulator (the tile
-// sums all of K in TMEM), three stages (the fourth does not fit beside the
-// per-stage scale-factor areas and the output staging).
-constexpr Candidate kUECandidate = {256, 3, 1};
+// sums all of K in TMEM), four stages (beside the per-stage scale-factor
+// areas and a 64-column output staging tile).
+constexpr Candidate kUECandidate = {256, 4, 1};
 
 template <int BN, int STAGES, int NBUF, int STAGED, bool KG = false, bool UE = false,
           bool PAIR = false>
@@ -1658,9 +1670,9 @@ int single_smem(int sched, int extra) {
 
 int config_smem(int bn, int extra, int sched) {
   if (is_ue8m0(sched))
-    // (both UE8M0 schedules stage the BF16 tile: kind 1)
+    // (both UE8M0 schedules stage the BF16 tile 64 columns at a time: kind 3)
     return smem_bytes_for<kUECandidate.bn, kUECandidate.stages, kUECandidate.nbuf,
-                          staged_epilogue(kDense), false, true>(extra);
+                          instance_staging(kDenseUE8M0), false, true>(extra);
   switch (bn) {
     case 256: return single_smem<256, 4, 2>(sched, extra);
     case 128: return single_smem<128, 6, 4>(sched, extra);
