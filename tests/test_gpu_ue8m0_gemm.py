@@ -112,6 +112,33 @@ def test_pow2_quantized_inputs_match_the_oracle(m, n, k):
     assert torch.equal(d.view(torch.int16), d3.view(torch.int16))
 
 
+@pytest.mark.parametrize("m,n", [(200, 392), (1, 520), (130, 2112)])
+def test_stores_stay_inside_d(m, n):
+    # D sits inside a buffer of sentinels: the epilogue's TMA stores (boxes of
+    # 128 rows x 64 columns, one per 64-column phase, clipped at D's last row
+    # and column) leave every element around it as it was
+    k = 512
+    x = inputs.activations(m, k, seed=5 * m + n, outliers=True)
+    w = inputs.weights((n, k), seed=5 * m + n + 1)
+    qa_d, sfa_d = dg.dg_quantize_1x128(torch.from_numpy(x).cuda(), pow2=True)
+    qb_d, sfb_d = dg.dg_quantize_128x128(torch.from_numpy(w).cuda(), pow2=True)
+    pa = dg.dg_pack_ue8m0(sfa_d, m)
+    pb = dg.dg_pack_ue8m0_128x128(sfb_d, n)
+    pad = 4096  # elements on each side (keeps D 16-byte aligned)
+    buf = torch.full((pad + m * n + pad,), SENTINEL, dtype=torch.int16, device="cuda")
+    d = buf[pad:pad + m * n].view(m, n).view(torch.bfloat16)
+    dg.dg_fp8_gemm_nt_ue8m0(qa_d, pa, qb_d, pb, d)
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    host = buf.cpu().numpy()
+    assert np.all(host[:pad] == SENTINEL) and np.all(host[pad + m * n:] == SENTINEL)
+    qa, alpha = quant.quantize_1x128(x, pow2=True)
+    qb, beta = quant.quantize_128x128(w, pow2=True)
+    want = gemm.fp8_gemm_nt_ue8m0_f64(qa, ue8m0.pack_1x128(alpha), qb,
+                                      ue8m0.pack_1x128(block_rows(beta, n)))
+    check_gemm(host[pad:pad + m * n].reshape(m, n).view(np.uint16), want, f"UE8M0 {m}x{n}")
+
+
 def test_pack_128x128_grouped_bit_exact_and_rejects_non_powers_of_two():
     rng = np.random.default_rng(4)
     G, n, kg = 3, 300, 9
